@@ -1,0 +1,17 @@
+"""Exact IO-aware attention for NVIDIA B200 (sm_100a).
+
+The compute lives in ``libattn_b200.so`` (hand-written CUDA behind a C ABI, see
+``include/attn.h``); ``binding`` marshals torch tensors into that ABI.  The
+library is loaded lazily on first use, so host-side helpers such as
+``accounting`` import without a GPU.
+"""
+from .binding import (  # noqa: F401
+    AttnError,
+    attn_bwd,
+    attn_bwd_workspace_size,
+    attn_fwd,
+    attn_get_device_status,
+    attn_status_string,
+    lib,
+    library_path,
+)

@@ -1,0 +1,130 @@
+"""Thin ctypes binding over the C ABI in ``include/attn.h``.
+
+Argument marshalling only: shapes are read from the tensors, pointers and the
+current CUDA stream are passed through, outputs are allocated with torch when
+the caller gives none.  Every step of attention runs in the CUDA library; there
+is no CPU or PyTorch fallback, and a missing or unloadable library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libattn_b200.so")
+
+ATTN_OK = 0
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {attn_status_string(status)} ({status})")
+
+
+def lib():
+    """Load libattn_b200.so (built by ``__graft_entry__.build()``); raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise ImportError(f"{library_path} is not built; run __graft_entry__.build()")
+    L = ctypes.CDLL(library_path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    L.attn_fwd.restype = i
+    L.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
+    L.attn_bwd_workspace_size.restype = sz
+    L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    L.attn_bwd.restype = i
+    L.attn_get_device_status.argtypes = [vp]
+    L.attn_get_device_status.restype = i
+    L.attn_status_string.argtypes = [i]
+    L.attn_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def attn_status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check(t, name, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def attn_fwd(q, k, v, o=None, lse=None, *, scale=None, causal=False, stream=None):
+    """O = softmax(scale * Q K^T) V and the per-row log-sum-exp; returns (o, lse).
+
+    q: [B, Hq, N, d] bf16; k, v: [B, Hkv, N, d] bf16; o: like q; lse: [B, Hq, N] fp32.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _check(o, "o")
+    _check(lse, "lse", torch.float32)
+    if scale is None:
+        scale = d ** -0.5
+    st = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                        float(scale), int(bool(causal)), _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def attn_bwd_workspace_size(B, Hq, Hkv, N, d, causal=False) -> int:
+    return int(lib().attn_bwd_workspace_size(B, Hq, Hkv, N, d, int(bool(causal))))
+
+
+def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale=None, causal=False,
+             workspace=None, stream=None):
+    """Gradients of sum(O * dO) with respect to q, k, v; returns (dq, dk, dv)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _check(t, n)
+    _check(lse, "lse", torch.float32)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _check(t, n)
+    if scale is None:
+        scale = d ** -0.5
+    need = attn_bwd_workspace_size(B, Hq, Hkv, N, d, causal)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                        _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+                        _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device-side error word."""
+    return int(lib().attn_get_device_status(_stream_ptr(stream)))

@@ -1,0 +1,142 @@
+"""numpy fp64 oracle for exact attention (TEST INFRASTRUCTURE ONLY, see package docstring).
+
+Definition followed (page "attention 的显存线性化", §一, and page "注意力计算的计算与
+显存瓶颈", §1.1.1): S = Q K^T / sqrt(d_k), P = softmax(S) row by row, O = P V.
+The row softmax subtracts the row maximum first (same page 1, §1.1.8 formula):
+P_ij = exp(S_ij - m_i) / sum_j exp(S_ij - m_i).
+
+Readings where the pages are silent (each is listed in the design doc):
+* ``scale`` is an explicit argument; the intended value is 1/sqrt(d).
+* causal: query i sees keys j <= i (equal query and key lengths).
+* GQA (page "attn-efficient", table of the three families, row ③): q-head h uses
+  kv-head h // (Hq // Hkv), contiguous groups.
+* LSE_i = m_i + ln sum_j exp(S_ij - m_i), natural log over the scaled scores,
+  masked keys excluded.
+* Backward (the pages only say it recomputes local blocks, page
+  "attention 的显存线性化" §五): exact gradient of L = sum(O * dO):
+  dV = P^T dO, dP = dO V^T, D_i = sum_k dO_ik O_ik, dS = P * (dP - D),
+  dQ = scale dS K, dK = scale dS^T Q; GQA sums dK, dV over the group.
+
+Rows are independent (page 1 §1.1.8), so computing S and P for a block of rows
+at a time gives the same values as the whole matrix; this is the only
+restructuring here and it exists only to bound memory at N = 32768.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _scores(qh, kh, scale, causal, rows):
+    """S for the query rows ``rows`` (array of indices) of one head, fp64, masked with -inf."""
+    s = scale * (qh[rows] @ kh.T)
+    if causal:
+        keys = np.arange(kh.shape[0])
+        s = np.where(keys[None, :] <= rows[:, None], s, -np.inf)
+    return s
+
+
+def _softmax_rows(s):
+    """Row softmax with max subtraction; returns (P, m, LSE)."""
+    m = s.max(axis=1)
+    e = np.exp(s - m[:, None])
+    l = e.sum(axis=1)
+    return e / l[:, None], m, m + np.log(l)
+
+
+def attend_head(qh, kh, vh, scale, causal, rows=None, block=1024):
+    """O and LSE for the given query rows of one head (all rows when ``rows`` is None).
+
+    qh: [N, d]; kh, vh: [N, d]; fp64.  Returns (O[len(rows), d], LSE[len(rows)]).
+    """
+    n = qh.shape[0]
+    rows = np.arange(n) if rows is None else np.asarray(rows, dtype=np.int64)
+    o = np.empty((rows.shape[0], vh.shape[1]))
+    lse = np.empty(rows.shape[0])
+    for a in range(0, rows.shape[0], block):
+        r = rows[a:a + block]
+        p, _, lse[a:a + block] = _softmax_rows(_scores(qh, kh, scale, causal, r))
+        o[a:a + block] = p @ vh
+    return o, lse
+
+
+def ref_fwd(q, k, v, scale, causal, block=1024):
+    """Forward oracle.  q [B,Hq,N,d], k/v [B,Hkv,N,d] fp64 -> O [B,Hq,N,d], LSE [B,Hq,N]."""
+    B, Hq, N, d = q.shape
+    G = Hq // k.shape[1]
+    o = np.empty((B, Hq, N, v.shape[3]))
+    lse = np.empty((B, Hq, N))
+    for b in range(B):
+        for h in range(Hq):
+            o[b, h], lse[b, h] = attend_head(q[b, h], k[b, h // G], v[b, h // G], scale, causal,
+                                             block=block)
+    return o, lse
+
+
+def grad_head(qh, kh, vh, doh, scale, causal, block=1024):
+    """Gradients of sum(O * dO) for one q-head against its kv-head: (dQ, dK, dV), fp64."""
+    n = qh.shape[0]
+    dq = np.empty_like(qh)
+    dk = np.zeros_like(kh)
+    dv = np.zeros_like(vh)
+    for a in range(0, n, block):
+        r = np.arange(a, min(n, a + block))
+        p, _, _ = _softmax_rows(_scores(qh, kh, scale, causal, r))
+        o = p @ vh
+        dd = (doh[r] * o).sum(axis=1)              # D_i = sum_k dO_ik O_ik
+        dp = doh[r] @ vh.T                          # dP = dO V^T
+        ds = p * (dp - dd[:, None])                 # dS = P * (dP - D)
+        dq[r] = scale * (ds @ kh)
+        dk += scale * (ds.T @ qh[r])
+        dv += p.T @ doh[r]
+    return dq, dk, dv
+
+
+def ref_bwd(q, k, v, do, scale, causal, block=1024):
+    """Backward oracle: (dQ [B,Hq,N,d], dK [B,Hkv,N,d], dV [B,Hkv,N,d]) in fp64."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    dq = np.empty_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            dq[b, h], dkh, dvh = grad_head(q[b, h], k[b, g], v[b, g], do[b, h], scale, causal,
+                                           block=block)
+            dk[b, g] += dkh
+            dv[b, g] += dvh
+    return dq, dk, dv
+
+
+def online_fwd_head(qh, kh, vh, scale, causal, bounds):
+    """The pages' blockwise online softmax for one head (used only in self-tests).
+
+    Page "attention 的显存线性化" §三: for each key block j, with S_ij = Q_i K_j^T,
+      m^(j) = max(m^(j-1), rowmax S_ij)
+      l^(j) = exp(m^(j-1) - m^(j)) l^(j-1) + rowsum exp(S_ij - m^(j)).
+    The output update printed there is incomplete; page "attn-efficient"
+    (online-softmax section) completes it: whenever the max grows, the partial
+    output is multiplied by exp(m_old - m_new).  Reading used:
+      O_acc^(j) = exp(m^(j-1) - m^(j)) O_acc^(j-1) + exp(S_ij - m^(j)) V_j,
+      O = O_acc / l,  LSE = m + ln l.
+    ``bounds`` are the key-block edges, e.g. [0, 3, 4, 10, N].
+    """
+    n, dv = qh.shape[0], vh.shape[1]
+    rows = np.arange(n)
+    m = np.full(n, -np.inf)
+    l = np.zeros(n)
+    acc = np.zeros((n, dv))
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        s = scale * (qh @ kh[a:b].T)
+        if causal:
+            keys = np.arange(a, b)
+            s = np.where(keys[None, :] <= rows[:, None], s, -np.inf)
+        m_new = np.maximum(m, s.max(axis=1))
+        live = np.isfinite(m_new)   # rows that have seen at least one unmasked key
+        alpha = np.where(live, np.exp(np.where(live, m - m_new, 0.0)), 1.0)
+        pt = np.where(live[:, None], np.exp(s - np.where(live, m_new, 0.0)[:, None]), 0.0)
+        l = alpha * l + pt.sum(axis=1)
+        acc = alpha[:, None] * acc + pt @ vh[a:b]
+        m = m_new
+    return acc / l[:, None], m + np.log(l)
