@@ -1,0 +1,90 @@
+/* attn.h -- C ABI of the B200 exact-attention library (libattn_b200.so).
+ *
+ * The operation is exact scaled-dot-product attention,
+ *     O = softmax(scale * Q K^T) V,
+ * as defined on page "attention 的显存线性化" §一 (softmax(Q K^T / sqrt(d_k)) V)
+ * and page "注意力计算的计算与显存瓶颈" §1.1.1 (S = Q K^T / sqrt(d), P = softmax(S),
+ * O = P V), computed tile by tile with an online softmax so that the n x n
+ * matrices S and P never reach device memory (page "attention 的显存线性化" §三;
+ * page "attn-efficient", online-softmax section).  The backward recomputes the
+ * needed S/P tiles from the saved log-sum-exp instead of storing them (page
+ * "attention 的显存线性化" §五; page "attn-efficient", recompute paragraph).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers: all tensor pointers are DEVICE pointers on the current CUDA device,
+ *   owned by the caller, contiguous row-major, 16-byte aligned.  The library
+ *   keeps no pointer after a call returns.
+ * Layouts (bf16 = IEEE bfloat16, 2 bytes; fp32 = 4 bytes):
+ *   q, o, dO, dq : bf16 [B][Hq][N][d]
+ *   k, v, dk, dv : bf16 [B][Hkv][N][d]
+ *   lse          : fp32 [B][Hq][N], natural log of sum_j exp(scale * q_i . k_j)
+ *                  over the keys row i may see.
+ * Heads: grouped-query attention maps q-head h to kv-head h / (Hq / Hkv)
+ *   (contiguous groups; page "attn-efficient", GQA / MQA row of the family table).
+ *   Hkv == Hq is ordinary multi-head attention, Hkv == 1 is multi-query attention.
+ * causal: 0 = every query sees every key; 1 = query i sees keys j <= i
+ *   (equal query and key lengths).
+ * scale: finite and >= 0; the usual value is 1/sqrt(d).
+ * d: 64 or 128.  N: any value >= 1 (ragged tails are masked on device).
+ * Streams: work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and the call returns without waiting.  Results are stream-ordered.
+ * Errors: arguments are validated on the host before any launch; a rejected
+ *   call launches nothing and returns a negative attn_status_t.  Device-side
+ *   waits are bounded: if one expires the kernel records an error word and
+ *   exits; attn_get_device_status() reports it.  No entry point aborts, traps
+ *   or throws.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1,   /* null pointer, bad shape, Hq % Hkv != 0, bad scale */
+  ATTN_ERR_UNSUPPORTED = -2,   /* d not in {64, 128}, or no sm_100 device */
+  ATTN_ERR_ALIGNMENT = -3,     /* a pointer is not 16-byte aligned */
+  ATTN_ERR_LAUNCH = -4,        /* the CUDA runtime refused a launch or an attribute */
+  ATTN_ERR_DEVICE_TIMEOUT = -5,/* a bounded device wait expired (see attn_get_device_status) */
+  ATTN_ERR_WORKSPACE = -6      /* backward workspace missing or too small */
+} attn_status_t;
+
+/* Forward: O and LSE for every (b, h, i).
+ * Reads q, k, v; writes o and lse.  Returns ATTN_OK or a negative status. */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+             void* stream);
+
+/* Bytes of device workspace attn_bwd needs for this shape (caller allocates;
+ * contents need no initialisation).  Returns 0 for arguments attn_bwd would reject. */
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int causal);
+
+/* Backward: gradients of sum(O * dO) with respect to q, k, v.
+ * Reads q, k, v, o (the forward output), lse (the forward log-sum-exp) and dO;
+ * writes dq, dk, dv.  For GQA, dk and dv sum over the q-heads of each group.
+ * The reduction order is fixed, so two calls on the same inputs give the same
+ * bits.  `workspace` must hold attn_bwd_workspace_size(...) bytes, 16-byte
+ * aligned; it is overwritten. */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dO, void* dq, void* dk, void* dv,
+             int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns ATTN_OK if no kernel of this library
+ * recorded a device-side error since the last call, else ATTN_ERR_DEVICE_TIMEOUT;
+ * the error word is cleared.  While the word is set, later launches exit early. */
+int attn_get_device_status(void* stream);
+
+/* Static, human-readable text for a status code. */
+const char* attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

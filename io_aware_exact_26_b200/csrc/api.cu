@@ -1,0 +1,267 @@
+// Host side of libattn_b200.so: the extern "C" entry points declared in
+// include/attn.h.  Validates arguments, encodes the TMA tensor maps, picks the
+// kernel instance and launches it on the caller's stream.  No allocation, no
+// synchronisation on the launch path.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+#include "fwd.cuh"
+#include "bwd.cuh"
+
+namespace {
+
+using attn::FwdCfg;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D view [heads][rows][d] of a bf16 tensor; box = 64 columns x box_rows rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int d, int rows, long long heads, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(d) * 2 * rows};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+  bool fwd64 = false, fwd128 = false;
+};
+
+int device_info(DeviceInfo** out) {
+  static DeviceInfo infos[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo& di = infos[dev];
+  if (di.sms == 0) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return 1;
+    di.major = prop.major;
+    di.sms = prop.multiProcessorCount;
+  }
+  *out = &di;
+  return di.major == 10 ? 0 : 1;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int Hq, int Hkv, int N, int d, float scale, int causal) {
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  const long long tiles = static_cast<long long>(B) * Hq * ((N + 127) / 128);
+  if (tiles > INT_MAX / 2) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(N) * d * 2 * 2 >= (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+template <int D>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+               int N, float scale, int causal, cudaStream_t stream, const DeviceInfo& di) {
+  using C = FwdCfg<D>;
+  static std::once_flag attr_once[64];
+  static bool attr_ok[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(attr_once[dev], [&] {
+    attr_ok[dev] = cudaFuncSetAttribute(attn::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmem) == cudaSuccess;
+  });
+  if (!attr_ok[dev]) return ATTN_ERR_LAUNCH;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, N, static_cast<long long>(B) * Hq, 128) ||
+      !make_map(&tk, k, D, N, static_cast<long long>(B) * Hkv, 128) ||
+      !make_map(&tv, v, D, N, static_cast<long long>(B) * Hkv, 128))
+    return ATTN_ERR_LAUNCH;
+  attn::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.G = Hq / Hkv;
+  p.n_qtiles = (N + 127) / 128;
+  p.total_tiles = p.n_qtiles * B * Hq;
+  p.c = scale * 1.4426950408889634f;
+  p.causal = causal;
+  const int grid = p.total_tiles < di.sms ? p.total_tiles : di.sms;
+  attn::attn_fwd_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+}  // namespace
+
+namespace attn {
+
+template <int D>
+static int launch_bwd_d(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, float scale,
+                        int causal, void* workspace, cudaStream_t stream, int sms) {
+  using C = BwdCfg<D>;
+  static std::once_flag attr_once[64];
+  static bool attr_ok[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(attr_once[dev], [&] {
+    attr_ok[dev] = cudaFuncSetAttribute(attn_bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmem) == cudaSuccess;
+  });
+  if (!attr_ok[dev]) return ATTN_ERR_LAUNCH;
+  const long long BHq = static_cast<long long>(B) * Hq;
+  const BwdLayout L = bwd_layout(BHq, N, D);
+  char* ws = static_cast<char*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(ws + L.lse2_off);
+  float* dd = reinterpret_cast<float*>(ws + L.dd_off);
+  float* acc = reinterpret_cast<float*>(ws + L.acc_off);
+  int* tickets = reinterpret_cast<int*>(ws + L.ticket_off);
+  const int nt = (N + 127) / 128;
+  const long long n_tickets = BHq * nt * 4;
+  {
+    const long long rows = BHq * nt * 128;
+    long long blocks = (rows * 32 + 255) / 256;
+    const long long cap = static_cast<long long>(sms) * 16;
+    if (blocks > cap) blocks = cap;
+    attn_bwd_prep_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dd, tickets, BHq,
+        N, n_tickets);
+    if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, D, N, BHq, 128) || !make_map(&tk, k, D, N, static_cast<long long>(B) * Hkv, 128) ||
+      !make_map(&tv, v, D, N, static_cast<long long>(B) * Hkv, 128) || !make_map(&tdo, dO, D, N, BHq, 128))
+    return ATTN_ERR_LAUNCH;
+  BwdParams p;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.lse2 = lse2;
+  p.dd = dd;
+  p.acc = acc;
+  p.tickets = tickets;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.G = Hq / Hkv;
+  p.nt = nt;
+  p.total_items = B * Hkv * nt;
+  p.c = scale * 1.4426950408889634f;
+  p.scale = scale;
+  int grid;
+  if (causal) {
+    p.order = 0;
+    grid = p.total_items < sms ? p.total_items : sms;
+  } else if (nt <= sms) {
+    // cyclic order: the nt items of one head run side by side, so grid is a multiple of nt
+    p.order = 2;
+    const int g = (sms / nt) * nt;
+    grid = p.total_items < g ? p.total_items : g;
+  } else {
+    p.order = 1;
+    grid = p.total_items < sms ? p.total_items : sms;
+  }
+  attn_bwd_main_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, tdo, p);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+               void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+               void* workspace, cudaStream_t stream, int sms) {
+  if (d == 64)
+    return launch_bwd_d<64>(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, stream, sms);
+  return launch_bwd_d<128>(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, stream, sms);
+}
+
+}  // namespace attn
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+             int d, float scale, int causal, void* stream) {
+  int st = check_common(B, Hq, Hkv, N, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_fwd<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, *di);
+  return launch_fwd<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, *di);
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int causal) {
+  if (check_common(B, Hq, Hkv, N, d, 1.f, causal) != ATTN_OK) return 0;
+  return attn::bwd_workspace_bytes(B, Hq, Hkv, N, d);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_common(B, Hq, Hkv, N, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return ATTN_ERR_ALIGNMENT;
+  const size_t need = attn::bwd_workspace_bytes(B, Hq, Hkv, N, d);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return ATTN_ERR_WORKSPACE;
+  if (workspace && !aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
+  return attn::launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, workspace,
+                          static_cast<cudaStream_t>(stream), di->sms);
+}
+
+int attn_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, attn::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (v != 0 && cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int)) != cudaSuccess)
+    return ATTN_ERR_LAUNCH;
+  return v == 0 ? ATTN_OK : ATTN_ERR_DEVICE_TIMEOUT;
+}
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported (head dim must be 64 or 128; device must be sm_100)";
+    case ATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case ATTN_ERR_LAUNCH: return "CUDA launch or attribute error";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+    case ATTN_ERR_WORKSPACE: return "backward workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

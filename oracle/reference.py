@@ -140,3 +140,36 @@ def online_fwd_head(qh, kh, vh, scale, causal, bounds):
         acc = alpha[:, None] * acc + pt @ vh[a:b]
         m = m_new
     return acc / l[:, None], m + np.log(l)
+
+
+def grad_q_rows(qh, kh, vh, doh, scale, causal, rows):
+    """dQ for the given query rows of one head (full key range), from the same formulas as
+    ``grad_head``; used to check sampled rows of full-size problems."""
+    rows = np.asarray(rows, dtype=np.int64)
+    p, _, _ = _softmax_rows(_scores(qh, kh, scale, causal, rows))
+    o = p @ vh
+    dd = (doh[rows] * o).sum(axis=1)
+    ds = p * (doh[rows] @ vh.T - dd[:, None])
+    return scale * (ds @ kh)
+
+
+def grad_kv_rows(qhs, kh, vh, dohs, scale, causal, keys, block=1024):
+    """dK and dV for the given key rows of one kv-head, summed over the q-heads in
+    ``qhs`` / ``dohs`` (the GQA group).  Needs LSE and D of every query row, so it
+    costs one full forward per q-head."""
+    keys = np.asarray(keys, dtype=np.int64)
+    dk = np.zeros((keys.shape[0], kh.shape[1]))
+    dv = np.zeros((keys.shape[0], vh.shape[1]))
+    n = kh.shape[0]
+    for qh, doh in zip(qhs, dohs):
+        for a in range(0, n, block):
+            r = np.arange(a, min(n, a + block))
+            p_full, m, lse = _softmax_rows(_scores(qh, kh, scale, causal, r))
+            o = p_full @ vh
+            dd = (doh[r] * o).sum(axis=1)
+            p = p_full[:, keys]                          # P[r, keys]
+            dp = doh[r] @ vh[keys].T
+            ds = p * (dp - dd[:, None])
+            dk += scale * (ds.T @ qh[r])
+            dv += p.T @ doh[r]
+    return dk, dv

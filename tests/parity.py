@@ -1,0 +1,57 @@
+"""Tolerances for comparing the CUDA path (bf16 outputs) with the fp64 oracle.
+
+Forward, per element:  |dO| <= 1e-2 + half a bf16 ulp of |O_ref|  (an exactly computed
+  O rounded to bf16 already misses 1e-2 once |O| >= 2, so the bf16 rounding of the
+  output itself is allowed on top of the 1e-2 budget);
+  relative RMS over the tensor <= 5e-3;  |dLSE| <= 1e-3 (LSE stays fp32).
+Gradients, per tensor: max |d| <= 2e-2 * max(1, max |ref|), relative RMS <= 1e-2.
+All of these reduce to the plain 1e-2 / 5e-3 / 1e-3 / 2e-2 bounds wherever values are O(1).
+"""
+import numpy as np
+import torch
+
+O_ATOL = 1e-2
+O_RRMS = 5e-3
+LSE_ATOL = 1e-3
+G_REL = 2e-2
+G_RRMS = 1e-2
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def half_ulp_bf16(x):
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    e = np.floor(np.log2(ax))
+    return 2.0 ** (e - 8)
+
+
+def rel_rms(got, ref):
+    den = np.sqrt(np.mean(ref ** 2))
+    return float(np.sqrt(np.mean((got - ref) ** 2)) / max(den, 1e-30))
+
+
+def check_o(got, ref, what="O"):
+    got = np.asarray(got, np.float64)
+    err = np.abs(got - ref)
+    bound = O_ATOL + half_ulp_bf16(ref)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert np.all(err <= bound), f"{what}: max |err| {err.max():.3g}, worst at {worst}: got {got[worst]} ref {ref[worst]}"
+    rr = rel_rms(got, ref)
+    assert rr <= O_RRMS, f"{what}: relative RMS {rr:.3g}"
+
+
+def check_lse(got, ref):
+    err = np.abs(np.asarray(got, np.float64) - ref)
+    assert err.max() <= LSE_ATOL, f"LSE: max |err| {err.max():.3g} at {np.unravel_index(np.argmax(err), err.shape)}"
+
+
+def check_grad(got, ref, what):
+    got = np.asarray(got, np.float64)
+    err = np.abs(got - ref)
+    bound = G_REL * max(1.0, float(np.abs(ref).max()))
+    worst = np.unravel_index(np.argmax(err), err.shape)
+    assert err.max() <= bound, f"{what}: max |err| {err.max():.3g} > {bound:.3g} at {worst}: got {got[worst]} ref {ref[worst]}"
+    rr = rel_rms(got, ref)
+    assert rr <= G_RRMS, f"{what}: relative RMS {rr:.3g}"

@@ -1,0 +1,89 @@
+"""The C ABI: the library loads, exports every symbol include/attn.h declares, and
+rejects bad arguments on the host before any launch (no GPU needed for these)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import __graft_entry__
+from io_aware_exact_26_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    __graft_entry__.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted(
+        ["attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_get_device_status", "attn_status_string"])
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in range(-6, 1):
+        assert binding.attn_status_string(code)
+    assert binding.attn_status_string(-99) == "unknown status"
+
+
+FAKE = ctypes.c_void_p(0x10000)       # 16-byte aligned, never dereferenced on these paths
+ODD = ctypes.c_void_p(0x10008)
+
+
+def fwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=1, Hkv=1, N=128, d=64, scale=0.125, causal=0):
+    return L.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), -2), (dict(d=256), -2), (dict(N=0), -1), (dict(B=0), -1), (dict(Hq=3, Hkv=2), -1),
+    (dict(Hkv=0), -1), (dict(scale=float("nan")), -1), (dict(scale=float("inf")), -1), (dict(scale=-1.0), -1),
+    (dict(causal=2), -1), (dict(q=ctypes.c_void_p(0)), -1), (dict(lse=ctypes.c_void_p(0)), -1),
+    (dict(q=ODD), -3), (dict(o=ODD), -3), (dict(lse=ODD), -3),
+])
+def test_fwd_rejects_bad_arguments(L, kw, code):
+    assert fwd(L, **kw) == code
+
+
+def test_bwd_rejects_bad_arguments(L):
+    size = L.attn_bwd_workspace_size(1, 2, 1, 300, 128, 1)
+    assert size > 0
+    assert L.attn_bwd_workspace_size(1, 3, 2, 300, 128, 1) == 0
+    assert L.attn_bwd_workspace_size(1, 2, 1, 300, 96, 1) == 0
+
+    def bwd(ws=FAKE, wsb=size, dq=FAKE, d=128, Hq=2, Hkv=1):
+        return L.attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, dq, FAKE, FAKE, 1, Hq, Hkv, 300, d, 0.1, 1,
+                          ws, ctypes.c_size_t(wsb), None)
+    assert bwd(ws=ctypes.c_void_p(0)) == -6
+    assert bwd(wsb=size - 1) == -6
+    assert bwd(dq=ODD) == -3
+    assert bwd(dq=ctypes.c_void_p(0)) == -1
+    assert bwd(d=80) == -2
+    assert bwd(Hq=3, Hkv=2) == -1
+    assert bwd(Hq=3) == -6   # valid shape, but the workspace was sized for Hq=2
+
+
+def test_workspace_size_grows_linearly_in_n(L):
+    a = L.attn_bwd_workspace_size(2, 8, 2, 4096, 128, 1)
+    b = L.attn_bwd_workspace_size(2, 8, 2, 8192, 128, 1)
+    assert 1.9 < b / a < 2.1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "library_path", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        binding.lib()

@@ -305,3 +305,17 @@ def test_seeded_inputs_are_bf16_and_reproducible():
     ratio = to_f64(a["k"]) / np.where(to_f64(c["k"]) == 0, 1, to_f64(c["k"]))
     per_row = np.isclose(ratio, 8.0).all(axis=-1)
     assert per_row.sum(axis=-1).tolist() == [[3, 3]]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_gradient_rows_match_full_backward(causal):
+    B, Hq, Hkv, N, d = 1, 4, 2, 45, 6
+    q, k, v, do = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d), rand(B, Hq, N, d)
+    dq, dk, dv = ref.ref_bwd(q, k, v, do, 0.45, causal)
+    rows = np.array([0, 7, 44])
+    np.testing.assert_allclose(ref.grad_q_rows(q[0, 3], k[0, 1], v[0, 1], do[0, 3], 0.45, causal, rows),
+                               dq[0, 3, rows], rtol=1e-12, atol=1e-13)
+    gk, gv = ref.grad_kv_rows([q[0, 2], q[0, 3]], k[0, 1], v[0, 1], [do[0, 2], do[0, 3]], 0.45, causal,
+                              rows, block=16)
+    np.testing.assert_allclose(gk, dk[0, 1, rows], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(gv, dv[0, 1, rows], rtol=1e-11, atol=1e-12)
