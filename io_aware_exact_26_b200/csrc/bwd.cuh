@@ -37,24 +37,6 @@
 
 namespace attn {
 
-__device__ __forceinline__ bool bwd_aborted() {
-  return *reinterpret_cast<volatile int*>(&g_attn_status) != 0;
-}
-
-__device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023) == 1023 && bwd_aborted()) return false;
-  }
-  record_error(&g_attn_status, 1);
-  return false;
-}
-
-__device__ __forceinline__ void bwd_drain_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < (1u << 22); ++i)
-    if (mbar_try_wait(bar, parity)) return;
-}
-
 // Untiled bulk copy global -> shared (both 16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -265,7 +247,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
         int bhkv, j;
         bwd_item(p, t, bhkv, j);
-        if (it >= 1) ok = bwd_wait(&sh.kv_empty, (it - 1) & 1);
+        if (it >= 1) ok = mbar_wait(&sh.kv_empty, (it - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&sh.kv_full, 2 * C::kTile);
         for (int c = 0; c < D / 64; ++c) {
@@ -281,7 +263,7 @@ __global__ void __launch_bounds__(320, 1)
             int i, pos; bool last;
             bwd_step(p, j, s, i, pos, last);
             const int st = gs & 1;
-            if (gs >= 2) ok = bwd_wait(&sh.qdo_empty[st], ((gs >> 1) - 1) & 1);
+            if (gs >= 2) ok = mbar_wait(&sh.qdo_empty[st], ((gs >> 1) - 1) & 1);
             if (!ok) break;
             mbar_arrive_expect_tx(&sh.qdo_full[st], 2 * C::kTile + 1024);
             for (int c = 0; c < D / 64; ++c) {
@@ -296,8 +278,8 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (!ok) {
-        if (nkv >= 1) bwd_drain_wait(&sh.kv_full, (nkv - 1) & 1);
-        for (int g = max(0, nq - 2); g < nq; ++g) bwd_drain_wait(&sh.qdo_full[g & 1], (g >> 1) & 1);
+        if (nkv >= 1) mbar_drain_wait(&sh.kv_full, (nkv - 1) & 1);
+        for (int g = max(0, nq - 2); g < nq; ++g) mbar_drain_wait(&sh.qdo_full[g & 1], (g >> 1) & 1);
       }
     }
   } else if (warp == 9) {
@@ -311,7 +293,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
         int bhkv, j;
         bwd_item(p, t, bhkv, j);
-        ok = bwd_wait(&sh.kv_full, it & 1);
+        ok = mbar_wait(&sh.kv_full, it & 1);
         if (!ok) break;
         const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), ds_addr = smem_u32(sDS);
         const int steps = bwd_steps_per_head(p, j);
@@ -319,9 +301,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int h = 0; h < p.G && ok; ++h) {
           for (int s = 0; s < steps; ++s, ++gs) {
             const int st = gs & 1;
-            ok = bwd_wait(&sh.qdo_full[st], (gs >> 1) & 1);
-            if (ok && gs >= 1) ok = bwd_wait(&sh.step_done, (gs - 1) & 1);
-            if (ok && D == 128 && gs >= 1) ok = bwd_wait(&sh.dq_free, (gs - 1) & 1);  // dQ aliases dP^T
+            ok = mbar_wait(&sh.qdo_full[st], (gs >> 1) & 1);
+            if (ok && gs >= 1) ok = mbar_wait(&sh.step_done, (gs - 1) & 1);
+            if (ok && D == 128 && gs >= 1) ok = mbar_wait(&sh.dq_free, (gs - 1) & 1);  // dQ aliases dP^T
             if (!ok) break;
             tc_fence_after();
             const uint32_t q_addr = smem_u32(sQ + st * C::kTile), do_addr = smem_u32(sDO + st * C::kTile);
@@ -339,8 +321,8 @@ __global__ void __launch_bounds__(320, 1)
                       idST, k > 0);
             }
             umma_commit(&sh.st_full);
-            ok = bwd_wait(&sh.ds_ready, gs & 1);
-            if (ok && first && it >= 1) ok = bwd_wait(&sh.acc_free, (it - 1) & 1);
+            ok = mbar_wait(&sh.ds_ready, gs & 1);
+            if (ok && first && it >= 1) ok = mbar_wait(&sh.acc_free, (it - 1) & 1);
             if (!ok) break;
             tc_fence_after();
             // dV += P^T dO  (A = P^T from TMEM, B = dO MN-major; K = queries)
@@ -357,7 +339,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             // dQ = dS K  (A = dS^T read MN-major, B = K MN-major; K = keys)
             if (D != 128 && gs >= 1) {
-              ok = bwd_wait(&sh.dq_free, (gs - 1) & 1);
+              ok = mbar_wait(&sh.dq_free, (gs - 1) & 1);
               if (!ok) break;
               tc_fence_after();
             }
@@ -375,7 +357,7 @@ __global__ void __launch_bounds__(320, 1)
         umma_commit(&sh.kv_empty);
       }
       umma_commit(&sh.drain);
-      bwd_wait(&sh.drain, 0);
+      mbar_wait(&sh.drain, 0);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ dS warpgroup (rows = keys)
@@ -399,9 +381,9 @@ __global__ void __launch_bounds__(320, 1)
           const int st = gs & 1;
           const float* sLse = sVec + st * 256;
           const float* sDd = sLse + 128;
-          ok = __all_sync(0xffffffffu, bwd_wait(&sh.qdo_full[st], (gs >> 1) & 1));
-          if (ok) ok = __all_sync(0xffffffffu, bwd_wait(&sh.st_full, gs & 1));
-          if (ok && gs >= 1) ok = __all_sync(0xffffffffu, bwd_wait(&sh.step_done, (gs - 1) & 1));
+          ok = __all_sync(0xffffffffu, mbar_wait(&sh.qdo_full[st], (gs >> 1) & 1));
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.st_full, gs & 1));
+          if (ok && gs >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&sh.step_done, (gs - 1) & 1));
           if (!ok) break;
           tc_fence_after();
           // visible queries of this key row: causal needs query >= key; both need < N
@@ -465,7 +447,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int s = 0; s < steps; ++s, ++gs) {
           int i, pos; bool last;
           bwd_step(p, j, s, i, pos, last);
-          ok = __all_sync(0xffffffffu, bwd_wait(&sh.dq_full, gs & 1));
+          ok = __all_sync(0xffffffffu, mbar_wait(&sh.dq_full, gs & 1));
           if (!ok) break;
           tc_fence_after();
           float part[D];
@@ -486,14 +468,18 @@ __global__ void __launch_bounds__(320, 1)
           if (pos > 0) {
             if (lane == 0) {
               turn = false;
-              for (uint32_t spin = 0; spin < kSpinLimit; ++spin) {
+              const uint64_t t0 = globaltimer_ns();
+              for (uint32_t spin = 0;; ++spin) {
                 if (ld_acquire(ticket) == pos) { turn = true; break; }
-                if ((spin & 255) == 255) {
-                  if (bwd_aborted()) break;
-                  __nanosleep(64);
+                if ((spin & 15) == 15) {
+                  if (status_set()) break;
+                  if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+                    record_error(&g_attn_status, 2);
+                    break;
+                  }
+                  __nanosleep(32);
                 }
               }
-              if (!turn && !bwd_aborted()) record_error(&g_attn_status, 2);
             }
             turn = __shfl_sync(0xffffffffu, turn, 0);
           }
@@ -533,7 +519,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (!ok) break;
       // epilogue of the item: dV and scale * dK rows (TMEM lane = key)
-      ok = __all_sync(0xffffffffu, bwd_wait(&sh.step_done, (gs - 1) & 1));
+      ok = __all_sync(0xffffffffu, mbar_wait(&sh.step_done, (gs - 1) & 1));
       if (!ok) break;
       tc_fence_after();
       const int key = j * 128 + r;

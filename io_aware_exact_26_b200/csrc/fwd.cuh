@@ -23,7 +23,9 @@
 // invariance of softmax (page "attn-efficient": subtracting the same number from
 // a whole score row leaves the result unchanged) any reference value works as
 // long as O and l use the same one; this keeps p <= 2^tau and skips most O
-// rescales.  l accumulates the bf16-rounded p that the PV MMA consumes.
+// rescales.  Two row sums are kept: l of the bf16-rounded p that the PV MMA
+// consumes (O is normalised by it, so a constant V comes out exactly), and the
+// fp32 sum of the unrounded p, from which the LSE is formed.
 #pragma once
 #include "sm100.cuh"
 
@@ -62,26 +64,6 @@ struct FwdShared {
   uint64_t drain;
   uint32_t tmem_base;
 };
-
-__device__ __forceinline__ bool aborted() {
-  return *reinterpret_cast<volatile int*>(&g_attn_status) != 0;
-}
-
-// Bounded wait that also gives up early once any CTA recorded an error.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023) == 1023 && aborted()) return false;
-  }
-  record_error(&g_attn_status, 1);
-  return false;
-}
-
-// Bounded wait used only to let in-flight copies land on the error path.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < (1u << 22); ++i)
-    if (mbar_try_wait(bar, parity)) return;
-}
 
 // Work tile t -> (query tile, batch*head).  Causal: longest rows first.
 __device__ __forceinline__ void fwd_tile_coords(const FwdParams& p, int t, int& qt, int& bh) {
@@ -141,7 +123,7 @@ __global__ void __launch_bounds__(192, 1)
         const int n_kv = fwd_n_kv(p, qt);
         const int bkv = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.G;
         const int qb = tl & 1;
-        if (tl >= 2) ok = wait_bar(&sh.q_empty[qb], ((tl >> 1) - 1) & 1);
+        if (tl >= 2) ok = mbar_wait(&sh.q_empty[qb], ((tl >> 1) - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&sh.q_full[qb], C::kTile);
         for (int c = 0; c < D / 64; ++c)
@@ -151,7 +133,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int s = 0; s <= n_kv && ok; ++s) {
           if (s < n_kv) {
             const int g = it + s, st = g % C::KST;
-            if (g >= C::KST) ok = wait_bar(&sh.k_empty[st], ((g / C::KST) - 1) & 1);
+            if (g >= C::KST) ok = mbar_wait(&sh.k_empty[st], ((g / C::KST) - 1) & 1);
             if (!ok) break;
             mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
             for (int c = 0; c < D / 64; ++c)
@@ -160,7 +142,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           if (s >= 1) {
             const int g = it + s - 1, st = g % C::VST;
-            if (g >= C::VST) ok = wait_bar(&sh.v_empty[st], ((g / C::VST) - 1) & 1);
+            if (g >= C::VST) ok = mbar_wait(&sh.v_empty[st], ((g / C::VST) - 1) & 1);
             if (!ok) break;
             mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
             for (int c = 0; c < D / 64; ++c)
@@ -172,9 +154,9 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!ok) {
         // Let the copies already in flight land before the CTA exits (bounded).
-        for (int g = max(0, nk - C::KST); g < nk; ++g) drain_wait(&sh.k_full[g % C::KST], (g / C::KST) & 1);
-        for (int g = max(0, nv - C::VST); g < nv; ++g) drain_wait(&sh.v_full[g % C::VST], (g / C::VST) & 1);
-        for (int g = max(0, nq - 2); g < nq; ++g) drain_wait(&sh.q_full[g & 1], (g >> 1) & 1);
+        for (int g = max(0, nk - C::KST); g < nk; ++g) mbar_drain_wait(&sh.k_full[g % C::KST], (g / C::KST) & 1);
+        for (int g = max(0, nv - C::VST); g < nv; ++g) mbar_drain_wait(&sh.v_full[g % C::VST], (g / C::VST) & 1);
+        for (int g = max(0, nq - 2); g < nq; ++g) mbar_drain_wait(&sh.q_full[g & 1], (g >> 1) & 1);
       }
     }
   } else if (warp == 5) {
@@ -189,7 +171,7 @@ __global__ void __launch_bounds__(192, 1)
         fwd_tile_coords(p, t, qt, bh);
         const int n_kv = fwd_n_kv(p, qt);
         const int qb = tl & 1;
-        ok = wait_bar(&sh.q_full[qb], (tl >> 1) & 1);
+        ok = mbar_wait(&sh.q_full[qb], (tl >> 1) & 1);
         if (!ok) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sQ + qb * C::kTile);
@@ -197,8 +179,8 @@ __global__ void __launch_bounds__(192, 1)
           if (s < n_kv) {
             // S(g) = Q K(g)^T into S buffer g % 3
             const int g = it + s, kst = g % C::KST, sb = g % 3;
-            ok = wait_bar(&sh.k_full[kst], (g / C::KST) & 1);
-            if (ok && g >= 3) ok = wait_bar(&sh.pv_done[sb], ((g / 3) - 1) & 1);
+            ok = mbar_wait(&sh.k_full[kst], (g / C::KST) & 1);
+            if (ok && g >= 3) ok = mbar_wait(&sh.pv_done[sb], ((g / 3) - 1) & 1);
             if (!ok) break;
             tc_fence_after();
             const uint32_t k_addr = smem_u32(sK + kst * C::kTile);
@@ -215,9 +197,9 @@ __global__ void __launch_bounds__(192, 1)
           if (s >= 1) {
             // O (+)= P(g) V(g)
             const int g = it + s - 1, vst = g % C::VST, sb = g % 3;
-            ok = wait_bar(&sh.v_full[vst], (g / C::VST) & 1);
-            if (ok) ok = wait_bar(&sh.p_ready[sb], (g / 3) & 1);
-            if (ok && s == 1 && tl >= 1) ok = wait_bar(&sh.o_free, (tl - 1) & 1);
+            ok = mbar_wait(&sh.v_full[vst], (g / C::VST) & 1);
+            if (ok) ok = mbar_wait(&sh.p_ready[sb], (g / 3) & 1);
+            if (ok && s == 1 && tl >= 1) ok = mbar_wait(&sh.o_free, (tl - 1) & 1);
             if (!ok) break;
             tc_fence_after();
             const uint32_t v_addr = smem_u32(sV + vst * C::kTile);
@@ -233,7 +215,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       // Drain every MMA this thread issued before TMEM is released.
       umma_commit(&sh.drain);
-      wait_bar(&sh.drain, 0);
+      mbar_wait(&sh.drain, 0);
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroup
@@ -247,10 +229,10 @@ __global__ void __launch_bounds__(192, 1)
       fwd_tile_coords(p, t, qt, bh);
       const int n_kv = fwd_n_kv(p, qt);
       const int qrow = qt * 128 + row;
-      float m_used = -INFINITY, l = 0.f;
+      float m_used = -INFINITY, l = 0.f, l_exact = 0.f;
       for (int j = 0; j < n_kv && ok; ++j) {
         const int g = it + j, sb = g % 3;
-        ok = __all_sync(0xffffffffu, wait_bar(&sh.s_full[sb], (g / 3) & 1));
+        ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[sb], (g / 3) & 1));
         if (!ok) break;
         tc_fence_after();
         uint32_t r[128];
@@ -277,6 +259,7 @@ __global__ void __launch_bounds__(192, 1)
           const float m_new = fmaxf(m_used, m_tile);
           alpha = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
           l *= alpha;
+          l_exact *= alpha;
           m_used = m_new;
         }
         const float neg_m = -m_used;
@@ -289,6 +272,7 @@ __global__ void __launch_bounds__(192, 1)
             const float b = ex2_approx(fmaf(__uint_as_float(r[q4 * 32 + 2 * k + 1]), c, neg_m));
             __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
             l += __low2float(h) + __high2float(h);
+            l_exact += a + b;
             pk[k] = *reinterpret_cast<uint32_t*>(&h);
           }
           tmem_st16(lane_base + sb * 128 + q4 * 16, pk);
@@ -296,7 +280,7 @@ __global__ void __launch_bounds__(192, 1)
         // Rescale the running output when this warp's max moved (rare after the first tiles).
         if (__any_sync(0xffffffffu, need && j > 0)) {
           const int gp = g - 1;
-          ok = __all_sync(0xffffffffu, wait_bar(&sh.pv_done[gp % 3], (gp / 3) & 1));
+          ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[gp % 3], (gp / 3) & 1));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -317,7 +301,7 @@ __global__ void __launch_bounds__(192, 1)
       if (!ok) break;
       // epilogue: wait for the last PV, O / l -> bf16, LSE
       const int glast = it + n_kv - 1;
-      ok = __all_sync(0xffffffffu, wait_bar(&sh.pv_done[glast % 3], (glast / 3) & 1));
+      ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[glast % 3], (glast / 3) & 1));
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
@@ -338,7 +322,7 @@ __global__ void __launch_bounds__(192, 1)
           for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      if (live) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      if (live) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + __log2f(l_exact)) * 0.69314718055994531f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.o_free);

@@ -2,7 +2,7 @@
 // mbarriers with bounded waits, TMA tile loads, tcgen05 (TMEM alloc, MMA, commit,
 // TMEM load/store) and the UMMA shared-memory / instruction descriptors.
 //
-// Every wait here is bounded: after kSpinLimit polls it records an error code
+// Every wait here is bounded: past a time limit it records an error code
 // in the device status word and returns false, so a kernel can drain and exit
 // instead of hanging the GPU.
 #pragma once
@@ -20,8 +20,6 @@ __device__ int g_attn_status = 0;
 __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
-
-constexpr uint32_t kSpinLimit = 1u << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -66,12 +64,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool status_set() {
+  return *reinterpret_cast<volatile int*>(&g_attn_status) != 0;
+}
+
+// A legitimate wait inside these kernels lasts microseconds to milliseconds;
+// anything past this bound is treated as a lost arrival.
+constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
+
+// Bounded wait for the mbarrier phase with the given parity to complete.  Gives
+// up (returns false) after kWaitTimeoutNs, recording error 1, or as soon as any
+// CTA has recorded an error.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-  record_error(status, 1);
-  return false;
+    if ((i & 63) == 0) {
+      if (status_set()) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        record_error(&g_attn_status, 1);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait used only on error paths, to let copies already in flight land.
+__device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > 100000000ull) return;
 }
 
 // ---------------------------------------------------------------- TMA
