@@ -1,0 +1,369 @@
+"""Benchmark: exact attention forward + backward TFLOPS on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: attn_fwd (O, LSE) then
+attn_bwd (dQ, dK, dV) for workloads that train, attn_fwd alone for forward-only
+ones.  Inputs are synthetic and seeded (attn_inputs), resident in HBM when the
+timed region starts, and larger than the 126 MB L2, so no flush is needed.
+Timing uses CUDA events on the launching stream, W warm-up steps, then K steps
+bracketed by a barrier and a synchronize; with N > 1 ranks each rank processes
+its own batch (independent (b, kv-head) units, no collective on the data path)
+and the max time over ranks is reported.
+
+Printed as one JSON line by rank 0.  ``--impl reference`` times the fp64 CPU
+oracle instead (the reference arm), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attn_inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+from io_aware_exact_26_b200 import accounting as acc  # noqa: E402
+
+DEFAULT_WORKLOAD = "gpt2_medium_b64_h16_n1024_d64"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "io_aware_exact_26_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload, kernel):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on this source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def time_oracle(w: Workload, budget_s: float, max_heads=None):
+    """Time the fp64 oracle on whole heads of the workload until the budget is spent.
+
+    Returns (TFLOPS, seconds, heads, threads).  Test infrastructure: only this
+    baseline leg of the benchmark runs the oracle.
+    """
+    import numpy as np
+    from attn_inputs import to_f64
+    from oracle import reference as ref
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"),
+                      default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    heads, spent, flops = 0, 0.0, 0.0
+    b = h = 0
+    while True:
+        x = make_inputs(1, 1, 1, w.N, w.d, seed=w.seed + 17 * heads, qk_std=w.qk_std, vo_std=w.vo_std,
+                        boost_frac=w.boost_frac, boost=w.boost, with_grad="bwd" in w.passes)
+        q, k, v = to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"])
+        t0 = time.perf_counter()
+        ref.ref_fwd(q, k, v, w.scale, w.causal)
+        f = acc.flops_fwd(1, 1, w.N, w.d, w.causal)
+        if "bwd" in w.passes:
+            ref.ref_bwd(q, k, v, to_f64(x["do"]), w.scale, w.causal)
+            f += acc.flops_bwd(1, 1, w.N, w.d, w.causal)
+        spent += time.perf_counter() - t0
+        flops += f
+        heads += 1
+        if spent >= budget_s or (max_heads and heads >= max_heads):
+            break
+    del b, h, np
+    return flops / spent / 1e12, spent, heads, threads
+
+
+def step_flops(w: Workload):
+    f = acc.flops_fwd(w.B, w.Hq, w.N, w.d, w.causal)
+    fb = acc.flops_bwd(w.B, w.Hq, w.N, w.d, w.causal) if "bwd" in w.passes else 0.0
+    return f, fb
+
+
+def config_dict(w: Workload, n_gpus):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+            "passes": w.passes, "scale": "1/sqrt(d)", "parallelism": f"independent replicas x{n_gpus}",
+            "l2": "inputs larger than L2 (126 MB); no flush"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle on the host cores, bounded samples per step."""
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    budget = min(2.0, max(0.2, 90.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    total_heads = 0
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        v, spent, heads, threads = time_oracle(w, budget)
+        if i >= args.warmup:
+            vals.append(v)
+            total_heads += heads
+    value = statistics.median(vals) if vals else None
+    sample = f"{total_heads} whole heads (B=1,H=1 slices of {w.name}) over {args.steps} timed steps"
+    line = {"impl": "reference", "metric": "attention fwd+bwd TFLOPS" if "bwd" in w.passes else "attention fwd TFLOPS",
+            "value": value, "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": "f64", "data": "synthetic", "config": config_dict(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import io_aware_exact_26_b200 as attn
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    w = WORKLOADS[args.workload]
+    has_bwd = "bwd" in w.passes
+    dev = torch.device("cuda", local)
+    x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed + 101 * rank, qk_std=w.qk_std, vo_std=w.vo_std,
+                    boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=has_bwd)
+    q, k, v = x["q"], x["k"], x["v"]
+    do = x.get("do")
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    if has_bwd:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(attn.attn_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.N, w.d, w.causal), dtype=torch.uint8,
+                         device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev_a=None, ev_b=None, ev_c=None):
+        if ev_a is not None:
+            ev_a.record(stream)
+        attn.attn_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal)
+        if ev_b is not None:
+            ev_b.record(stream)
+        if has_bwd:
+            attn.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale=w.scale, causal=w.causal, workspace=ws)
+        if ev_c is not None:
+            ev_c.record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if attn.attn_get_device_status() != 0:
+        raise SystemExit("device-side error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.1)
+    start.record(stream)
+    for s in range(args.steps):
+        step(*evs[s])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist:
+        dist.barrier()
+    if attn.attn_get_device_status() != 0:
+        raise SystemExit("device-side error during the timed steps")
+
+    total_ms = start.elapsed_time(stop)
+    fwd_ms = [a.elapsed_time(b) for a, b, _ in evs]
+    bwd_ms = [b.elapsed_time(c) for _, b, c in evs] if has_bwd else []
+    t = torch.tensor([total_ms, statistics.mean(fwd_ms), statistics.mean(bwd_ms) if bwd_ms else 0.0],
+                     dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_avg, bwd_avg = t.tolist()
+    ms_per_step = total_ms / args.steps
+    f_fwd, f_bwd = step_flops(w)
+    value = (f_fwd + f_bwd) * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    host = {n: x[n].cpu().pin_memory() for n in x}
+    outs_dev = {"dq": dq, "dk": dk, "dv": dv} if has_bwd else {"o": o}
+    out_host = {n: torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for n, t_ in outs_dev.items()}
+    h2d = sum(t_.numel() * t_.element_size() for t_ in host.values())
+    d2h = sum(t_.numel() * t_.element_size() for t_ in out_host.values())
+
+    def e2e_step():
+        for n in host:
+            x[n].copy_(host[n], non_blocking=True)
+        step()
+        for n, t_ in outs_dev.items():
+            out_host[n].copy_(t_, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = te.item() / args.e2e_steps
+    e2e_value = (f_fwd + f_bwd) * world / (e2e_ms * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel (backward when present)
+    peaks, peaks_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    if has_bwd and bwd_avg >= fwd_avg:
+        kname, kflops, kms = "attn_bwd (prep + main)", f_bwd, bwd_avg
+        traffic = measured_traffic(w.name, "bwd")
+    else:
+        kname, kflops, kms = "attn_fwd_kernel", f_fwd, fwd_avg
+        traffic = measured_traffic(w.name, "fwd")
+    achieved = kflops / (kms * 1e-3) / 1e12
+    roofline = {"kernel": kname, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "frac_of_sustained": round(achieved / float(peaks.get("bf16_tflops_sustained", peak)), 4),
+                "peak_source": f"{peaks_kind} bf16 dense (burst)", "traffic": traffic}
+
+    line = {"metric": "attention fwd+bwd TFLOPS" if has_bwd else "attention fwd TFLOPS",
+            "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(w, world),
+            "fwd": {"ms": round(fwd_avg, 4), "tflops": round(f_fwd / (fwd_avg * 1e-3) / 1e12, 1),
+                    "frac_of_peak": round(f_fwd / (fwd_avg * 1e-3) / 1e12 / peak, 4)},
+            "roofline": roofline,
+            "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
+            "gpu_launches": args.steps * (3 if has_bwd else 1),
+            "clocks": clocks}
+    if has_bwd:
+        line["bwd"] = {"ms": round(bwd_avg, 4), "tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 1),
+                       "frac_of_peak": round(f_bwd / (bwd_avg * 1e-3) / 1e12 / peak, 4)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, spent, heads, threads = time_oracle(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                                "sample": f"{heads} whole heads (B=1,H=1 slices of the workload), {spent:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
