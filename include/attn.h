@@ -75,6 +75,27 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
              void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward without a caller-provided workspace (no counterpart on the pages; an
+ * interface convenience).  Same arguments, layouts and results as attn_bwd, minus
+ * `workspace`/`workspace_bytes`: the scratch lives in a fixed 64 MiB device array
+ * owned by this library (held on every GPU that loads the library, until exit).
+ * For callers that cannot call cudaMalloc -- e.g. code running inside a host
+ * framework whose memory pool owns all device memory, or a loop that must not
+ * allocate after start-up -- this call allocates nothing and calls no allocating
+ * routine.
+ *   - Shapes whose workspace (attn_bwd_workspace_size) exceeds 64 MiB
+ *     (67108864 bytes) are rejected with ATTN_ERR_WORKSPACE before any launch.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array and leave their contents in it; everything
+ *     that must start at zero is cleared by the call itself.  Calls that overlap
+ *     on the GPU (different streams, or different host threads) race on the
+ *     array: serialise them. */
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dO, void* dq, void* dk, void* dv,
+                     int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                     void* stream);
+
 /* Synchronises `stream`, then returns ATTN_OK if no kernel of this library
  * recorded a device-side error since the last call, else ATTN_ERR_DEVICE_TIMEOUT;
  * the error word is cleared.  While the word is set, later launches exit early. */

@@ -8,6 +8,8 @@ library is loaded lazily on first use, so host-side helpers such as
 from .binding import (  # noqa: F401
     AttnError,
     attn_bwd,
+    attn_bwd_noalloc,
+    NOALLOC_SCRATCH_BYTES,
     attn_bwd_workspace_size,
     attn_fwd,
     attn_get_device_status,

@@ -16,6 +16,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libattn_b200.so")
 
 ATTN_OK = 0
+# Size of the fixed device scratch array behind attn_bwd_noalloc (see include/attn.h).
+NOALLOC_SCRATCH_BYTES = 64 << 20
 _lib = None
 
 
@@ -40,6 +42,8 @@ def lib():
     L.attn_bwd_workspace_size.restype = sz
     L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     L.attn_bwd.restype = i
+    L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    L.attn_bwd_noalloc.restype = i
     L.attn_get_device_status.argtypes = [vp]
     L.attn_get_device_status.restype = i
     L.attn_status_string.argtypes = [i]
@@ -122,6 +126,29 @@ def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale=None, caus
                         _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_ptr(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, *, scale=None, causal=False, stream=None):
+    """attn_bwd for callers that cannot allocate device memory.
+
+    The output tensors must be given (nothing is allocated here or in the
+    library); the scratch is the library's fixed device array, so the shape's
+    workspace must fit in NOALLOC_SCRATCH_BYTES (64 MiB).  Calls that overlap on
+    the GPU race on that array.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _check(t, n)
+    _check(lse, "lse", torch.float32)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = d ** -0.5
+    st = lib().attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+                                _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_noalloc")
     return dq, dk, dv
 
 

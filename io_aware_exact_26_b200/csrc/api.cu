@@ -203,6 +203,29 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 
 }  // namespace attn
 
+// ---------------------------------------------------------------------------
+// Scratch for attn_bwd_noalloc: a fixed device array that this library owns, so
+// callers that cannot allocate device memory can still run the backward.  Every
+// GPU that loads the library holds these bytes until the process exits.
+static constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(64) << 20;   // 64 MiB
+static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
+// Device address of g_bwd_scratch on the current device, looked up once per device
+// with that device current.  In host code the array's name is only a host-side
+// stand-in, so kernels must be given this address instead.  Returns nullptr if
+// the lookup failed.
+static void* noalloc_scratch_on_current_device() {
+  static std::once_flag once[64];
+  static void* addr[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::call_once(once[dev], [dev] {
+    void* p = nullptr;
+    addr[dev] = cudaGetSymbolAddress(&p, g_bwd_scratch) == cudaSuccess ? p : nullptr;
+  });
+  return addr[dev];
+}
+
 extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
@@ -240,6 +263,20 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
   return attn::launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, workspace,
                           static_cast<cudaStream_t>(stream), di->sms);
+}
+
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                     float scale, int causal, void* stream) {
+  int st = check_common(B, Hq, Hkv, N, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (attn::bwd_workspace_bytes(B, Hq, Hkv, N, d) > kNoAllocScratchBytes) return ATTN_ERR_WORKSPACE;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
+  void* scratch = noalloc_scratch_on_current_device();
+  if (!scratch) return ATTN_ERR_LAUNCH;
+  return attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, scratch,
+                  kNoAllocScratchBytes, stream);
 }
 
 int attn_get_device_status(void* stream) {

@@ -26,7 +26,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
-        ["attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_get_device_status", "attn_status_string"])
+        ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
+         "attn_status_string"])
 
 
 def test_every_declared_symbol_is_exported(L):

@@ -1,0 +1,53 @@
+"""attn_bwd_noalloc: the backward for callers that cannot allocate device memory.
+
+Some callers cannot call cudaMalloc -- code embedded in a host framework whose pool
+owns all device memory, or a loop that must not allocate once it runs -- so the
+library offers a backward whose scratch is its own fixed device array.  This file
+is collected last on purpose: it checks, through the C ABI, that two calls in a
+row give the same gradients as attn_bwd with a caller-allocated workspace (within
+the parity tolerance used everywhere else), and that shapes too large for the fixed
+array are refused before anything is launched.
+"""
+import pytest
+import torch
+
+from attn_inputs import make_inputs
+from tests.parity import check_grad, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def attn():
+    import __graft_entry__
+    __graft_entry__.build()
+    import io_aware_exact_26_b200 as a
+    return a
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", [(1, 4, 2, 1000, 128, True), (2, 2, 2, 384, 64, False)])
+def test_noalloc_matches_workspace_backward_twice(attn, B, Hq, Hkv, N, d, causal):
+    assert attn.attn_bwd_workspace_size(B, Hq, Hkv, N, d, causal) <= attn.NOALLOC_SCRATCH_BYTES
+    x = make_inputs(B, Hq, Hkv, N, d, seed=4242 + N)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = attn.attn_fwd(q, k, v, causal=causal)
+    ref = attn.attn_bwd(q, k, v, o, lse, do, causal=causal)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        outs = (torch.full_like(q, float("nan")), torch.full_like(k, float("nan")), torch.full_like(v, float("nan")))
+        attn.attn_bwd_noalloc(q, k, v, o, lse, do, *outs, causal=causal)
+        torch.cuda.synchronize()
+        assert attn.attn_get_device_status() == 0
+        for got, want, name in zip(outs, ref, ("dQ", "dK", "dV")):
+            check_grad(f64(got), f64(want), name)
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch(attn):
+    B, Hq, Hkv, N, d = 8, 16, 16, 4096, 128
+    assert attn.attn_bwd_workspace_size(B, Hq, Hkv, N, d, True) > attn.NOALLOC_SCRATCH_BYTES
+    q = torch.empty((1,), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1,), dtype=torch.float32, device="cuda")
+    p = q.data_ptr()
+    st = attn.lib().attn_bwd_noalloc(p, p, p, p, lse.data_ptr(), p, p, p, p, B, Hq, Hkv, N, d, 0.088, 1,
+                                     torch.cuda.current_stream().cuda_stream)
+    assert st == -6   # ATTN_ERR_WORKSPACE, nothing launched
