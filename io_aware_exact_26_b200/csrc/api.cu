@@ -144,7 +144,7 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   float* acc = reinterpret_cast<float*>(ws + L.acc_off);
   int* tickets = reinterpret_cast<int*>(ws + L.ticket_off);
   const int nt = (N + 127) / 128;
-  const long long n_tickets = BHq * nt * 4;
+  const long long n_tickets = BHq * nt * kChains * 4;
   {
     const long long rows = BHq * nt * 128;
     long long blocks = (rows * 32 + 255) / 256;
@@ -172,6 +172,7 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   p.Hkv = Hkv;
   p.N = N;
   p.G = Hq / Hkv;
+  p.BHq = BHq;
   p.nt = nt;
   p.total_items = B * Hkv * nt;
   p.c = scale * 1.4426950408889634f;
@@ -190,6 +191,15 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
     grid = p.total_items < sms ? p.total_items : sms;
   }
   attn_bwd_main_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, tdo, p);
+  if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  {
+    const long long vecs = BHq * N * (D / 8);
+    long long blocks = (vecs + 255) / 256;
+    const long long cap = static_cast<long long>(sms) * 16;
+    if (blocks > cap) blocks = cap;
+    attn_bwd_dq_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(acc, static_cast<__nv_bfloat16*>(dq), BHq,
+                                                                        N, nt, causal, scale);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 

@@ -14,19 +14,22 @@
 //   bwd_main   : persistent, one work item = (b, kv-head, 128-key tile j); K_j, V_j
 //                stay in shared memory while the item walks its G q-heads and
 //                the query tiles that see tile j (i >= j when causal).
+//   bwd_dq     : sums the dQ chains in a fixed order, scales, rounds to bf16.
 // Roles in bwd_main (320 threads):
 //   warps 0-3  "dS" warpgroup, thread = key row = TMEM lane: reads S^T and dP^T
 //              from TMEM, forms P^T (bf16, back into TMEM over S^T) and dS^T
 //              (bf16, 128B-swizzled shared memory).
-//   warps 4-7  dQ warpgroup, thread = query row: moves the dQ tile out of TMEM and
-//              adds it into the fp32 accumulator in a fixed order (tickets); the
-//              last contributor writes bf16 dq.  At the end of an item it writes
-//              dK (scaled) and dV from TMEM.
+//   warps 4-7  dQ warpgroup, thread = head-dim column of dQ^T: moves the dQ^T tile
+//              out of TMEM and adds it into the fp32 accumulator in a fixed order
+//              (tickets), one coalesced line per query row and warp; the last
+//              contributor writes bf16 dq.  At the end of an item it writes dK
+//              (scaled) and dV from TMEM (thread = key row there).
 //   warp 8     TMA producer: K_j, V_j per item; Q_i, dO_i per step (2 stages).
 //   warp 9     MMA issuer: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
-//              dK += dS^T Q, dQ = dS K.
+//              dK += dS^T Q, dQ^T = K^T dS^T.
 // The dS^T tile in shared memory is the K-major A operand of dK and, read as
-// MN-major, the A operand of dQ.
+// MN-major, the B operand of dQ^T; the K tile is the A operand of S^T (K-major)
+// and, read MN-major, of dQ^T.
 //
 // Determinism: dK and dV of an item are accumulated in TMEM by one CTA in a
 // fixed loop order.  dQ of query tile i collects one partial per key tile; the
@@ -45,6 +48,10 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
                : "memory");
 }
 
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -59,6 +66,13 @@ struct BwdLayout {
   size_t lse2_off, dd_off, acc_off, ticket_off, total;
 };
 
+// Number of independent fixed-order dQ accumulation chains per query tile.  The
+// key tiles contributing to a query tile are dealt round-robin (by their position
+// in the order) to kChains fp32 accumulators; within a chain the adds happen in a
+// fixed order, and the chains are summed in a fixed order at the end.  Consecutive
+// contributors of one chain are kChains steps apart, which hides the hand-off.
+constexpr int kChains = 4;
+
 __host__ __device__ inline BwdLayout bwd_layout(long long BHq, int N, int d) {
   const long long npad = (N + 127) / 128 * 128;
   const long long nq = npad / 128;
@@ -67,8 +81,8 @@ __host__ __device__ inline BwdLayout bwd_layout(long long BHq, int N, int d) {
   L.lse2_off = 0;
   L.dd_off = up(L.lse2_off + BHq * npad * 4);
   L.acc_off = up(L.dd_off + BHq * npad * 4);
-  L.ticket_off = up(L.acc_off + BHq * npad * d * 4);
-  L.total = up(L.ticket_off + BHq * nq * 4 * 4);
+  L.ticket_off = up(L.acc_off + static_cast<size_t>(kChains) * BHq * npad * d * 4);
+  L.total = up(L.ticket_off + BHq * nq * kChains * 4 * 4);
   return L;
 }
 
@@ -79,45 +93,49 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
 
 // ------------------------------------------------------------------ preprocess
 // D_i = sum_k dO_ik O_ik (fp32) and lse2_i = LSE_i * log2(e); padded rows get 0.
+// Each row is read with 16-byte loads by D/8 lanes, so one warp covers 256/D rows.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dO,
                                                             const float* __restrict__ lse, float* lse2,
                                                             float* dd, int* tickets, long long BHq, int N,
                                                             long long n_tickets) {
+  constexpr int LPR = D / 8;             // lanes per row
+  constexpr int RPW = 32 / LPR;          // rows per warp pass
   const int npad = (N + 127) / 128 * 128;
   const long long rows = BHq * npad;
   const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, part = lane % LPR;
   const long long warp0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long r = warp0; r < rows; r += nwarps) {
-    const long long bh = r / npad;
-    const int n = static_cast<int>(r - bh * npad);
+  for (long long r0 = warp0 * RPW; r0 < rows; r0 += nwarps * RPW) {
+    const long long r = r0 + sub;
     float acc = 0.f, l2 = 0.f;
-    if (n < N) {
-      const size_t base = (static_cast<size_t>(bh) * N + n) * D;
-      constexpr int PER = D / 32;  // elements per lane (2 or 4)
-      if constexpr (PER == 4) {
-        uint2 a = *reinterpret_cast<const uint2*>(o + base + lane * 4);
-        uint2 b = *reinterpret_cast<const uint2*>(dO + base + lane * 4);
-        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
-        for (int k = 0; k < 2; ++k) {
-          float2 fa = __bfloat1622float2(pa[k]), fb = __bfloat1622float2(pb[k]);
-          acc = fmaf(fa.x, fb.x, acc);
-          acc = fmaf(fa.y, fb.y, acc);
-        }
-      } else {
-        __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + base + lane * 2);
-        __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(dO + base + lane * 2);
-        float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-        acc = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, 0.f));
-      }
+    bool live = false;
+    long long bh = 0;
+    int n = 0;
+    if (r < rows) {
+      bh = r / npad;
+      n = static_cast<int>(r - bh * npad);
+      live = n < N;
+    }
+    if (live) {
+      const size_t base = (static_cast<size_t>(bh) * N + n) * D + part * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(o + base);
+      const uint4 b = *reinterpret_cast<const uint4*>(dO + base);
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      for (int k = 0; k < 4; ++k) {
+        const float2 fa = __bfloat1622float2(pa[k]), fb = __bfloat1622float2(pb[k]);
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+      }
       l2 = lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f;
     }
-    if (lane == 0) {
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (part == 0 && r < rows) {
       dd[r] = acc;
       lse2[r] = l2;
     }
@@ -136,6 +154,7 @@ struct BwdParams {
   float* acc;
   int* tickets;
   int B, Hq, Hkv, N, G;
+  long long BHq;
   int nt;           // number of 128-row tiles along N
   int total_items;
   int order;        // 0 = causal, 1 = linear (non-causal), 2 = cyclic (non-causal)
@@ -150,9 +169,10 @@ struct BwdCfg {
   static constexpr int kThreads = 320;
   // TMEM columns
   static constexpr int kS = 0, kDP = 128;
-  static constexpr int kDQ = (D == 128) ? 128 : 256;   // aliases dP^T when D == 128
-  static constexpr int kDV = (D == 128) ? 256 : 320;
-  static constexpr int kDK = (D == 128) ? 384 : 384;
+  // dQ^T (128 lanes = head dim, 128 columns = queries) aliases dP^T when D == 128
+  static constexpr int kDQ = (D == 128) ? 128 : 256;
+  static constexpr int kDV = (D == 128) ? 256 : 384;
+  static constexpr int kDK = (D == 128) ? 384 : 448;
   static constexpr int kTmemCols = 512;
   // shared memory (offsets from the 1024-aligned base)
   static constexpr int kOffK = 0;
@@ -186,15 +206,20 @@ __device__ __forceinline__ int bwd_steps_per_head(const BwdParams& p, int j) {
   return p.order == 0 ? (p.nt - j) : p.nt;
 }
 
-// step s of a head -> query tile i, and this key tile's position in the dQ order of tile i
-__device__ __forceinline__ void bwd_step(const BwdParams& p, int j, int s, int& i, int& pos, bool& last) {
+// step s of a head -> query tile i and this key tile's place in the dQ order of tile
+// i: global position `gpos` among the tile's contributors, its chain (gpos mod
+// kChains) and its position inside that chain (gpos / kChains).
+__device__ __forceinline__ void bwd_step(const BwdParams& p, int j, int s, int& i, int& chain, int& pos) {
+  int gpos;
   if (p.order == 0) {
-    i = j + s; pos = i - j; last = (j == 0);
+    i = j + s; gpos = i - j;
   } else if (p.order == 1) {
-    i = s; pos = p.nt - 1 - j; last = (j == 0);
+    i = s; gpos = p.nt - 1 - j;
   } else {
-    i = (j + s) % p.nt; pos = (i - j + p.nt) % p.nt; last = (pos == p.nt - 1);
+    i = (j + s) % p.nt; gpos = (i - j + p.nt) % p.nt;
   }
+  chain = gpos % kChains;
+  pos = gpos / kChains;
 }
 
 template <int D>
@@ -260,8 +285,8 @@ __global__ void __launch_bounds__(320, 1)
         for (int h = 0; h < p.G && ok; ++h) {
           const int bhq = b * p.Hq + hk * p.G + h;
           for (int s = 0; s < steps; ++s, ++gs) {
-            int i, pos; bool last;
-            bwd_step(p, j, s, i, pos, last);
+            int i, chain, pos;
+            bwd_step(p, j, s, i, chain, pos);
             const int st = gs & 1;
             if (gs >= 2) ok = mbar_wait(&sh.qdo_empty[st], ((gs >> 1) - 1) & 1);
             if (!ok) break;
@@ -287,7 +312,7 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t idST = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);   // dV, dK
-      constexpr uint32_t idQ = idesc_bf16_f32(128, D, true, true);     // dQ
+      constexpr uint32_t idQ = idesc_bf16_f32(128, 128, true, true);   // dQ^T
       int gs = 0, it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
@@ -337,7 +362,9 @@ __global__ void __launch_bounds__(320, 1)
               umma_ss(tmem + C::kDK, sdesc_sw128(ds_addr + off, 16, 1024),
                       sdesc_sw128(q_addr + k * 2048, C::kBox, 1024), idKV, !(first && k == 0));
             }
-            // dQ = dS K  (A = dS^T read MN-major, B = K MN-major; K = keys)
+            // dQ^T = K^T dS^T  (M = head dim, N = queries, K = keys; A = K read MN-major,
+            // B = dS^T read MN-major).  For D = 64 the A operand spans 128 rows: rows 64-127
+            // read the next smem tile and land in TMEM lanes 64-127, which nobody reads.
             if (D != 128 && gs >= 1) {
               ok = mbar_wait(&sh.dq_free, (gs - 1) & 1);
               if (!ok) break;
@@ -345,8 +372,8 @@ __global__ void __launch_bounds__(320, 1)
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              umma_ss(tmem + C::kDQ, sdesc_sw128(ds_addr + k * 2048, C::kBox, 1024),
-                      sdesc_sw128(k_addr + k * 2048, C::kBox, 1024), idQ, k > 0);
+              umma_ss(tmem + C::kDQ, sdesc_sw128(k_addr + k * 2048, C::kBox, 1024),
+                      sdesc_sw128(ds_addr + k * 2048, C::kBox, 1024), idQ, k > 0);
             umma_commit(&sh.dq_full);
             umma_commit(&sh.qdo_empty[st]);
             umma_commit(&sh.step_done);
@@ -375,9 +402,9 @@ __global__ void __launch_bounds__(320, 1)
       for (int h = 0; h < p.G && ok; ++h) {
         const int bhq = b * p.Hq + hk * p.G + h;
         for (int s = 0; s < steps; ++s, ++gs) {
-          int i, pos; bool last;
-          bwd_step(p, j, s, i, pos, last);
-          (void)bhq; (void)pos; (void)last;
+          int i, chain, pos;
+          bwd_step(p, j, s, i, chain, pos);
+          (void)bhq; (void)pos; (void)chain;
           const int st = gs & 1;
           const float* sLse = sVec + st * 256;
           const float* sDd = sLse + 128;
@@ -391,26 +418,48 @@ __global__ void __launch_bounds__(320, 1)
           const int qmax = p.N - 1 - qbase;                           // last valid column
           const int qmin = (p.order == 0) ? (key - qbase) : 0;        // first causal column
           const bool key_live = key < p.N;
+          // most tiles are fully visible: skip the per-element mask there (warp-uniform choice)
+          const bool full = __all_sync(0xffffffffu, key_live && qmin <= 0 && qmax >= 127);
 #pragma unroll 1
           for (int q4 = 0; q4 < 4; ++q4) {
             uint32_t sr[32], dr[32];
             tmem_ld32(lane_base + C::kS + q4 * 32, sr);
             tmem_ld32(lane_base + C::kDP + q4 * 32, dr);
+            // this chunk's 32 values of lse2 and D: same address in every thread (broadcast)
+            float lv[32], dv[32];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float4 a = reinterpret_cast<const float4*>(sLse + q4 * 32)[k];
+              const float4 b = reinterpret_cast<const float4*>(sDd + q4 * 32)[k];
+              lv[4 * k] = a.x; lv[4 * k + 1] = a.y; lv[4 * k + 2] = a.z; lv[4 * k + 3] = a.w;
+              dv[4 * k] = b.x; dv[4 * k + 1] = b.y; dv[4 * k + 2] = b.z; dv[4 * k + 3] = b.w;
+            }
             tmem_wait_ld();
             uint32_t pk[16], dk[16];
+            if (full) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              float pv[2], dv2[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int col = q4 * 32 + 2 * k + e;
-                const bool vis = key_live && col >= qmin && col <= qmax;
-                const float pe = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * k + e]), c, -sLse[col])) : 0.f;
-                pv[e] = pe;
-                dv2[e] = pe * (__uint_as_float(dr[2 * k + e]) - sDd[col]);
+              for (int k = 0; k < 16; ++k) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * k]), c, -lv[2 * k]));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * k + 1]), c, -lv[2 * k + 1]));
+                pk[k] = pack_bf16x2(p0, p1);
+                dk[k] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * k]) - dv[2 * k]),
+                                    p1 * (__uint_as_float(dr[2 * k + 1]) - dv[2 * k + 1]));
               }
-              pk[k] = pack_bf16x2(pv[0], pv[1]);
-              dk[k] = pack_bf16x2(dv2[0], dv2[1]);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                float pv[2], dv2[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int col = q4 * 32 + 2 * k + e;
+                  const bool vis = key_live && col >= qmin && col <= qmax;
+                  const float pe = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * k + e]), c, -lv[2 * k + e])) : 0.f;
+                  pv[e] = pe;
+                  dv2[e] = pe * (__uint_as_float(dr[2 * k + e]) - dv[2 * k + e]);
+                }
+                pk[k] = pack_bf16x2(pv[0], pv[1]);
+                dk[k] = pack_bf16x2(dv2[0], dv2[1]);
+              }
             }
             tmem_st16(lane_base + C::kS + q4 * 16, pk);
             // dS^T row r, queries [32 q4, 32 q4 + 32): 4 chunks of 16 bytes, 128B swizzle
@@ -432,8 +481,11 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ / epilogue warpgroup
+    // dQ^T lives in TMEM with lane = head-dim index, column = query row, so a warp's
+    // accumulator accesses for one query row are 32 consecutive floats (one line).
     const int wq = warp - 4;
-    const int r = wq * 32 + lane;
+    const int r = wq * 32 + lane;               // key row (epilogue) / head-dim index (dQ)
+    const bool dd_live = r < D;                 // D = 64: warps 6-7 carry no dQ columns
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     int gs = 0, it = 0;
     bool ok = true;
@@ -445,14 +497,14 @@ __global__ void __launch_bounds__(320, 1)
       for (int h = 0; h < p.G && ok; ++h) {
         const int bhq = b * p.Hq + hk * p.G + h;
         for (int s = 0; s < steps; ++s, ++gs) {
-          int i, pos; bool last;
-          bwd_step(p, j, s, i, pos, last);
+          int i, chain, pos;
+          bwd_step(p, j, s, i, chain, pos);
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.dq_full, gs & 1));
           if (!ok) break;
           tc_fence_after();
-          float part[D];
+          float part[128];
 #pragma unroll
-          for (int q4 = 0; q4 < D / 32; ++q4) {
+          for (int q4 = 0; q4 < 4; ++q4) {
             uint32_t x[32];
             tmem_ld32(lane_base + C::kDQ + q4 * 32, x);
             tmem_wait_ld();
@@ -462,8 +514,9 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.dq_free);
-          // wait for this warp's turn on query tile i
-          int* ticket = p.tickets + (static_cast<size_t>(bhq) * p.nt + i) * 4 + wq;
+          if (!dd_live) continue;
+          // wait for this warp's turn in its chain on query tile i
+          int* ticket = p.tickets + ((static_cast<size_t>(bhq) * p.nt + i) * kChains + chain) * 4 + wq;
           bool turn = true;
           if (pos > 0) {
             if (lane == 0) {
@@ -484,37 +537,22 @@ __global__ void __launch_bounds__(320, 1)
             turn = __shfl_sync(0xffffffffu, turn, 0);
           }
           if (!turn) { ok = false; break; }
-          const int qrow = i * 128 + r;
-          if (qrow < p.N) {
-            float* accp = p.acc + (static_cast<size_t>(bhq) * (p.nt * 128) + qrow) * D;
-            if (pos > 0) {
+          // one coalesced 128-byte line per query row and warp; the chain's first
+          // contributor stores, the others add with fire-and-forget reductions
+          const int nrows = min(128, p.N - i * 128);
+          float* accp = p.acc + ((static_cast<size_t>(chain) * p.BHq + bhq) * (p.nt * 128) + i * 128) * D + r;
+          if (pos == 0) {
 #pragma unroll
-              for (int k = 0; k < D / 4; ++k) {
-                const float4 a = reinterpret_cast<const float4*>(accp)[k];
-                part[4 * k] += a.x; part[4 * k + 1] += a.y; part[4 * k + 2] += a.z; part[4 * k + 3] += a.w;
-              }
-            }
-            if (last) {
-              __nv_bfloat16* dqp = p.dq + (static_cast<size_t>(bhq) * p.N + qrow) * D;
+            for (int q = 0; q < 128; ++q)
+              if (q < nrows) accp[static_cast<size_t>(q) * D] = part[q];
+          } else {
 #pragma unroll
-              for (int k = 0; k < D / 8; ++k)
-                reinterpret_cast<uint4*>(dqp)[k] = make_uint4(
-                    pack_bf16x2(part[8 * k] * p.scale, part[8 * k + 1] * p.scale),
-                    pack_bf16x2(part[8 * k + 2] * p.scale, part[8 * k + 3] * p.scale),
-                    pack_bf16x2(part[8 * k + 4] * p.scale, part[8 * k + 5] * p.scale),
-                    pack_bf16x2(part[8 * k + 6] * p.scale, part[8 * k + 7] * p.scale));
-            } else {
-#pragma unroll
-              for (int k = 0; k < D / 4; ++k)
-                reinterpret_cast<float4*>(accp)[k] =
-                    make_float4(part[4 * k], part[4 * k + 1], part[4 * k + 2], part[4 * k + 3]);
-            }
+            for (int q = 0; q < 128; ++q)
+              if (q < nrows) red_add_f32(accp + static_cast<size_t>(q) * D, part[q]);
           }
-          if (!last) {
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(ticket, pos + 1);
-          }
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) st_release(ticket, pos + 1);
         }
       }
       if (!ok) break;
@@ -557,6 +595,36 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ dQ convert
+// dq = bf16(scale * sum_c acc[c]) with the chains summed in order c = 0, 1, ...;
+// chain c holds a contribution for query tile i only if the tile has more than c
+// contributors (i + 1 of them when causal, nt otherwise).
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* dq,
+                                                          long long BHq, int N, int nt, int causal, float scale) {
+  const long long npad = static_cast<long long>(nt) * 128;
+  const long long vecs = BHq * N * (D / 8);
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < vecs; x += stride) {
+    const long long row = x / (D / 8);
+    const int c8 = static_cast<int>(x - row * (D / 8)) * 8;
+    const long long bh = row / N;
+    const int n = static_cast<int>(row - bh * N);
+    const int contributors = causal ? (n / 128 + 1) : nt;
+    const int nch = contributors < kChains ? contributors : kChains;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c = 0; c < nch; ++c) {
+      const float4* src = reinterpret_cast<const float4*>(acc + ((c * BHq + bh) * npad + n) * D + c8);
+      const float4 a = src[0], b = src[1];
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+    *reinterpret_cast<uint4*>(dq + row * D + c8) =
+        make_uint4(pack_bf16x2(v[0] * scale, v[1] * scale), pack_bf16x2(v[2] * scale, v[3] * scale),
+                   pack_bf16x2(v[4] * scale, v[5] * scale), pack_bf16x2(v[6] * scale, v[7] * scale));
   }
 }
 

@@ -249,9 +249,15 @@ __global__ void __launch_bounds__(192, 1)
           for (int k = 0; k < 128; ++k)
             if (k > lim) r[k] = __float_as_uint(-INFINITY);
         }
-        float mx = __uint_as_float(r[0]);
+        // row max with 8 independent chains (one warp per SMSP: no other warp hides latency)
+        float mx8[8];
 #pragma unroll
-        for (int k = 1; k < 128; ++k) mx = fmaxf(mx, __uint_as_float(r[k]));
+        for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(r[k]);
+#pragma unroll
+        for (int k = 8; k < 128; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(r[k]));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
+        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
         const float m_tile = mx * c;
         float alpha = 1.f;
         const bool need = (m_used == -INFINITY) || (m_tile > m_used + kRescaleTau);
@@ -263,6 +269,7 @@ __global__ void __launch_bounds__(192, 1)
           m_used = m_new;
         }
         const float neg_m = -m_used;
+        float lr[4] = {0.f, 0.f, 0.f, 0.f}, le[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t pk[16];
@@ -271,12 +278,14 @@ __global__ void __launch_bounds__(192, 1)
             const float a = ex2_approx(fmaf(__uint_as_float(r[q4 * 32 + 2 * k]), c, neg_m));
             const float b = ex2_approx(fmaf(__uint_as_float(r[q4 * 32 + 2 * k + 1]), c, neg_m));
             __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-            l += __low2float(h) + __high2float(h);
-            l_exact += a + b;
+            lr[k & 3] += __low2float(h) + __high2float(h);
+            le[k & 3] += a + b;
             pk[k] = *reinterpret_cast<uint32_t*>(&h);
           }
           tmem_st16(lane_base + sb * 128 + q4 * 16, pk);
         }
+        l += (lr[0] + lr[1]) + (lr[2] + lr[3]);
+        l_exact += (le[0] + le[1]) + (le[2] + le[3]);
         // Rescale the running output when this warp's max moved (rare after the first tiles).
         if (__any_sync(0xffffffffu, need && j > 0)) {
           const int gp = g - 1;
