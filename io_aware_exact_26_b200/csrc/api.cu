@@ -126,33 +126,30 @@ template <int D>
 static int launch_bwd_d(const void* q, const void* k, const void* v, const void* o, const float* lse,
                         const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, float scale,
                         int causal, void* workspace, cudaStream_t stream, int sms) {
-  using C = BwdCfg<D>;
   static std::once_flag attr_once[64];
   static bool attr_ok[64];
   int dev = 0;
   cudaGetDevice(&dev);
   std::call_once(attr_once[dev], [&] {
-    attr_ok[dev] = cudaFuncSetAttribute(attn_bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::kSmem) == cudaSuccess;
+    attr_ok[dev] = cudaFuncSetAttribute(attn_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        KvCfg<D>::kSmem) == cudaSuccess &&
+                   cudaFuncSetAttribute(attn_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        QCfg<D>::kSmem) == cudaSuccess;
   });
   if (!attr_ok[dev]) return ATTN_ERR_LAUNCH;
   const long long BHq = static_cast<long long>(B) * Hq;
-  const BwdLayout L = bwd_layout(BHq, N, D);
+  const BwdLayout L = bwd_layout(BHq, N);
   char* ws = static_cast<char*>(workspace);
   float* lse2 = reinterpret_cast<float*>(ws + L.lse2_off);
   float* dd = reinterpret_cast<float*>(ws + L.dd_off);
-  float* acc = reinterpret_cast<float*>(ws + L.acc_off);
-  int* tickets = reinterpret_cast<int*>(ws + L.ticket_off);
   const int nt = (N + 127) / 128;
-  const long long n_tickets = BHq * nt * kChains * 4;
   {
     const long long rows = BHq * nt * 128;
-    long long blocks = (rows * 32 + 255) / 256;
+    long long blocks = (rows * (D / 8) + 255) / 256;
     const long long cap = static_cast<long long>(sms) * 16;
     if (blocks > cap) blocks = cap;
     attn_bwd_prep_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dd, tickets, BHq,
-        N, n_tickets);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dd, BHq, N);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   CUtensorMap tq, tk, tv, tdo;
@@ -165,41 +162,24 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.lse2 = lse2;
   p.dd = dd;
-  p.acc = acc;
-  p.tickets = tickets;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.N = N;
   p.G = Hq / Hkv;
-  p.BHq = BHq;
   p.nt = nt;
-  p.total_items = B * Hkv * nt;
+  p.causal = causal;
   p.c = scale * 1.4426950408889634f;
   p.scale = scale;
-  int grid;
-  if (causal) {
-    p.order = 0;
-    grid = p.total_items < sms ? p.total_items : sms;
-  } else if (nt <= sms) {
-    // cyclic order: the nt items of one head run side by side, so grid is a multiple of nt
-    p.order = 2;
-    const int g = (sms / nt) * nt;
-    grid = p.total_items < g ? p.total_items : g;
-  } else {
-    p.order = 1;
-    grid = p.total_items < sms ? p.total_items : sms;
-  }
-  attn_bwd_main_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, tdo, p);
+  // dK, dV: one item per (b, kv-head, key tile)
+  p.total_items = B * Hkv * nt;
+  int grid = p.total_items < sms ? p.total_items : sms;
+  attn_bwd_kv_kernel<D><<<grid, KvCfg<D>::kThreads, KvCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
   if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  {
-    const long long vecs = BHq * N * (D / 8);
-    long long blocks = (vecs + 255) / 256;
-    const long long cap = static_cast<long long>(sms) * 16;
-    if (blocks > cap) blocks = cap;
-    attn_bwd_dq_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(acc, static_cast<__nv_bfloat16*>(dq), BHq,
-                                                                        N, nt, causal, scale);
-  }
+  // dQ: one item per (b, q-head, query tile)
+  p.total_items = B * Hq * nt;
+  grid = p.total_items < sms ? p.total_items : sms;
+  attn_bwd_q_kernel<D><<<grid, QCfg<D>::kThreads, QCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 

@@ -2,39 +2,28 @@
 //
 // Recompute instead of store (page "attention 的显存线性化" §五; page
 // "attn-efficient", recompute paragraph): the forward keeps only O and the
-// log-sum-exp; here every S/P tile is rebuilt on chip from Q, K and the saved
-// LSE.  Gradient formulas (chain rule through the row softmax; the pages state
-// none): with D_i = sum_k dO_ik O_ik,
+// log-sum-exp; every S/P tile is rebuilt on chip from Q, K and the saved LSE.
+// Gradient formulas (chain rule through the row softmax; the pages state none):
+// with D_i = sum_k dO_ik O_ik,
 //   P = exp(scale Q K^T - LSE),  dV = P^T dO,  dP = dO V^T,
 //   dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Kernels
-//   bwd_prep   : one warp per query row: D_i and LSE in log2 units; zeroes the
-//                dQ ordering tickets.
-//   bwd_main   : persistent, one work item = (b, kv-head, 128-key tile j); K_j, V_j
-//                stay in shared memory while the item walks its G q-heads and
-//                the query tiles that see tile j (i >= j when causal).
-//   bwd_dq     : sums the dQ chains in a fixed order, scales, rounds to bf16.
-// Roles in bwd_main (320 threads):
-//   warps 0-3  "dS" warpgroup, thread = key row = TMEM lane: reads S^T and dP^T
-//              from TMEM, forms P^T (bf16, back into TMEM over S^T) and dS^T
-//              (bf16, 128B-swizzled shared memory).
-//   warps 4-7  dQ warpgroup, thread = head-dim column of dQ^T: moves the dQ^T tile
-//              out of TMEM and adds it into the fp32 accumulator in a fixed order
-//              (tickets), one coalesced line per query row and warp; the last
-//              contributor writes bf16 dq.  At the end of an item it writes dK
-//              (scaled) and dV from TMEM (thread = key row there).
-//   warp 8     TMA producer: K_j, V_j per item; Q_i, dO_i per step (2 stages).
-//   warp 9     MMA issuer: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
-//              dK += dS^T Q, dQ^T = K^T dS^T.
-// The dS^T tile in shared memory is the K-major A operand of dK and, read as
-// MN-major, the B operand of dQ^T; the K tile is the A operand of S^T (K-major)
-// and, read MN-major, of dQ^T.
+//   bwd_prep : one row per D/8 lanes: D_i and LSE in log2 units.
+//   bwd_kv   : persistent; one work item = (b, kv-head, 128-key tile j).  K_j, V_j
+//              stay in shared memory while the item walks its G q-heads and the
+//              query tiles that see tile j; dK_j and dV_j accumulate in TMEM and are
+//              written once.
+//   bwd_q    : persistent; one work item = (b, q-head, 128-query tile i).  Q_i, dO_i
+//              stay in shared memory while the item walks the key tiles tile i sees;
+//              dQ_i accumulates in TMEM and is written once.
+// Splitting dQ from dK/dV costs a second recompute of S and dP (7 instead of 5
+// tile contractions per query/key tile pair) but removes every cross-CTA
+// reduction: no atomics, no ordering, no fp32 scratch for dQ, and each output is
+// summed by one CTA in a fixed order, so results are bitwise reproducible.
 //
-// Determinism: dK and dV of an item are accumulated in TMEM by one CTA in a
-// fixed loop order.  dQ of query tile i collects one partial per key tile; the
-// partials are added in a fixed order of key tiles (position below) enforced by
-// per-(tile, warp) tickets, so the fp32 sums are bitwise reproducible.
+// Every tcgen05.mma here has M = 128 and N >= 128 where the head dim allows it
+// (an M = 128, N = 64 MMA takes as long as N = 128 on this part).
 #pragma once
 #include "sm100.cuh"
 
@@ -48,47 +37,25 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
                : "memory");
 }
 
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
-}
-
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 struct BwdLayout {
-  // workspace carve-up (byte offsets, each 256-byte aligned)
-  size_t lse2_off, dd_off, acc_off, ticket_off, total;
+  // workspace carve-up (byte offsets, each 256-byte aligned): lse2 and D per row
+  size_t lse2_off, dd_off, total;
 };
 
-// Number of independent fixed-order dQ accumulation chains per query tile.  The
-// key tiles contributing to a query tile are dealt round-robin (by their position
-// in the order) to kChains fp32 accumulators; within a chain the adds happen in a
-// fixed order, and the chains are summed in a fixed order at the end.  Consecutive
-// contributors of one chain are kChains steps apart, which hides the hand-off.
-constexpr int kChains = 4;
-
-__host__ __device__ inline BwdLayout bwd_layout(long long BHq, int N, int d) {
+__host__ __device__ inline BwdLayout bwd_layout(long long BHq, int N) {
   const long long npad = (N + 127) / 128 * 128;
-  const long long nq = npad / 128;
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   BwdLayout L;
   L.lse2_off = 0;
   L.dd_off = up(L.lse2_off + BHq * npad * 4);
-  L.acc_off = up(L.dd_off + BHq * npad * 4);
-  L.ticket_off = up(L.acc_off + static_cast<size_t>(kChains) * BHq * npad * d * 4);
-  L.total = up(L.ticket_off + BHq * nq * kChains * 4 * 4);
+  L.total = up(L.dd_off + BHq * npad * 4);
   return L;
 }
 
 inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   (void)Hkv;
-  return bwd_layout(static_cast<long long>(B) * Hq, N, d).total;
+  (void)d;
+  return bwd_layout(static_cast<long long>(B) * Hq, N).total;
 }
 
 // ------------------------------------------------------------------ preprocess
@@ -98,8 +65,7 @@ template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dO,
                                                             const float* __restrict__ lse, float* lse2,
-                                                            float* dd, int* tickets, long long BHq, int N,
-                                                            long long n_tickets) {
+                                                            float* dd, long long BHq, int N) {
   constexpr int LPR = D / 8;             // lanes per row
   constexpr int RPW = 32 / LPR;          // rows per warp pass
   const int npad = (N + 127) / 128 * 128;
@@ -140,120 +106,108 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
       lse2[r] = l2;
     }
   }
-  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (long long t = tid; t < n_tickets; t += static_cast<long long>(gridDim.x) * blockDim.x) tickets[t] = 0;
 }
 
-// ------------------------------------------------------------------ main kernel
 struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   const float* lse2;
   const float* dd;
-  float* acc;
-  int* tickets;
   int B, Hq, Hkv, N, G;
-  long long BHq;
   int nt;           // number of 128-row tiles along N
   int total_items;
-  int order;        // 0 = causal, 1 = linear (non-causal), 2 = cyclic (non-causal)
+  int causal;
   float c;          // scale * log2(e)
   float scale;
 };
 
+// Exps of one 16-column slice of a score tile held by this thread: p = 2^(s c - l).
+// Masked columns (only on diagonal / ragged tiles) get s = -inf first, so p = 0
+// exactly; the exp loop itself has no branch.
+__device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const float (&lv)[16], float c, bool masked,
+                                          int col0, int lo, int hi, float* pf) {
+  if (masked) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (col0 + k < lo || col0 + k > hi) sr[k] = 0xff800000u;
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) pf[k] = ex2_approx(fmaf(__uint_as_float(sr[k]), c, -lv[k]));
+}
+
+// ================================================================== bwd_kv
 template <int D>
-struct BwdCfg {
+struct KvCfg {
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kBox = 128 * 128;
   static constexpr int kThreads = 320;
-  // TMEM columns
-  static constexpr int kS = 0, kDP = 128;
-  // dQ^T (128 lanes = head dim, 128 columns = queries) aliases dP^T when D == 128
-  static constexpr int kDQ = (D == 128) ? 128 : 256;
-  static constexpr int kDV = (D == 128) ? 256 : 384;
-  static constexpr int kDK = (D == 128) ? 384 : 448;
+  // TMEM columns: S^T (lane = key, column = query), P^T as bf16 over it (queries
+  // 0-63 in columns 0-31, queries 64-127 in columns 64-95: each dS warpgroup
+  // overwrites only columns it has read); dP^T with dS^T as bf16 over it (same
+  // placement); dV and dK accumulators (D columns each).
+  static constexpr int kS = 0, kDP = 128, kDV = 256, kDK = 256 + D;
   static constexpr int kTmemCols = 512;
-  // shared memory (offsets from the 1024-aligned base)
-  static constexpr int kOffK = 0;
-  static constexpr int kOffV = kTile;
-  static constexpr int kOffQ = 2 * kTile;                // 2 stages of Q
-  static constexpr int kOffDO = 4 * kTile;               // 2 stages of dO
-  static constexpr int kOffDS = 6 * kTile;               // dS^T, 128 x 128 bf16
-  static constexpr int kOffVec = kOffDS + 32768;         // per stage: lse2[128], dd[128]
-  static constexpr int kOffBar = kOffVec + 2048;         // BwdShared
+  static constexpr int kOffK = 0, kOffV = kTile;
+  static constexpr int kOffQ = 2 * kTile;                // 2 stages
+  static constexpr int kOffDO = 4 * kTile;               // 2 stages
+  static constexpr int kOffVec = 6 * kTile;              // per stage: lse2[128], dd[128]
+  static constexpr int kOffBar = kOffVec + 2048;
   static constexpr int kLayout = kOffBar + 256;
-  // request what the layout needs plus alignment slack, capped at the opt-in maximum
-  static constexpr int kSmem = (kLayout + 1024 <= 232448) ? kLayout + 1024 : 232448;
+  static constexpr int kSmem = kLayout + 1024;
 };
 
-struct BwdShared {
+struct KvShared {
   uint64_t kv_full, kv_empty;
   uint64_t qdo_full[2], qdo_empty[2];
-  uint64_t st_full, ds_ready, step_done, dq_full, dq_free, acc_free;
+  uint64_t s_full, dp_full;     // S^T / dP^T of the step in TMEM
+  uint64_t p_ready, ds_ready;   // P^T / dS^T (bf16) written back by both dS warpgroups
+  uint64_t v_done, k_done;      // dV / dK MMA of the step complete
+  uint64_t acc_free;            // dV / dK of the previous item read out
   uint64_t drain;
   uint32_t tmem_base;
 };
 
-// item t -> (bh_kv, key tile j)
-__device__ __forceinline__ void bwd_item(const BwdParams& p, int t, int& bhkv, int& j) {
-  bhkv = t / p.nt;
-  const int r = t - bhkv * p.nt;
-  j = (p.order == 2) ? r : (p.nt - 1 - r);
+// item t -> (bh_kv, key tile j); key tile outermost, so the key tiles with the most
+// query tiles (causal) come first
+__device__ __forceinline__ void kv_item(const BwdParams& p, int t, int& bhkv, int& j) {
+  const int BHkv = p.B * p.Hkv;
+  const int r = t / BHkv;
+  bhkv = t - r * BHkv;
+  j = r;
 }
-
-__device__ __forceinline__ int bwd_steps_per_head(const BwdParams& p, int j) {
-  return p.order == 0 ? (p.nt - j) : p.nt;
-}
-
-// step s of a head -> query tile i and this key tile's place in the dQ order of tile
-// i: global position `gpos` among the tile's contributors, its chain (gpos mod
-// kChains) and its position inside that chain (gpos / kChains).
-__device__ __forceinline__ void bwd_step(const BwdParams& p, int j, int s, int& i, int& chain, int& pos) {
-  int gpos;
-  if (p.order == 0) {
-    i = j + s; gpos = i - j;
-  } else if (p.order == 1) {
-    i = s; gpos = p.nt - 1 - j;
-  } else {
-    i = (j + s) % p.nt; gpos = (i - j + p.nt) % p.nt;
-  }
-  chain = gpos % kChains;
-  pos = gpos / kChains;
-}
+__device__ __forceinline__ int kv_first_q(const BwdParams& p, int j) { return p.causal ? j : 0; }
 
 template <int D>
 __global__ void __launch_bounds__(320, 1)
-    attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                         const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
-                         const BwdParams p) {
-  using C = BwdCfg<D>;
+    attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
+                       const BwdParams p) {
+  using C = KvCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if (static_cast<int>(smem - smem_raw) + C::kLayout > C::kSmem) {
-    // the 128B-swizzled tiles need a 1024-byte aligned base that this launch cannot give
-    if (threadIdx.x == 0) record_error(&g_attn_status, 3);
-    return;
-  }
-  BwdShared& sh = *reinterpret_cast<BwdShared*>(smem + C::kOffBar);
+  KvShared& sh = *reinterpret_cast<KvShared*>(smem + C::kOffBar);
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sDO = smem + C::kOffDO;
-  uint8_t* sDS = smem + C::kOffDS;
   float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);   // [stage][lse2 128 | dd 128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(&sh.kv_full, 1);
     mbar_init(&sh.kv_empty, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&sh.qdo_full[i], 1); mbar_init(&sh.qdo_empty[i], 1); }
-    mbar_init(&sh.st_full, 1);
-    mbar_init(&sh.ds_ready, 4);
-    mbar_init(&sh.step_done, 1);
-    mbar_init(&sh.dq_full, 1);
-    mbar_init(&sh.dq_free, 4);
-    mbar_init(&sh.acc_free, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.qdo_full[i], 1);
+      mbar_init(&sh.qdo_empty[i], 1);
+    }
+    mbar_init(&sh.s_full, 1);
+    mbar_init(&sh.dp_full, 1);
+    mbar_init(&sh.p_ready, 8);
+    mbar_init(&sh.ds_ready, 8);
+    mbar_init(&sh.v_done, 1);
+    mbar_init(&sh.k_done, 1);
+    mbar_init(&sh.acc_free, 8);
     mbar_init(&sh.drain, 1);
     fence_barrier_init();
   }
@@ -271,7 +225,7 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
         int bhkv, j;
-        bwd_item(p, t, bhkv, j);
+        kv_item(p, t, bhkv, j);
         if (it >= 1) ok = mbar_wait(&sh.kv_empty, (it - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&sh.kv_full, 2 * C::kTile);
@@ -281,12 +235,9 @@ __global__ void __launch_bounds__(320, 1)
         }
         nkv = it + 1;
         const int b = bhkv / p.Hkv, hk = bhkv - b * p.Hkv;
-        const int steps = bwd_steps_per_head(p, j);
         for (int h = 0; h < p.G && ok; ++h) {
           const int bhq = b * p.Hq + hk * p.G + h;
-          for (int s = 0; s < steps; ++s, ++gs) {
-            int i, chain, pos;
-            bwd_step(p, j, s, i, chain, pos);
+          for (int i = kv_first_q(p, j); i < p.nt; ++i, ++gs) {
             const int st = gs & 1;
             if (gs >= 2) ok = mbar_wait(&sh.qdo_empty[st], ((gs >> 1) - 1) & 1);
             if (!ok) break;
@@ -309,76 +260,76 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // Order per step g:  dV(g) S^T(g+1) dK(g) dP^T(g+1).  The exps of step g+1
+    // (phase A) run under dK(g) and dP^T(g+1); dS of step g (phase B) under dV(g)
+    // and S^T(g+1).
     if (lane == 0) {
-      constexpr uint32_t idST = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);   // dV, dK
-      constexpr uint32_t idQ = idesc_bf16_f32(128, 128, true, true);   // dQ^T
+      constexpr uint32_t idST = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);      // dV, dK
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       int gs = 0, it = 0;
       bool ok = true;
+      auto issue_st = [&](int g) -> bool {   // S^T(g) = K Q(g)^T
+        const int st = g & 1;
+        if (!mbar_wait(&sh.qdo_full[st], (g >> 1) & 1)) return false;
+        if (g >= 1 && !mbar_wait(&sh.v_done, (g - 1) & 1)) return false;      // P^T(g-1) consumed
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sQ + st * C::kTile);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+          umma_ss(tmem + C::kS, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idST,
+                  k > 0);
+        }
+        umma_commit(&sh.s_full);
+        return true;
+      };
+      auto issue_dp = [&](int g) -> bool {   // dP^T(g) = V dO(g)^T
+        const int st = g & 1;
+        if (g >= 1 && !mbar_wait(&sh.k_done, (g - 1) & 1)) return false;      // dS^T(g-1) consumed
+        tc_fence_after();
+        const uint32_t do_addr = smem_u32(sDO + st * C::kTile);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+          umma_ss(tmem + C::kDP, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
+                  idST, k > 0);
+        }
+        umma_commit(&sh.dp_full);
+        return true;
+      };
       for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
         int bhkv, j;
-        bwd_item(p, t, bhkv, j);
+        kv_item(p, t, bhkv, j);
         ok = mbar_wait(&sh.kv_full, it & 1);
         if (!ok) break;
-        const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), ds_addr = smem_u32(sDS);
-        const int steps = bwd_steps_per_head(p, j);
-        bool first = true;
-        for (int h = 0; h < p.G && ok; ++h) {
-          for (int s = 0; s < steps; ++s, ++gs) {
-            const int st = gs & 1;
-            ok = mbar_wait(&sh.qdo_full[st], (gs >> 1) & 1);
-            if (ok && gs >= 1) ok = mbar_wait(&sh.step_done, (gs - 1) & 1);
-            if (ok && D == 128 && gs >= 1) ok = mbar_wait(&sh.dq_free, (gs - 1) & 1);  // dQ aliases dP^T
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t q_addr = smem_u32(sQ + st * C::kTile), do_addr = smem_u32(sDO + st * C::kTile);
-            // S^T = K Q^T and dP^T = V dO^T  (M = keys, N = queries, K = head dim)
+        const int n_steps = p.G * (p.nt - kv_first_q(p, j));
+        ok = issue_st(gs) && issue_dp(gs);
+        for (int u = 0; u < n_steps && ok; ++u, ++gs) {
+          const int st = gs & 1;
+          const uint32_t q_addr = smem_u32(sQ + st * C::kTile), do_addr = smem_u32(sDO + st * C::kTile);
+          // dV += P^T dO  (A = P^T in TMEM, K = queries; B = dO MN-major)
+          ok = mbar_wait(&sh.p_ready, gs & 1);
+          if (ok && u == 0 && it >= 1) ok = mbar_wait(&sh.acc_free, (it - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-              umma_ss(tmem + C::kS, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idST,
-                      k > 0);
-            }
+          for (int k = 0; k < 8; ++k)
+            umma_ts(tmem + C::kDV, tmem + C::kS + (k >> 2) * 64 + (k & 3) * 8,
+                    sdesc_sw128(do_addr + k * 2048, C::kBox, 1024), idKV, !(u == 0 && k == 0));
+          umma_commit(&sh.v_done);
+          if (u + 1 < n_steps && !issue_st(gs + 1)) { ok = false; break; }
+          // dK += dS^T Q  (A = dS^T in TMEM; B = Q MN-major)
+          ok = mbar_wait(&sh.ds_ready, gs & 1);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-              umma_ss(tmem + C::kDP, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
-                      idST, k > 0);
-            }
-            umma_commit(&sh.st_full);
-            ok = mbar_wait(&sh.ds_ready, gs & 1);
-            if (ok && first && it >= 1) ok = mbar_wait(&sh.acc_free, (it - 1) & 1);
-            if (!ok) break;
-            tc_fence_after();
-            // dV += P^T dO  (A = P^T from TMEM, B = dO MN-major; K = queries)
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              umma_ts(tmem + C::kDV, tmem + C::kS + k * 8, sdesc_sw128(do_addr + k * 2048, C::kBox, 1024), idKV,
-                      !(first && k == 0));
-            // dK += dS^T Q  (A = dS^T K-major smem, B = Q MN-major)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-              umma_ss(tmem + C::kDK, sdesc_sw128(ds_addr + off, 16, 1024),
-                      sdesc_sw128(q_addr + k * 2048, C::kBox, 1024), idKV, !(first && k == 0));
-            }
-            // dQ^T = K^T dS^T  (M = head dim, N = queries, K = keys; A = K read MN-major,
-            // B = dS^T read MN-major).  For D = 64 the A operand spans 128 rows: rows 64-127
-            // read the next smem tile and land in TMEM lanes 64-127, which nobody reads.
-            if (D != 128 && gs >= 1) {
-              ok = mbar_wait(&sh.dq_free, (gs - 1) & 1);
-              if (!ok) break;
-              tc_fence_after();
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              umma_ss(tmem + C::kDQ, sdesc_sw128(k_addr + k * 2048, C::kBox, 1024),
-                      sdesc_sw128(ds_addr + k * 2048, C::kBox, 1024), idQ, k > 0);
-            umma_commit(&sh.dq_full);
-            umma_commit(&sh.qdo_empty[st]);
-            umma_commit(&sh.step_done);
-            first = false;
-          }
+          for (int k = 0; k < 8; ++k)
+            umma_ts(tmem + C::kDK, tmem + C::kDP + (k >> 2) * 64 + (k & 3) * 8,
+                    sdesc_sw128(q_addr + k * 2048, C::kBox, 1024), idKV, !(u == 0 && k == 0));
+          umma_commit(&sh.k_done);
+          umma_commit(&sh.qdo_empty[st]);
+          if (u + 1 < n_steps && !issue_dp(gs + 1)) { ok = false; break; }
         }
         if (!ok) break;
         umma_commit(&sh.kv_empty);
@@ -386,202 +337,108 @@ __global__ void __launch_bounds__(320, 1)
       umma_commit(&sh.drain);
       mbar_wait(&sh.drain, 0);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ dS warpgroup (rows = keys)
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  } else {
+    // ------------------------------------------------------------ dS warpgroups (rows = keys)
+    // warps 0-3: queries 0-63 of every step and the dV epilogue; warps 4-7: queries
+    // 64-127 and the dK epilogue.
+    const int hb = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.c;
     int gs = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x) {
       int bhkv, j;
-      bwd_item(p, t, bhkv, j);
-      const int b = bhkv / p.Hkv, hk = bhkv - b * p.Hkv;
-      const int steps = bwd_steps_per_head(p, j);
+      kv_item(p, t, bhkv, j);
       const int key = j * 128 + r;
+      const bool key_live = key < p.N;
       for (int h = 0; h < p.G && ok; ++h) {
-        const int bhq = b * p.Hq + hk * p.G + h;
-        for (int s = 0; s < steps; ++s, ++gs) {
-          int i, chain, pos;
-          bwd_step(p, j, s, i, chain, pos);
-          (void)bhq; (void)pos; (void)chain;
+        for (int i = kv_first_q(p, j); i < p.nt && ok; ++i, ++gs) {
           const int st = gs & 1;
-          const float* sLse = sVec + st * 256;
+          const float* sLse = sVec + st * 256 + 64 * hb;
           const float* sDd = sLse + 128;
+          // visible query columns (relative to this warpgroup's 64) for this key row
+          const int qbase = i * 128 + 64 * hb;
+          const int hi = key_live ? (p.N - 1 - qbase) : -1;
+          const int lo = p.causal ? (key - qbase) : 0;
+          const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= 63);
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.qdo_full[st], (gs >> 1) & 1));
-          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.st_full, gs & 1));
-          if (ok && gs >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&sh.step_done, (gs - 1) & 1));
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full, gs & 1));
           if (!ok) break;
           tc_fence_after();
-          // visible queries of this key row: causal needs query >= key; both need < N
-          const int qbase = i * 128;
-          const int qmax = p.N - 1 - qbase;                           // last valid column
-          const int qmin = (p.order == 0) ? (key - qbase) : 0;        // first causal column
-          const bool key_live = key < p.N;
-          // most tiles are fully visible: skip the per-element mask there (warp-uniform choice)
-          const bool full = __all_sync(0xffffffffu, key_live && qmin <= 0 && qmax >= 127);
-#pragma unroll 1
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t sr[32], dr[32];
-            tmem_ld32(lane_base + C::kS + q4 * 32, sr);
-            tmem_ld32(lane_base + C::kDP + q4 * 32, dr);
-            // this chunk's 32 values of lse2 and D: same address in every thread (broadcast)
-            float lv[32], dv[32];
+          // ---- phase A: P^T = exp2(S^T c - lse2); bf16 into TMEM, fp32 kept for phase B
+          float pf[64];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const float4 a = reinterpret_cast<const float4*>(sLse + q4 * 32)[k];
-              const float4 b = reinterpret_cast<const float4*>(sDd + q4 * 32)[k];
+          for (int q16 = 0; q16 < 4; ++q16) {
+            uint32_t sr[16];
+            tmem_ld16(lane_base + C::kS + 64 * hb + q16 * 16, sr);
+            float lv[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float4 a = reinterpret_cast<const float4*>(sLse + q16 * 16)[k];
               lv[4 * k] = a.x; lv[4 * k + 1] = a.y; lv[4 * k + 2] = a.z; lv[4 * k + 3] = a.w;
+            }
+            tmem_wait_ld();
+            bwd_exp16(sr, lv, c, masked, q16 * 16, lo, hi, pf + q16 * 16);
+            uint32_t pk[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k], pf[q16 * 16 + 2 * k + 1]);
+            tmem_st8(lane_base + C::kS + 64 * hb + q16 * 8, pk);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.p_ready);
+          // ---- phase B: dS^T = P^T (dP^T - D); bf16 into TMEM over dP^T
+          ok = __all_sync(0xffffffffu, mbar_wait(&sh.dp_full, gs & 1));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int q16 = 0; q16 < 4; ++q16) {
+            uint32_t dr[16];
+            tmem_ld16(lane_base + C::kDP + 64 * hb + q16 * 16, dr);
+            float dv[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float4 b = reinterpret_cast<const float4*>(sDd + q16 * 16)[k];
               dv[4 * k] = b.x; dv[4 * k + 1] = b.y; dv[4 * k + 2] = b.z; dv[4 * k + 3] = b.w;
             }
             tmem_wait_ld();
-            uint32_t pk[16], dk[16];
-            if (full) {
+            uint32_t dk[8];
 #pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * k]), c, -lv[2 * k]));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * k + 1]), c, -lv[2 * k + 1]));
-                pk[k] = pack_bf16x2(p0, p1);
-                dk[k] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * k]) - dv[2 * k]),
-                                    p1 * (__uint_as_float(dr[2 * k + 1]) - dv[2 * k + 1]));
-              }
-            } else {
-#pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                float pv[2], dv2[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                  const int col = q4 * 32 + 2 * k + e;
-                  const bool vis = key_live && col >= qmin && col <= qmax;
-                  const float pe = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * k + e]), c, -lv[2 * k + e])) : 0.f;
-                  pv[e] = pe;
-                  dv2[e] = pe * (__uint_as_float(dr[2 * k + e]) - dv[2 * k + e]);
-                }
-                pk[k] = pack_bf16x2(pv[0], pv[1]);
-                dk[k] = pack_bf16x2(dv2[0], dv2[1]);
-              }
-            }
-            tmem_st16(lane_base + C::kS + q4 * 16, pk);
-            // dS^T row r, queries [32 q4, 32 q4 + 32): 4 chunks of 16 bytes, 128B swizzle
-            uint8_t* rowp = sDS + (q4 >> 1) * C::kBox + r * 128;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-              const int chunk = (q4 & 1) * 4 + ch;
-              *reinterpret_cast<uint4*>(rowp + ((chunk ^ (r & 7)) << 4)) =
-                  make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
-            }
+            for (int k = 0; k < 8; ++k)
+              dk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k] * (__uint_as_float(dr[2 * k]) - dv[2 * k]),
+                                  pf[q16 * 16 + 2 * k + 1] * (__uint_as_float(dr[2 * k + 1]) - dv[2 * k + 1]));
+            tmem_st8(lane_base + C::kDP + 64 * hb + q16 * 8, dk);
           }
-          fence_proxy_async_smem();
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.ds_ready);
         }
       }
-    }
-  } else {
-    // ------------------------------------------------------------ dQ / epilogue warpgroup
-    // dQ^T lives in TMEM with lane = head-dim index, column = query row, so a warp's
-    // accumulator accesses for one query row are 32 consecutive floats (one line).
-    const int wq = warp - 4;
-    const int r = wq * 32 + lane;               // key row (epilogue) / head-dim index (dQ)
-    const bool dd_live = r < D;                 // D = 64: warps 6-7 carry no dQ columns
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    int gs = 0, it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
-      int bhkv, j;
-      bwd_item(p, t, bhkv, j);
-      const int b = bhkv / p.Hkv, hk = bhkv - b * p.Hkv;
-      const int steps = bwd_steps_per_head(p, j);
-      for (int h = 0; h < p.G && ok; ++h) {
-        const int bhq = b * p.Hq + hk * p.G + h;
-        for (int s = 0; s < steps; ++s, ++gs) {
-          int i, chain, pos;
-          bwd_step(p, j, s, i, chain, pos);
-          ok = __all_sync(0xffffffffu, mbar_wait(&sh.dq_full, gs & 1));
-          if (!ok) break;
-          tc_fence_after();
-          float part[128];
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t x[32];
-            tmem_ld32(lane_base + C::kDQ + q4 * 32, x);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) part[q4 * 32 + k] = __uint_as_float(x[k]);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.dq_free);
-          if (!dd_live) continue;
-          // wait for this warp's turn in its chain on query tile i
-          int* ticket = p.tickets + ((static_cast<size_t>(bhq) * p.nt + i) * kChains + chain) * 4 + wq;
-          bool turn = true;
-          if (pos > 0) {
-            if (lane == 0) {
-              turn = false;
-              const uint64_t t0 = globaltimer_ns();
-              for (uint32_t spin = 0;; ++spin) {
-                if (ld_acquire(ticket) == pos) { turn = true; break; }
-                if ((spin & 15) == 15) {
-                  if (status_set()) break;
-                  if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-                    record_error(&g_attn_status, 2);
-                    break;
-                  }
-                  __nanosleep(32);
-                }
-              }
-            }
-            turn = __shfl_sync(0xffffffffu, turn, 0);
-          }
-          if (!turn) { ok = false; break; }
-          // one coalesced 128-byte line per query row and warp; the chain's first
-          // contributor stores, the others add with fire-and-forget reductions
-          const int nrows = min(128, p.N - i * 128);
-          float* accp = p.acc + ((static_cast<size_t>(chain) * p.BHq + bhq) * (p.nt * 128) + i * 128) * D + r;
-          if (pos == 0) {
-#pragma unroll
-            for (int q = 0; q < 128; ++q)
-              if (q < nrows) accp[static_cast<size_t>(q) * D] = part[q];
-          } else {
-#pragma unroll
-            for (int q = 0; q < 128; ++q)
-              if (q < nrows) red_add_f32(accp + static_cast<size_t>(q) * D, part[q]);
-          }
-          __threadfence();
-          __syncwarp();
-          if (lane == 0) st_release(ticket, pos + 1);
-        }
-      }
       if (!ok) break;
-      // epilogue of the item: dV and scale * dK rows (TMEM lane = key)
-      ok = __all_sync(0xffffffffu, mbar_wait(&sh.step_done, (gs - 1) & 1));
+      // epilogue of the item (TMEM lane = key): warps 0-3 write dV, warps 4-7 scale * dK
+      ok = __all_sync(0xffffffffu, mbar_wait(&sh.k_done, (gs - 1) & 1));
       if (!ok) break;
       tc_fence_after();
-      const int key = j * 128 + r;
       const bool live = key < p.N;
-      const size_t krow = (static_cast<size_t>(bhkv) * p.N + key) * D;
+      const float mul = hb == 0 ? 1.f : p.scale;
+      __nv_bfloat16* dst = (hb == 0 ? p.dv : p.dk) + (static_cast<size_t>(bhkv) * p.N + key) * D;
+      const uint32_t col = hb == 0 ? C::kDV : C::kDK;
+#pragma unroll 1
+      for (int q4 = 0; q4 < D / 32; ++q4) {
+        uint32_t x[32];
+        tmem_ld32(lane_base + col + q4 * 32, x);
+        tmem_wait_ld();
+        if (live) {
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const float mul = which == 0 ? 1.f : p.scale;
-        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + krow;
-        const uint32_t col = which == 0 ? C::kDV : C::kDK;
-#pragma unroll
-        for (int q4 = 0; q4 < D / 32; ++q4) {
-          uint32_t x[32];
-          tmem_ld32(lane_base + col + q4 * 32, x);
-          tmem_wait_ld();
-          if (live) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              reinterpret_cast<uint4*>(dst + q4 * 32)[k] = make_uint4(
-                  pack_bf16x2(__uint_as_float(x[8 * k]) * mul, __uint_as_float(x[8 * k + 1]) * mul),
-                  pack_bf16x2(__uint_as_float(x[8 * k + 2]) * mul, __uint_as_float(x[8 * k + 3]) * mul),
-                  pack_bf16x2(__uint_as_float(x[8 * k + 4]) * mul, __uint_as_float(x[8 * k + 5]) * mul),
-                  pack_bf16x2(__uint_as_float(x[8 * k + 6]) * mul, __uint_as_float(x[8 * k + 7]) * mul));
-          }
+          for (int k = 0; k < 4; ++k)
+            reinterpret_cast<uint4*>(dst + q4 * 32)[k] = make_uint4(
+                pack_bf16x2(__uint_as_float(x[8 * k]) * mul, __uint_as_float(x[8 * k + 1]) * mul),
+                pack_bf16x2(__uint_as_float(x[8 * k + 2]) * mul, __uint_as_float(x[8 * k + 3]) * mul),
+                pack_bf16x2(__uint_as_float(x[8 * k + 4]) * mul, __uint_as_float(x[8 * k + 5]) * mul),
+                pack_bf16x2(__uint_as_float(x[8 * k + 6]) * mul, __uint_as_float(x[8 * k + 7]) * mul));
         }
       }
       tc_fence_before();
@@ -598,33 +455,303 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-// ------------------------------------------------------------------ dQ convert
-// dq = bf16(scale * sum_c acc[c]) with the chains summed in order c = 0, 1, ...;
-// chain c holds a contribution for query tile i only if the tile has more than c
-// contributors (i + 1 of them when causal, nt otherwise).
+// ================================================================== bwd_q
 template <int D>
-__global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* dq,
-                                                          long long BHq, int N, int nt, int causal, float scale) {
-  const long long npad = static_cast<long long>(nt) * 128;
-  const long long vecs = BHq * N * (D / 8);
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < vecs; x += stride) {
-    const long long row = x / (D / 8);
-    const int c8 = static_cast<int>(x - row * (D / 8)) * 8;
-    const long long bh = row / N;
-    const int n = static_cast<int>(row - bh * N);
-    const int contributors = causal ? (n / 128 + 1) : nt;
-    const int nch = contributors < kChains ? contributors : kChains;
-    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int c = 0; c < nch; ++c) {
-      const float4* src = reinterpret_cast<const float4*>(acc + ((c * BHq + bh) * npad + n) * D + c8);
-      const float4 a = src[0], b = src[1];
-      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+struct QCfg {
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kBox = 128 * 128;
+  static constexpr int kThreads = 320;
+  static constexpr int KVST = 2;                         // K/V ring stages
+  // TMEM columns: two S buffers (lane = query, column = key) with dS as bf16 over
+  // them (keys 0-63 in columns 0-31, keys 64-127 in columns 64-95 of the buffer),
+  // dP, and the dQ accumulator.
+  static constexpr int kS0 = 0, kS1 = 128, kDP = 256, kDQ = 384;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kOffQ = 0, kOffDO = kTile;
+  static constexpr int kOffK = 2 * kTile;                // KVST stages
+  static constexpr int kOffV = kOffK + KVST * kTile;     // KVST stages
+  static constexpr int kOffBar = kOffV + KVST * kTile;
+  static constexpr int kLayout = kOffBar + 256;
+  static constexpr int kSmem = kLayout + 1024;
+};
+
+struct QShared {
+  uint64_t qdo_full, qdo_empty;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2];           // S(j) in buffer j % 2
+  uint64_t dp_full;             // dP(j)
+  uint64_t dp_free;             // dP(j) read by both warpgroups
+  uint64_t ds_ready;            // dS(j) (bf16) written over S buffer j % 2
+  uint64_t q_done[2];           // dQ MMA of step j complete (S buffer j % 2 free)
+  uint64_t acc_free;            // dQ of the previous item read out
+  uint64_t drain;
+  uint32_t tmem_base;
+};
+
+// item t -> (bh_q, query tile i); causal: longest rows first
+__device__ __forceinline__ void q_item(const BwdParams& p, int t, int& bhq, int& i) {
+  const int BH = p.B * p.Hq;
+  const int r = t / BH;
+  bhq = t - r * BH;
+  i = p.causal ? (p.nt - 1 - r) : r;
+}
+__device__ __forceinline__ int q_n_kv(const BwdParams& p, int i) { return p.causal ? (i + 1) : p.nt; }
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
+                      const BwdParams p) {
+  using C = QCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  QShared& sh = *reinterpret_cast<QShared*>(smem + C::kOffBar);
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sDO = smem + C::kOffDO;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&sh.qdo_full, 1);
+    mbar_init(&sh.qdo_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.k_full[i], 1);
+      mbar_init(&sh.k_empty[i], 1);
+      mbar_init(&sh.v_full[i], 1);
+      mbar_init(&sh.v_empty[i], 1);
+      mbar_init(&sh.s_full[i], 1);
+      mbar_init(&sh.q_done[i], 1);
     }
-    *reinterpret_cast<uint4*>(dq + row * D + c8) =
-        make_uint4(pack_bf16x2(v[0] * scale, v[1] * scale), pack_bf16x2(v[2] * scale, v[3] * scale),
-                   pack_bf16x2(v[4] * scale, v[5] * scale), pack_bf16x2(v[6] * scale, v[7] * scale));
+    mbar_init(&sh.dp_full, 1);
+    mbar_init(&sh.dp_free, 8);
+    mbar_init(&sh.ds_ready, 8);
+    mbar_init(&sh.acc_free, 8);
+    mbar_init(&sh.drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) { tmem_alloc(&sh.tmem_base, C::kTmemCols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv); tma_prefetch_desc(&tmdo);
+      int gj = 0, it = 0, nk = 0, nv = 0, nqd = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
+        int bhq, i;
+        q_item(p, t, bhq, i);
+        const int bkv = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / p.G;
+        const int n_kv = q_n_kv(p, i);
+        if (it >= 1) ok = mbar_wait(&sh.qdo_empty, (it - 1) & 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&sh.qdo_full, 2 * C::kTile);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(sQ + c * C::kBox, &tmq, &sh.qdo_full, c * 64, i * 128, bhq);
+          tma_load_3d(sDO + c * C::kBox, &tmdo, &sh.qdo_full, c * 64, i * 128, bhq);
+        }
+        nqd = it + 1;
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const int g = gj + j, st = g % C::KVST;
+          if (g >= C::KVST) ok = mbar_wait(&sh.k_empty[st], ((g / C::KVST) - 1) & 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, j * 128, bkv);
+          nk = g + 1;
+          if (g >= C::KVST) ok = mbar_wait(&sh.v_empty[st], ((g / C::KVST) - 1) & 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sV + st * C::kTile + c * C::kBox, &tmv, &sh.v_full[st], c * 64, j * 128, bkv);
+          nv = g + 1;
+        }
+        gj += n_kv;
+      }
+      if (!ok) {
+        if (nqd >= 1) mbar_drain_wait(&sh.qdo_full, (nqd - 1) & 1);
+        for (int g = max(0, nk - C::KVST); g < nk; ++g) mbar_drain_wait(&sh.k_full[g % C::KVST], (g / C::KVST) & 1);
+        for (int g = max(0, nv - C::KVST); g < nv; ++g) mbar_drain_wait(&sh.v_full[g % C::KVST], (g / C::KVST) & 1);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    // Order per step j:  S(j+1)  [dS(j)] dQ(j)  dP(j+1).  The warpgroups' exps of step
+    // j+1 run under dQ(j) and dP(j+1); dS of step j needs dP(j).
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);   // S, dP
+      constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);      // dQ += dS K
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+      int gj = 0, it = 0;
+      bool ok = true;
+      auto issue_s = [&](int g) -> bool {     // S(g) = Q K(g)^T into buffer g % 2
+        const int st = g % C::KVST, sb = g & 1;
+        if (!mbar_wait(&sh.k_full[st], (g / C::KVST) & 1)) return false;
+        if (g >= 2 && !mbar_wait(&sh.q_done[sb], ((g >> 1) - 1) & 1)) return false;   // dS(g-2) consumed
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sK + st * C::kTile);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+          umma_ss(tmem + (sb ? C::kS1 : C::kS0), sdesc_sw128(q_addr + off, 16, 1024),
+                  sdesc_sw128(k_addr + off, 16, 1024), idS, k > 0);
+        }
+        umma_commit(&sh.s_full[sb]);
+        return true;
+      };
+      auto issue_dp = [&](int g) -> bool {    // dP(g) = dO V(g)^T
+        const int st = g % C::KVST;
+        if (!mbar_wait(&sh.v_full[st], (g / C::KVST) & 1)) return false;
+        if (g >= 1 && !mbar_wait(&sh.dp_free, (g - 1) & 1)) return false;       // dP(g-1) read
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sV + st * C::kTile);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+          umma_ss(tmem + C::kDP, sdesc_sw128(do_addr + off, 16, 1024), sdesc_sw128(v_addr + off, 16, 1024),
+                  idS, k > 0);
+        }
+        umma_commit(&sh.dp_full);
+        umma_commit(&sh.v_empty[st]);
+        return true;
+      };
+      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
+        int bhq, i;
+        q_item(p, t, bhq, i);
+        const int n_kv = q_n_kv(p, i);
+        ok = mbar_wait(&sh.qdo_full, it & 1);
+        if (!ok) break;
+        ok = issue_s(gj) && issue_dp(gj);
+        for (int u = 0; u < n_kv && ok; ++u) {
+          const int g = gj + u, st = g % C::KVST, sb = g & 1;
+          if (u + 1 < n_kv && !issue_s(g + 1)) { ok = false; break; }
+          // dQ += dS K  (A = dS in TMEM, M = queries, K = keys; B = K MN-major)
+          ok = mbar_wait(&sh.ds_ready, g & 1);
+          if (ok && u == 0 && it >= 1) ok = mbar_wait(&sh.acc_free, (it - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sK + st * C::kTile);
+          const uint32_t sbase = tmem + (sb ? C::kS1 : C::kS0);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_ts(tmem + C::kDQ, sbase + (k >> 2) * 64 + (k & 3) * 8, sdesc_sw128(k_addr + k * 2048, C::kBox, 1024),
+                    idQ, !(u == 0 && k == 0));
+          umma_commit(&sh.q_done[sb]);
+          umma_commit(&sh.k_empty[st]);
+          if (u + 1 < n_kv) {
+            if (!issue_dp(g + 1)) { ok = false; break; }
+          } else {
+            umma_commit(&sh.qdo_empty);     // the item's last reads of Q and dO are issued
+          }
+        }
+        if (!ok) break;
+        gj += n_kv;
+      }
+      umma_commit(&sh.drain);
+      mbar_wait(&sh.drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ dS warpgroups (rows = queries)
+    // warps 0-3: keys 0-63 of every step, warps 4-7: keys 64-127.  The row's LSE and D
+    // are this thread's own, held in registers for the whole item.
+    const int hb = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const float c = p.c;
+    int gj = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x) {
+      int bhq, i;
+      q_item(p, t, bhq, i);
+      const int n_kv = q_n_kv(p, i);
+      const int qrow = i * 128 + r;
+      const size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + qrow;
+      const float l2 = p.lse2[vrow], drow = p.dd[vrow];
+      float lv[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) lv[k] = l2;
+      for (int u = 0; u < n_kv && ok; ++u) {
+        const int g = gj + u, sb = g & 1;
+        const uint32_t sbase = lane_base + (sb ? C::kS1 : C::kS0) + 64 * hb;
+        // visible key columns (relative to this warpgroup's 64) for this query row
+        const int kbase = u * 128 + 64 * hb;
+        const int hi = min(p.N - 1, p.causal ? qrow : p.N - 1) - kbase;
+        const bool masked = !__all_sync(0xffffffffu, hi >= 63);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[sb], (g >> 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        // phase A: P = exp2(S c - lse2) for this warpgroup's 64 keys
+        float pf[64];
+#pragma unroll
+        for (int q16 = 0; q16 < 4; ++q16) {
+          uint32_t sr[16];
+          tmem_ld16(sbase + q16 * 16, sr);
+          tmem_wait_ld();
+          bwd_exp16(sr, lv, c, masked, q16 * 16, 0, hi, pf + q16 * 16);
+        }
+        // phase B: dS = P (dP - D) -> bf16 over the S buffer
+        ok = __all_sync(0xffffffffu, mbar_wait(&sh.dp_full, g & 1));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int q16 = 0; q16 < 4; ++q16) {
+          uint32_t dr[16];
+          tmem_ld16(lane_base + C::kDP + 64 * hb + q16 * 16, dr);
+          tmem_wait_ld();
+          uint32_t dk[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k] * (__uint_as_float(dr[2 * k]) - drow),
+                                pf[q16 * 16 + 2 * k + 1] * (__uint_as_float(dr[2 * k + 1]) - drow));
+          tmem_st8(sbase + q16 * 8, dk);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.dp_free);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.ds_ready);
+      }
+      if (!ok) break;
+      // epilogue: dQ (TMEM lane = query row), scaled, bf16; the two warpgroups split the columns
+      const int glast = gj + n_kv - 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sh.q_done[glast & 1], (glast >> 1) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      const bool live = qrow < p.N;
+      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bhq) * p.N + qrow) * D;
+#pragma unroll 1
+      for (int q4 = hb; q4 < D / 32; q4 += 2) {
+        uint32_t x[32];
+        tmem_ld32(lane_base + C::kDQ + q4 * 32, x);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            reinterpret_cast<uint4*>(dst + q4 * 32)[k] = make_uint4(
+                pack_bf16x2(__uint_as_float(x[8 * k]) * p.scale, __uint_as_float(x[8 * k + 1]) * p.scale),
+                pack_bf16x2(__uint_as_float(x[8 * k + 2]) * p.scale, __uint_as_float(x[8 * k + 3]) * p.scale),
+                pack_bf16x2(__uint_as_float(x[8 * k + 4]) * p.scale, __uint_as_float(x[8 * k + 5]) * p.scale),
+                pack_bf16x2(__uint_as_float(x[8 * k + 6]) * p.scale, __uint_as_float(x[8 * k + 7]) * p.scale));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.acc_free);
+      gj += n_kv;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
