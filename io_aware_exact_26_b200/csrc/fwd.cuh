@@ -7,15 +7,20 @@
 // output is rescaled by exp(m_old - m_new) when the max grows, and only O and the
 // log-sum-exp leave the chip.  S and P never reach HBM.
 //
-// B200 mapping (one persistent CTA per SM, 192 threads):
-//   warps 0-3  softmax warpgroup: thread = one query row = one TMEM lane.
-//              tcgen05.ld the S row, row max / exp2 / row sum in registers,
-//              P written back to TMEM as bf16 (aliasing S), O rescale, epilogue.
-//   warp 4     TMA producer: Q tile (double buffered), K ring, V ring.
-//   warp 5     MMA issuer (one thread): S = Q K^T (SS, both K-major) and
+// B200 mapping (one persistent CTA per SM, 320 threads):
+//   warps 0-3  softmax warpgroup A: keys 0-63 of every S tile, O columns [0, D/2)
+//   warps 4-7  softmax warpgroup B: keys 64-127, O columns [D/2, D)
+//              thread = one query row = one TMEM lane.  The two groups exchange
+//              their partial row maxima through shared memory once per tile, so
+//              both take the same rescale decisions; each keeps its own partial
+//              row sum, combined in the epilogue.
+//   warp 8     TMA producer: Q tile (double buffered), K ring, V ring.
+//   warp 9     MMA issuer (one thread): S = Q K^T (SS, both K-major) and
 //              O += P V (A = P from TMEM, B = V MN-major), accumulating in TMEM.
 // TMEM (512 columns): three 128-column S/P buffers, then O (D columns).  Three
 // S buffers let S(j+1) be issued while P(j-1) may still be read by its PV MMA.
+// P(j) (bf16) is written over the S buffer: keys 0-63 in columns 0-31, keys
+// 64-127 in columns 64-95, so neither group overwrites columns the other reads.
 //
 // exp2 with a folded scale: c = scale * log2(e), p = exp2(s*c - m) where m is
 // kept in log2 units; LSE = ln(2) * (m + log2 l).  The max used for the
@@ -23,9 +28,7 @@
 // invariance of softmax (page "attn-efficient": subtracting the same number from
 // a whole score row leaves the result unchanged) any reference value works as
 // long as O and l use the same one; this keeps p <= 2^tau and skips most O
-// rescales.  Two row sums are kept: l of the bf16-rounded p that the PV MMA
-// consumes (O is normalised by it, so a constant V comes out exactly), and the
-// fp32 sum of the unrounded p, from which the LSE is formed.
+// rescales.  l is the fp32 sum of the p that are rounded to bf16 for the PV MMA.
 #pragma once
 #include "sm100.cuh"
 
@@ -35,15 +38,21 @@ constexpr float kRescaleTau = 8.0f;
 
 template <int D>
 struct FwdCfg {
-  static constexpr int BM = 128, BN = 128;
   static constexpr int kTile = 128 * D * 2;          // bytes of one 128 x D bf16 tile
   static constexpr int kBox = 128 * 128;             // bytes of one 128 x 64 swizzled box
   static constexpr int KST = (D == 128) ? 3 : 4;     // K ring stages
   static constexpr int VST = (D == 128) ? 2 : 4;     // V ring stages
-  static constexpr int kSmem = (2 + KST + VST) * kTile + 1024;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = 384;                  // O accumulator column
+  static constexpr int kOffQ = 0;                    // 2 tiles
+  static constexpr int kOffK = 2 * kTile;
+  static constexpr int kOffV = kOffK + KST * kTile;
+  static constexpr int kOffSh = kOffV + VST * kTile; // FwdShared
+  static constexpr int kLayout = kOffSh + 2560;
+  // the d = 128 layout leaves no room for alignment slack under the 227 KB limit;
+  // the kernel checks the base alignment at run time
+  static constexpr int kSmem = (kLayout + 1024 <= 232448) ? kLayout + 1024 : kLayout;
 };
 
 struct FwdParams {
@@ -56,14 +65,22 @@ struct FwdParams {
 };
 
 struct FwdShared {
+  // [parity][group][row]: partial row maxima of tile g live in xch[g & 1]; the
+  // epilogue's partial row sums go to the half the last tile did not use
+  float xch[2][2][128];
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
   uint64_t s_full[3], p_ready[3], pv_done[3];
+  uint64_t xbar[2];          // both groups posted their maxima for a tile
+  uint64_t sbar;             // both groups posted their sums for a query tile
+  uint64_t sread;            // both groups read the sums (the half may be reused)
   uint64_t o_free;
   uint64_t drain;
+  uint64_t teardown;         // every warp is done with TMEM
   uint32_t tmem_base;
 };
+static_assert(sizeof(FwdShared) <= 2560, "FwdShared does not fit its slot");
 
 // Work tile t -> (query tile, batch*head).  Causal: longest rows first.
 __device__ __forceinline__ void fwd_tile_coords(const FwdParams& p, int t, int& qt, int& bh) {
@@ -79,16 +96,21 @@ __device__ __forceinline__ int fwd_n_kv(const FwdParams& p, int qt) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
   using C = FwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ FwdShared sh;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                              // 2 tiles
-  uint8_t* sK = smem + 2 * C::kTile;               // KST tiles
-  uint8_t* sV = sK + C::KST * C::kTile;            // VST tiles
+  if (static_cast<int>(smem - smem_raw) + C::kLayout > C::kSmem) {
+    // the 128B-swizzled tiles need a 1024-byte aligned base that this launch cannot give
+    if (threadIdx.x == 0) record_error(&g_attn_status, 3);
+    return;
+  }
+  FwdShared& sh = *reinterpret_cast<FwdShared*>(smem + C::kOffSh);
+  uint8_t* sQ = smem + C::kOffQ;                   // 2 tiles
+  uint8_t* sK = smem + C::kOffK;                   // KST tiles
+  uint8_t* sV = smem + C::kOffV;                   // VST tiles
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -98,11 +120,16 @@ __global__ void __launch_bounds__(192, 1)
     for (int i = 0; i < C::VST; ++i) { mbar_init(&sh.v_full[i], 1); mbar_init(&sh.v_empty[i], 1); }
     for (int i = 0; i < 3; ++i) {
       mbar_init(&sh.s_full[i], 1);
-      mbar_init(&sh.p_ready[i], 4);
+      mbar_init(&sh.p_ready[i], 8);
       mbar_init(&sh.pv_done[i], 1);
     }
-    mbar_init(&sh.o_free, 4);
+    mbar_init(&sh.xbar[0], 8);
+    mbar_init(&sh.xbar[1], 8);
+    mbar_init(&sh.sbar, 8);
+    mbar_init(&sh.sread, 8);
+    mbar_init(&sh.o_free, 8);
     mbar_init(&sh.drain, 1);
+    mbar_init(&sh.teardown, 10);
     fence_barrier_init();
   }
   if (warp == 0) { tmem_alloc(&sh.tmem_base, C::kTmemCols); tmem_relinquish(); }
@@ -111,7 +138,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv);
@@ -159,7 +186,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int g = max(0, nq - 2); g < nq; ++g) mbar_drain_wait(&sh.q_full[g & 1], (g >> 1) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
@@ -175,41 +202,43 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sQ + qb * C::kTile);
-        for (int s = 0; s <= n_kv && ok; ++s) {
-          if (s < n_kv) {
-            // S(g) = Q K(g)^T into S buffer g % 3
-            const int g = it + s, kst = g % C::KST, sb = g % 3;
-            ok = mbar_wait(&sh.k_full[kst], (g / C::KST) & 1);
-            if (ok && g >= 3) ok = mbar_wait(&sh.pv_done[sb], ((g / 3) - 1) & 1);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t k_addr = smem_u32(sK + kst * C::kTile);
+        // S(g) = Q K(g)^T into S buffer g % 3 (the buffer last held P(g - 3))
+        auto issue_s = [&](int j) -> bool {
+          const int g = it + j, kst = g % C::KST, sb = g % 3;
+          if (!mbar_wait(&sh.k_full[kst], (g / C::KST) & 1)) return false;
+          if (g >= 3 && !mbar_wait(&sh.pv_done[sb], ((g / 3) - 1) & 1)) return false;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sK + kst * C::kTile);
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-              umma_ss(tmem + sb * 128, sdesc_sw128(q_addr + off, 16, 1024),
-                      sdesc_sw128(k_addr + off, 16, 1024), idS, k > 0);
-            }
-            umma_commit(&sh.s_full[sb]);
-            umma_commit(&sh.k_empty[kst]);
-            if (s == n_kv - 1) umma_commit(&sh.q_empty[qb]);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+            umma_ss(tmem + sb * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
+                    idS, k > 0);
           }
-          if (s >= 1) {
-            // O (+)= P(g) V(g)
-            const int g = it + s - 1, vst = g % C::VST, sb = g % 3;
-            ok = mbar_wait(&sh.v_full[vst], (g / C::VST) & 1);
-            if (ok) ok = mbar_wait(&sh.p_ready[sb], (g / 3) & 1);
-            if (ok && s == 1 && tl >= 1) ok = mbar_wait(&sh.o_free, (tl - 1) & 1);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t v_addr = smem_u32(sV + vst * C::kTile);
+          umma_commit(&sh.s_full[sb]);
+          umma_commit(&sh.k_empty[kst]);
+          if (j == n_kv - 1) umma_commit(&sh.q_empty[qb]);
+          return true;
+        };
+        // S runs two tiles ahead of PV, so the softmax groups can load S(j+1) while
+        // they exponentiate tile j.
+        ok = issue_s(0) && (n_kv < 2 || issue_s(1));
+        for (int j = 0; j < n_kv && ok; ++j) {
+          if (j + 2 < n_kv && !issue_s(j + 2)) { ok = false; break; }
+          // O (+)= P(g) V(g); P keys 0-63 in columns 0-31, keys 64-127 in 64-95
+          const int g = it + j, vst = g % C::VST, sb = g % 3;
+          ok = mbar_wait(&sh.v_full[vst], (g / C::VST) & 1);
+          if (ok) ok = mbar_wait(&sh.p_ready[sb], (g / 3) & 1);
+          if (ok && j == 0 && tl >= 1) ok = mbar_wait(&sh.o_free, (tl - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(sV + vst * C::kTile);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              umma_ts(tmem + C::kOCol, tmem + sb * 128 + k * 8,
-                      sdesc_sw128(v_addr + k * 2048, C::kBox, 1024), idO, (s > 1 || k > 0));
-            umma_commit(&sh.pv_done[sb]);
-            umma_commit(&sh.v_empty[vst]);
-          }
+          for (int k = 0; k < 8; ++k)
+            umma_ts(tmem + C::kOCol, tmem + sb * 128 + (k >> 2) * 64 + (k & 3) * 8,
+                    sdesc_sw128(v_addr + k * 2048, C::kBox, 1024), idO, (j > 0 || k > 0));
+          umma_commit(&sh.pv_done[sb]);
+          umma_commit(&sh.v_empty[vst]);
         }
         it += n_kv;
       }
@@ -217,11 +246,15 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(&sh.drain);
       mbar_wait(&sh.drain, 0);
     }
-  } else {
-    // ------------------------------------------------------------ softmax warpgroup
-    const int row = warp * 32 + lane;                       // TMEM lane == tile row
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int hb = warp >> 2;                                   // 0: keys 0-63, 1: keys 64-127
+    const int row = (warp & 3) * 32 + lane;                     // TMEM lane == tile row
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    constexpr int OH = D / 2;                                   // O columns per group
+    const uint32_t o_base = lane_base + C::kOCol + hb * OH;
     const float c = p.c;
+    const uint64_t c2 = f2pack(c, c);
     int it = 0, tl = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x, ++tl) {
@@ -229,77 +262,130 @@ __global__ void __launch_bounds__(192, 1)
       fwd_tile_coords(p, t, qt, bh);
       const int n_kv = fwd_n_kv(p, qt);
       const int qrow = qt * 128 + row;
-      float m_used = -INFINITY, l = 0.f, l_exact = 0.f;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int g = it + j, sb = g % 3;
+      float m_used = -INFINITY;
+      uint64_t lsum = f2pack(0.f, 0.f);                         // two partial sums
+      // last visible key of this row within this group's 64 columns of tile j
+      auto last_col = [&](int j) -> int {
+        const int kbase = j * 128 + hb * 64;
+        const int lim = p.N - 1 - kbase;
+        return p.causal ? min(lim, qrow - kbase) : lim;
+      };
+      auto mask32 = [&](uint32_t (&r)[32], int col0, int lim) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (col0 + k > lim) r[k] = 0xff800000u;
+      };
+      auto max32 = [&](float (&mx4)[4], const uint32_t (&r)[32]) {
+#pragma unroll
+        for (int k = 0; k < 32; k += 8) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            mx4[e] = max3f(mx4[e], __uint_as_float(r[k + e]), __uint_as_float(r[k + e + 4]));
+        }
+      };
+      // post this group's partial max of tile j for the other group
+      auto post = [&](int j, const float (&mx4)[4]) -> bool {
+        const int g = it + j, xp = g & 1;
+        const float pm = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        if (j == 0 && tl >= 1) {       // the previous epilogue's sums used this half
+          if (!__all_sync(0xffffffffu, mbar_wait(&sh.sread, (tl - 1) & 1))) return false;
+        }
+        sh.xch[xp][hb][row] = pm;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.xbar[xp]);
+        return true;
+      };
+      // tile 0's maximum, before the pipelined loop
+      {
+        const int g = it, sb = g % 3;
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[sb], (g / 3) & 1));
         if (!ok) break;
         tc_fence_after();
-        uint32_t r[128];
+        const int lim = last_col(0);
+        const bool msk = __any_sync(0xffffffffu, lim < 63);
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          tmem_ld32(lane_base + sb * 128 + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
-        tmem_wait_ld();
-        // masking: causal diagonal tile and the ragged key tail
-        const int kbase = j * 128;
-        int lim = p.N - 1 - kbase;
-        if (p.causal) lim = min(lim, qrow - kbase);
-        if (lim < 127) {
-#pragma unroll
-          for (int k = 0; k < 128; ++k)
-            if (k > lim) r[k] = __float_as_uint(-INFINITY);
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + sb * 128 + hb * 64 + cc * 32, r);
+          tmem_wait_ld();
+          if (msk) mask32(r, cc * 32, lim);
+          max32(mx4, r);
         }
-        // row max with 8 independent chains (one warp per SMSP: no other warp hides latency)
-        float mx8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(r[k]);
-#pragma unroll
-        for (int k = 8; k < 128; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(r[k]));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
-        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
-        const float m_tile = mx * c;
+        ok = post(0, mx4);
+        if (!ok) break;
+      }
+      // Tile j: take the common max, exponentiate its scores chunk by chunk while the
+      // same chunk of tile j+1 is read for that tile's max, write P, rescale O if the
+      // max moved, hand P to the MMA warp.
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int g = it + j, sb = g % 3, xp = g & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sh.xbar[xp], (g >> 1) & 1));
+        if (!ok) break;
+        const float m_tile = fmaxf(sh.xch[xp][0][row], sh.xch[xp][1][row]) * c;
         float alpha = 1.f;
         const bool need = (m_used == -INFINITY) || (m_tile > m_used + kRescaleTau);
         if (need) {
           const float m_new = fmaxf(m_used, m_tile);
           alpha = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
-          l *= alpha;
-          l_exact *= alpha;
+          float l0, l1;
+          f2unpack(lsum, l0, l1);
+          lsum = f2pack(l0 * alpha, l1 * alpha);
           m_used = m_new;
         }
-        const float neg_m = -m_used;
-        float lr[4] = {0.f, 0.f, 0.f, 0.f}, le[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+        const bool has_next = j + 1 < n_kv;
+        const int sbn = (g + 1) % 3;
+        if (has_next) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[sbn], ((g + 1) / 3) & 1));
+          if (!ok) break;
+        }
+        tc_fence_after();
+        const int lim = last_col(j), limn = last_col(j + 1);
+        const bool msk = __any_sync(0xffffffffu, lim < 63);
+        const bool mskn = __any_sync(0xffffffffu, limn < 63);
+        const uint64_t nm2 = f2pack(-m_used, -m_used);
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t r[32], rn[32];
+          tmem_ld32(lane_base + sb * 128 + hb * 64 + cc * 32, r);
+          if (has_next) tmem_ld32(lane_base + sbn * 128 + hb * 64 + cc * 32, rn);
+          tmem_wait_ld();
+          if (msk) mask32(r, cc * 32, lim);
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const float a = ex2_approx(fmaf(__uint_as_float(r[q4 * 32 + 2 * k]), c, neg_m));
-            const float b = ex2_approx(fmaf(__uint_as_float(r[q4 * 32 + 2 * k + 1]), c, neg_m));
-            __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-            lr[k & 3] += __low2float(h) + __high2float(h);
-            le[k & 3] += a + b;
-            pk[k] = *reinterpret_cast<uint32_t*>(&h);
+            const uint64_t x = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
+            float x0, x1;
+            f2unpack(x, x0, x1);
+            const float a = ex2_approx(x0), b = ex2_approx(x1);
+            lsum = fadd2(lsum, f2pack(a, b));
+            pk[k] = pack_bf16x2(a, b);
           }
-          tmem_st16(lane_base + sb * 128 + q4 * 16, pk);
+          tmem_st16(lane_base + sb * 128 + hb * 64 + cc * 16, pk);
+          if (has_next) {
+            if (mskn) mask32(rn, cc * 32, limn);
+            max32(mx4, rn);
+          }
         }
-        l += (lr[0] + lr[1]) + (lr[2] + lr[3]);
-        l_exact += (le[0] + le[1]) + (le[2] + le[3]);
-        // Rescale the running output when this warp's max moved (rare after the first tiles).
+        if (has_next) {
+          ok = post(j + 1, mx4);
+          if (!ok) break;
+        }
+        // Rescale this group's half of the running output when its max moved.
         if (__any_sync(0xffffffffu, need && j > 0)) {
           const int gp = g - 1;
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[gp % 3], (gp / 3) & 1));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int q4 = 0; q4 < D / 32; ++q4) {
+          for (int q4 = 0; q4 < OH / 32; ++q4) {
             uint32_t o[32];
-            tmem_ld32(lane_base + C::kOCol + q4 * 32, o);
+            tmem_ld32(o_base + q4 * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(lane_base + C::kOCol + q4 * 32, o);
+            tmem_st32(o_base + q4 * 32, o);
           }
         }
         tmem_wait_st();
@@ -308,18 +394,29 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) mbar_arrive(&sh.p_ready[sb]);
       }
       if (!ok) break;
-      // epilogue: wait for the last PV, O / l -> bf16, LSE
+      // epilogue: combine the two partial sums, wait for the last PV, O / l -> bf16, LSE
       const int glast = it + n_kv - 1;
+      const int xs = (glast + 1) & 1;
+      float l0, l1;
+      f2unpack(lsum, l0, l1);
+      sh.xch[xs][hb][row] = l0 + l1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.sbar);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sh.sbar, tl & 1));
+      if (!ok) break;
+      const float l = sh.xch[xs][0][row] + sh.xch[xs][1][row];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.sread);
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[glast % 3], (glast / 3) & 1));
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool live = qrow < p.N;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D + hb * OH;
 #pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) {
+      for (int q4 = 0; q4 < OH / 32; ++q4) {
         uint32_t o[32];
-        tmem_ld32(lane_base + C::kOCol + q4 * 32, o);
+        tmem_ld32(o_base + q4 * 32, o);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
@@ -331,7 +428,7 @@ __global__ void __launch_bounds__(192, 1)
           for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      if (live) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + __log2f(l_exact)) * 0.69314718055994531f;
+      if (live && hb == 0) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + __log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.o_free);
@@ -339,9 +436,13 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
 
+  // Teardown without a shared code path (the warpgroups run under different
+  // register budgets): every warp posts, warp 0 releases TMEM once all have.
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sh.teardown);
   if (warp == 0) {
+    mbar_wait(&sh.teardown, 0);
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
