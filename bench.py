@@ -329,7 +329,7 @@ def main():
     peaks, peaks_kind = load_peaks()
     peak = float(peaks["bf16_tflops"])
     if has_bwd and bwd_avg >= fwd_avg:
-        kname, kflops, kms = "attn_bwd (prep + main)", f_bwd, bwd_avg
+        kname, kflops, kms = "attn_bwd (prep + dK/dV + dQ kernels)", f_bwd, bwd_avg
         traffic = measured_traffic(w.name, "bwd")
     else:
         kname, kflops, kms = "attn_fwd_kernel", f_fwd, fwd_avg
@@ -350,7 +350,7 @@ def main():
             "roofline": roofline,
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
-            "gpu_launches": args.steps * (3 if has_bwd else 1),
+            "gpu_launches": args.steps * (4 if has_bwd else 1),   # fwd; bwd = prep + dK/dV + dQ
             "clocks": clocks}
     if has_bwd:
         line["bwd"] = {"ms": round(bwd_avg, 4), "tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 1),

@@ -124,7 +124,7 @@ struct BwdParams {
 
 // Exps of one 16-column slice of a score tile held by this thread: p = 2^(s c - l).
 // Masked columns (only on diagonal / ragged tiles) get s = -inf first, so p = 0
-// exactly; the exp loop itself has no branch.
+// (or 2^-126.5 on the FMA-pipe path); the exp loop itself has no branch.
 __device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const float (&lv)[16], float c, bool masked,
                                           int col0, int lo, int hi, float* pf) {
   if (masked) {
@@ -133,7 +133,16 @@ __device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const float (&lv)[
       if (col0 + k < lo || col0 + k > hi) sr[k] = 0xff800000u;
   }
 #pragma unroll
-  for (int k = 0; k < 16; ++k) pf[k] = ex2_approx(fmaf(__uint_as_float(sr[k]), c, -lv[k]));
+  for (int k = 0; k < 16; k += 2) {
+    const float x0 = fmaf(__uint_as_float(sr[k]), c, -lv[k]);
+    const float x1 = fmaf(__uint_as_float(sr[k + 1]), c, -lv[k + 1]);
+    if ((k & 6) == 6) {
+      exp2_fma_pair(x0, x1, pf[k], pf[k + 1]);   // one pair in four on the FMA pipe
+    } else {
+      pf[k] = ex2_approx(x0);
+      pf[k + 1] = ex2_approx(x1);
+    }
+  }
 }
 
 // ================================================================== bwd_kv
@@ -460,7 +469,7 @@ template <int D>
 struct QCfg {
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kBox = 128 * 128;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 352;                   // 8 dS warps, K/Q/dO TMA, MMA, V TMA
   static constexpr int KVST = 2;                         // K/V ring stages
   // TMEM columns: two S buffers (lane = query, column = key) with dS as bf16 over
   // them (keys 0-63 in columns 0-31, keys 64-127 in columns 64-95 of the buffer),
@@ -498,7 +507,7 @@ __device__ __forceinline__ void q_item(const BwdParams& p, int t, int& bhq, int&
 __device__ __forceinline__ int q_n_kv(const BwdParams& p, int i) { return p.causal ? (i + 1) : p.nt; }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
                       const BwdParams p) {
@@ -537,10 +546,10 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = sh.tmem_base;
 
   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer: Q, dO and K
     if (lane == 0) {
-      tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv); tma_prefetch_desc(&tmdo);
-      int gj = 0, it = 0, nk = 0, nv = 0, nqd = 0;
+      tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmdo);
+      int gj = 0, it = 0, nk = 0, nqd = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
         int bhq, i;
@@ -563,6 +572,27 @@ __global__ void __launch_bounds__(320, 1)
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, j * 128, bkv);
           nk = g + 1;
+        }
+        gj += n_kv;
+      }
+      if (!ok) {
+        if (nqd >= 1) mbar_drain_wait(&sh.qdo_full, (nqd - 1) & 1);
+        for (int g = max(0, nk - C::KVST); g < nk; ++g) mbar_drain_wait(&sh.k_full[g % C::KVST], (g / C::KVST) & 1);
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ TMA producer: V
+    if (lane == 0) {
+      tma_prefetch_desc(&tmv);
+      int gj = 0, nv = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x) {
+        int bhq, i;
+        q_item(p, t, bhq, i);
+        const int bkv = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / p.G;
+        const int n_kv = q_n_kv(p, i);
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const int g = gj + j, st = g % C::KVST;
           if (g >= C::KVST) ok = mbar_wait(&sh.v_empty[st], ((g / C::KVST) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
@@ -572,11 +602,8 @@ __global__ void __launch_bounds__(320, 1)
         }
         gj += n_kv;
       }
-      if (!ok) {
-        if (nqd >= 1) mbar_drain_wait(&sh.qdo_full, (nqd - 1) & 1);
-        for (int g = max(0, nk - C::KVST); g < nk; ++g) mbar_drain_wait(&sh.k_full[g % C::KVST], (g / C::KVST) & 1);
+      if (!ok)
         for (int g = max(0, nv - C::KVST); g < nv; ++g) mbar_drain_wait(&sh.v_full[g % C::KVST], (g / C::KVST) & 1);
-      }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer

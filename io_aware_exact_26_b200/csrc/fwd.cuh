@@ -7,14 +7,16 @@
 // output is rescaled by exp(m_old - m_new) when the max grows, and only O and the
 // log-sum-exp leave the chip.  S and P never reach HBM.
 //
-// B200 mapping (one persistent CTA per SM, 320 threads):
+// B200 mapping (one persistent CTA per SM, 352 threads):
 //   warps 0-3  softmax warpgroup A: keys 0-63 of every S tile, O columns [0, D/2)
 //   warps 4-7  softmax warpgroup B: keys 64-127, O columns [D/2, D)
 //              thread = one query row = one TMEM lane.  The two groups exchange
 //              their partial row maxima through shared memory once per tile, so
 //              both take the same rescale decisions; each keeps its own partial
 //              row sum, combined in the epilogue.
-//   warp 8     TMA producer: Q tile (double buffered), K ring, V ring.
+//   warp 8     TMA producer for Q (double buffered) and the K ring
+//   warp 10    TMA producer for the V ring (its own stream, so a K load never
+//              queues behind a V load that waits for a free stage)
 //   warp 9     MMA issuer (one thread): S = Q K^T (SS, both K-major) and
 //              O += P V (A = P from TMEM, B = V MN-major), accumulating in TMEM.
 // TMEM (512 columns): three 128-column S/P buffers, then O (D columns).  Three
@@ -42,7 +44,7 @@ struct FwdCfg {
   static constexpr int kBox = 128 * 128;             // bytes of one 128 x 64 swizzled box
   static constexpr int KST = (D == 128) ? 3 : 4;     // K ring stages
   static constexpr int VST = (D == 128) ? 2 : 4;     // V ring stages
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 352;
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = 384;                  // O accumulator column
   static constexpr int kOffQ = 0;                    // 2 tiles
@@ -96,7 +98,7 @@ __device__ __forceinline__ int fwd_n_kv(const FwdParams& p, int qt) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
   using C = FwdCfg<D>;
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(&sh.sread, 8);
     mbar_init(&sh.o_free, 8);
     mbar_init(&sh.drain, 1);
-    mbar_init(&sh.teardown, 10);
+    mbar_init(&sh.teardown, 11);
     fence_barrier_init();
   }
   if (warp == 0) { tmem_alloc(&sh.tmem_base, C::kTmemCols); tmem_relinquish(); }
@@ -139,10 +141,10 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = sh.tmem_base;
 
   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer: Q and K
     if (lane == 0) {
-      tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv);
-      int it = 0, tl = 0, nk = 0, nv = 0, nq = 0;
+      tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk);
+      int it = 0, tl = 0, nk = 0, nq = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x, ++tl) {
         int qt, bh;
@@ -156,35 +158,47 @@ __global__ void __launch_bounds__(320, 1)
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(sQ + qb * C::kTile + c * C::kBox, &tmq, &sh.q_full[qb], c * 64, qt * 128, bh);
         nq = tl + 1;
-        // loads in the order the MMA warp consumes them: K0, K1, V0, K2, V1, ...
-        for (int s = 0; s <= n_kv && ok; ++s) {
-          if (s < n_kv) {
-            const int g = it + s, st = g % C::KST;
-            if (g >= C::KST) ok = mbar_wait(&sh.k_empty[st], ((g / C::KST) - 1) & 1);
-            if (!ok) break;
-            mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, s * 128, bkv);
-            nk = g + 1;
-          }
-          if (s >= 1) {
-            const int g = it + s - 1, st = g % C::VST;
-            if (g >= C::VST) ok = mbar_wait(&sh.v_empty[st], ((g / C::VST) - 1) & 1);
-            if (!ok) break;
-            mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sV + st * C::kTile + c * C::kBox, &tmv, &sh.v_full[st], c * 64, (s - 1) * 128, bkv);
-            nv = g + 1;
-          }
+        for (int s = 0; s < n_kv && ok; ++s) {
+          const int g = it + s, st = g % C::KST;
+          if (g >= C::KST) ok = mbar_wait(&sh.k_empty[st], ((g / C::KST) - 1) & 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, s * 128, bkv);
+          nk = g + 1;
         }
         it += n_kv;
       }
       if (!ok) {
         // Let the copies already in flight land before the CTA exits (bounded).
         for (int g = max(0, nk - C::KST); g < nk; ++g) mbar_drain_wait(&sh.k_full[g % C::KST], (g / C::KST) & 1);
-        for (int g = max(0, nv - C::VST); g < nv; ++g) mbar_drain_wait(&sh.v_full[g % C::VST], (g / C::VST) & 1);
         for (int g = max(0, nq - 2); g < nq; ++g) mbar_drain_wait(&sh.q_full[g & 1], (g >> 1) & 1);
       }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ TMA producer: V
+    if (lane == 0) {
+      tma_prefetch_desc(&tmv);
+      int it = 0, nv = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+        int qt, bh;
+        fwd_tile_coords(p, t, qt, bh);
+        const int n_kv = fwd_n_kv(p, qt);
+        const int bkv = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.G;
+        for (int s = 0; s < n_kv && ok; ++s) {
+          const int g = it + s, st = g % C::VST;
+          if (g >= C::VST) ok = mbar_wait(&sh.v_empty[st], ((g / C::VST) - 1) & 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sV + st * C::kTile + c * C::kBox, &tmv, &sh.v_full[st], c * 64, s * 128, bkv);
+          nv = g + 1;
+        }
+        it += n_kv;
+      }
+      if (!ok)
+        for (int g = max(0, nv - C::VST); g < nv; ++g) mbar_drain_wait(&sh.v_full[g % C::VST], (g / C::VST) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
@@ -356,9 +370,14 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const uint64_t x = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
-            float x0, x1;
+            float x0, x1, a, b;
             f2unpack(x, x0, x1);
-            const float a = ex2_approx(x0), b = ex2_approx(x1);
+            if ((k & 3) == 3) {
+              exp2_fma_pair(x0, x1, a, b);          // one pair in four on the FMA pipe
+            } else {
+              a = ex2_approx(x0);
+              b = ex2_approx(x1);
+            }
             lsum = fadd2(lsum, f2pack(a, b));
             pk[k] = pack_bf16x2(a, b);
           }

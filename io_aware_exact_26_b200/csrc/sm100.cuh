@@ -308,6 +308,34 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return r;
 }
 
+// exp2 of a pair on the FMA pipe, to take load off the MUFU pipe (16 ex2 per SM
+// per clock).  Range reduction x = n + f with n = round(x), |f| <= 1/2, via the
+// 1.5 * 2^23 rounding constant; 2^f from a cubic fitted for minimum relative error
+// on [-1/2, 1/2] (gen_exp2_poly.py: bound 7.5e-5, far below bf16 rounding); 2^n
+// added to the exponent field as an integer.  Inputs below -126 are clamped, so
+// the result is at least 2^-126.5 instead of underflowing (vanishing next to the
+// row's other terms, which include 2^0 or more).
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716648042202f;
+
+__device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = fadd2(x, f2pack(12582912.f, 12582912.f));            // 1.5 * 2^23 + n
+  const uint64_t r = fadd2(t, f2pack(-12582912.f, -12582912.f));          // n as a float
+  const uint64_t f = ffma2(r, f2pack(-1.f, -1.f), x);                     // x - n
+  uint64_t q = ffma2(f, f2pack(kExp2C3, kExp2C3), f2pack(kExp2C2, kExp2C2));
+  q = ffma2(q, f, f2pack(kExp2C1, kExp2C1));
+  q = ffma2(q, f, f2pack(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  // the low bits of t's pattern hold n; shifted by 23 only n's bits survive
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
