@@ -179,11 +179,12 @@ struct KvShared {
 
 // item t -> (bh_kv, key tile j); key tile outermost, so the key tiles with the most
 // query tiles (causal) come first
+// Items are numbered KV head by KV head, so the CTAs running at the same time
+// stream the Q/dO of the same few head groups (L2 hits); within a head, key tile
+// j ascending (causal: the item of key tile j sees nt - j query tiles, longest first).
 __device__ __forceinline__ void kv_item(const BwdParams& p, int t, int& bhkv, int& j) {
-  const int BHkv = p.B * p.Hkv;
-  const int r = t / BHkv;
-  bhkv = t - r * BHkv;
-  j = r;
+  bhkv = t / p.nt;
+  j = t - bhkv * p.nt;
 }
 __device__ __forceinline__ int kv_first_q(const BwdParams& p, int j) { return p.causal ? j : 0; }
 
@@ -388,6 +389,7 @@ __global__ void __launch_bounds__(320, 1)
               lv[4 * k] = a.x; lv[4 * k + 1] = a.y; lv[4 * k + 2] = a.z; lv[4 * k + 3] = a.w;
             }
             tmem_wait_ld();
+            reg_fence(sr);
             bwd_exp16(sr, lv, c, masked, q16 * 16, lo, hi, pf + q16 * 16);
             uint32_t pk[8];
 #pragma unroll
@@ -413,6 +415,7 @@ __global__ void __launch_bounds__(320, 1)
               dv[4 * k] = b.x; dv[4 * k + 1] = b.y; dv[4 * k + 2] = b.z; dv[4 * k + 3] = b.w;
             }
             tmem_wait_ld();
+            reg_fence(dr);
             uint32_t dk[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
@@ -440,6 +443,7 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t x[32];
         tmem_ld32(lane_base + col + q4 * 32, x);
         tmem_wait_ld();
+        reg_fence(x);
         if (live) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
@@ -497,12 +501,17 @@ struct QShared {
   uint32_t tmem_base;
 };
 
-// item t -> (bh_q, query tile i); causal: longest rows first
+// item t -> (bh_q, query tile i).  Numbered KV head by KV head (the G query heads
+// of a group interleaved), so CTAs running at the same time share K/V in L2;
+// causal: longest rows first within a group.
 __device__ __forceinline__ void q_item(const BwdParams& p, int t, int& bhq, int& i) {
-  const int BH = p.B * p.Hq;
-  const int r = t / BH;
-  bhq = t - r * BH;
-  i = p.causal ? (p.nt - 1 - r) : r;
+  const int per_group = p.G * p.nt;
+  const int gk = t / per_group;                  // b * Hkv + kv-head
+  const int r = t - gk * per_group;
+  const int rq = r / p.G;
+  const int hin = r - rq * p.G;
+  i = p.causal ? (p.nt - 1 - rq) : rq;
+  bhq = (gk / p.Hkv) * p.Hq + (gk % p.Hkv) * p.G + hin;
 }
 __device__ __forceinline__ int q_n_kv(const BwdParams& p, int i) { return p.causal ? (i + 1) : p.nt; }
 
@@ -718,6 +727,7 @@ __global__ void __launch_bounds__(352, 1)
           uint32_t sr[16];
           tmem_ld16(sbase + q16 * 16, sr);
           tmem_wait_ld();
+          reg_fence(sr);
           bwd_exp16(sr, lv, c, masked, q16 * 16, 0, hi, pf + q16 * 16);
         }
         // phase B: dS = P (dP - D) -> bf16 over the S buffer
@@ -729,6 +739,7 @@ __global__ void __launch_bounds__(352, 1)
           uint32_t dr[16];
           tmem_ld16(lane_base + C::kDP + 64 * hb + q16 * 16, dr);
           tmem_wait_ld();
+          reg_fence(dr);
           uint32_t dk[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k)
@@ -757,6 +768,7 @@ __global__ void __launch_bounds__(352, 1)
         uint32_t x[32];
         tmem_ld32(lane_base + C::kDQ + q4 * 32, x);
         tmem_wait_ld();
+        reg_fence(x);
         if (live) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)

@@ -42,8 +42,9 @@ template <int D>
 struct FwdCfg {
   static constexpr int kTile = 128 * D * 2;          // bytes of one 128 x D bf16 tile
   static constexpr int kBox = 128 * 128;             // bytes of one 128 x 64 swizzled box
-  static constexpr int KST = (D == 128) ? 3 : 4;     // K ring stages
-  static constexpr int VST = (D == 128) ? 2 : 4;     // V ring stages
+  static constexpr int KST = 3;                      // K ring stages (== S buffers: S(g) frees stage g % 3)
+  static constexpr int VST = (D == 128) ? 2 : 3;     // V ring stages (<= 3, see FwdShared::pv_done)
+  static_assert(VST <= 3, "the V producer's waits on pv_done need VST <= 3");
   static constexpr int kThreads = 352;
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = 384;                  // O accumulator column
@@ -71,9 +72,16 @@ struct FwdShared {
   // epilogue's partial row sums go to the half the last tile did not use
   float xch[2][2][128];
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[4], k_empty[4];
-  uint64_t v_full[4], v_empty[4];
-  uint64_t s_full[3], p_ready[3], pv_done[3];
+  uint64_t k_full[3];        // K(g) landed in stage g % 3 (the stage is free again once S(g) completes)
+  uint64_t v_full[3];        // V(g) landed in stage g % VST
+  uint64_t s_full[3];        // S(g) complete in buffer g % 3; K stage g % 3 free
+  uint64_t p_ready[3];       // P(g) written over buffer g % 3 by both groups
+  // PV(g) complete (P(g) consumed, and V(g) read) on pv_done[g % 3].  Every wait
+  // on it targets a PV whose successor on the same barrier, PV(g + 3), cannot
+  // have completed yet: it needs P(g + 3), or for the V producer (VST <= 3)
+  // V(g + 3 - VST), which that producer has not loaded.  So a parity wait never
+  // sees the barrier two phases ahead.
+  uint64_t pv_done[3];
   uint64_t xbar[2];          // both groups posted their maxima for a tile
   uint64_t sbar;             // both groups posted their sums for a query tile
   uint64_t sread;            // both groups read the sums (the half may be reused)
@@ -84,12 +92,18 @@ struct FwdShared {
 };
 static_assert(sizeof(FwdShared) <= 2560, "FwdShared does not fit its slot");
 
-// Work tile t -> (query tile, batch*head).  Causal: longest rows first.
+// Work tile t -> (query tile, batch*head).  Tiles are numbered KV head by KV
+// head (the G query heads of a group interleaved), so the CTAs that run at the
+// same time read the same K/V and it is fetched from HBM about once; inside a
+// group, causal tiles go longest first.
 __device__ __forceinline__ void fwd_tile_coords(const FwdParams& p, int t, int& qt, int& bh) {
-  int BH = p.B * p.Hq;
-  int r = t / BH;
-  bh = t - r * BH;
-  qt = p.causal ? (p.n_qtiles - 1 - r) : r;
+  const int per_group = p.G * p.n_qtiles;
+  const int gk = t / per_group;                  // b * Hkv + kv-head
+  const int r = t - gk * per_group;
+  const int rq = r / p.G;
+  const int hin = r - rq * p.G;
+  qt = p.causal ? (p.n_qtiles - 1 - rq) : rq;
+  bh = (gk / p.Hkv) * p.Hq + (gk % p.Hkv) * p.G + hin;
 }
 
 __device__ __forceinline__ int fwd_n_kv(const FwdParams& p, int qt) {
@@ -118,12 +132,12 @@ __global__ void __launch_bounds__(352, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) { mbar_init(&sh.q_full[i], 1); mbar_init(&sh.q_empty[i], 1); }
-    for (int i = 0; i < C::KST; ++i) { mbar_init(&sh.k_full[i], 1); mbar_init(&sh.k_empty[i], 1); }
-    for (int i = 0; i < C::VST; ++i) { mbar_init(&sh.v_full[i], 1); mbar_init(&sh.v_empty[i], 1); }
+    for (int i = 0; i < C::VST; ++i) mbar_init(&sh.v_full[i], 1);
     for (int i = 0; i < 3; ++i) {
+      mbar_init(&sh.pv_done[i], 1);
+      mbar_init(&sh.k_full[i], 1);
       mbar_init(&sh.s_full[i], 1);
       mbar_init(&sh.p_ready[i], 8);
-      mbar_init(&sh.pv_done[i], 1);
     }
     mbar_init(&sh.xbar[0], 8);
     mbar_init(&sh.xbar[1], 8);
@@ -160,7 +174,7 @@ __global__ void __launch_bounds__(352, 1)
         nq = tl + 1;
         for (int s = 0; s < n_kv && ok; ++s) {
           const int g = it + s, st = g % C::KST;
-          if (g >= C::KST) ok = mbar_wait(&sh.k_empty[st], ((g / C::KST) - 1) & 1);
+          if (g >= C::KST) ok = mbar_wait(&sh.s_full[st], ((g / C::KST) - 1) & 1);   // S(g - 3) read K
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
           for (int c = 0; c < D / 64; ++c)
@@ -188,7 +202,10 @@ __global__ void __launch_bounds__(352, 1)
         const int bkv = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.G;
         for (int s = 0; s < n_kv && ok; ++s) {
           const int g = it + s, st = g % C::VST;
-          if (g >= C::VST) ok = mbar_wait(&sh.v_empty[st], ((g / C::VST) - 1) & 1);
+          if (g >= C::VST) {                                  // PV(g - VST) read stage st
+            const int gp = g - C::VST;
+            ok = mbar_wait(&sh.pv_done[gp % 3], (gp / 3) & 1);
+          }
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
           for (int c = 0; c < D / 64; ++c)
@@ -202,64 +219,78 @@ __global__ void __launch_bounds__(352, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
-      int it = 0, tl = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x, ++tl) {
-        int qt, bh;
-        fwd_tile_coords(p, t, qt, bh);
-        const int n_kv = fwd_n_kv(p, qt);
-        const int qb = tl & 1;
-        ok = mbar_wait(&sh.q_full[qb], (tl >> 1) & 1);
-        if (!ok) break;
+    // The whole warp follows the schedule (so descriptor arithmetic stays
+    // warp-uniform); one lane, elected once, issues every MMA and commit, so its
+    // final commit covers all of them.
+    const bool leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
+    constexpr uint32_t hi = sdesc_hi_sw128(1024);
+    const uint32_t q_lo0 = sdesc_lo(smem_u32(sQ), 16);
+    const uint32_t k_lo0 = sdesc_lo(smem_u32(sK), 16);
+    const uint32_t v_lo0 = sdesc_lo(smem_u32(sV), C::kBox);
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    };
+    int it = 0, tl = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x, ++tl) {
+      int qt, bh;
+      fwd_tile_coords(p, t, qt, bh);
+      const int n_kv = fwd_n_kv(p, qt);
+      const int qb = tl & 1;
+      ok = wait(&sh.q_full[qb], (tl >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t q_lo = q_lo0 + qb * (C::kTile >> 4);
+      // S(g) = Q K(g)^T into S buffer g % 3 (the buffer last held P(g - 3))
+      auto issue_s = [&](int j) -> bool {
+        const int g = it + j, sb = g % 3;
+        if (!wait(&sh.k_full[sb], (g / 3) & 1)) return false;
+        if (g >= 3 && !wait(&sh.pv_done[sb], ((g - 3) / 3) & 1)) return false;   // P(g - 3) consumed
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ + qb * C::kTile);
-        // S(g) = Q K(g)^T into S buffer g % 3 (the buffer last held P(g - 3))
-        auto issue_s = [&](int j) -> bool {
-          const int g = it + j, kst = g % C::KST, sb = g % 3;
-          if (!mbar_wait(&sh.k_full[kst], (g / C::KST) & 1)) return false;
-          if (g >= 3 && !mbar_wait(&sh.pv_done[sb], ((g / 3) - 1) & 1)) return false;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sK + kst * C::kTile);
+        const uint32_t k_lo = k_lo0 + sb * (C::kTile >> 4);
+        if (leader) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-            umma_ss(tmem + sb * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                    idS, k > 0);
+            const uint32_t off = ((k >> 2) * C::kBox + (k & 3) * 32) >> 4;
+            umma_ss_lo(tmem + sb * 128, q_lo + off, k_lo + off, hi, idS, k > 0);
           }
           umma_commit(&sh.s_full[sb]);
-          umma_commit(&sh.k_empty[kst]);
           if (j == n_kv - 1) umma_commit(&sh.q_empty[qb]);
-          return true;
-        };
-        // S runs two tiles ahead of PV, so the softmax groups can load S(j+1) while
-        // they exponentiate tile j.
-        ok = issue_s(0) && (n_kv < 2 || issue_s(1));
-        for (int j = 0; j < n_kv && ok; ++j) {
-          if (j + 2 < n_kv && !issue_s(j + 2)) { ok = false; break; }
-          // O (+)= P(g) V(g); P keys 0-63 in columns 0-31, keys 64-127 in 64-95
-          const int g = it + j, vst = g % C::VST, sb = g % 3;
-          ok = mbar_wait(&sh.v_full[vst], (g / C::VST) & 1);
-          if (ok) ok = mbar_wait(&sh.p_ready[sb], (g / 3) & 1);
-          if (ok && j == 0 && tl >= 1) ok = mbar_wait(&sh.o_free, (tl - 1) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(sV + vst * C::kTile);
+        }
+        __syncwarp();
+        return true;
+      };
+      // S runs two tiles ahead of PV, so the softmax groups can load S(j+1) while
+      // they exponentiate tile j.
+      ok = issue_s(0) && (n_kv < 2 || issue_s(1));
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 2 < n_kv && !issue_s(j + 2)) { ok = false; break; }
+        // O (+)= P(g) V(g); P keys 0-63 in columns 0-31, keys 64-127 in 64-95
+        const int g = it + j, vst = g % C::VST, sb = g % 3;
+        ok = wait(&sh.v_full[vst], (g / C::VST) & 1) && wait(&sh.p_ready[sb], (g / 3) & 1);
+        if (ok && j == 0 && tl >= 1) ok = wait(&sh.o_free, (tl - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t v_lo = v_lo0 + vst * (C::kTile >> 4);
+        if (leader) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + C::kOCol, tmem + sb * 128 + (k >> 2) * 64 + (k & 3) * 8,
-                    sdesc_sw128(v_addr + k * 2048, C::kBox, 1024), idO, (j > 0 || k > 0));
+            umma_ts_lo(tmem + C::kOCol, tmem + sb * 128 + (k >> 2) * 64 + (k & 3) * 8, v_lo + ((k * 2048) >> 4), hi,
+                       idO, (j > 0 || k > 0));
           umma_commit(&sh.pv_done[sb]);
-          umma_commit(&sh.v_empty[vst]);
         }
-        it += n_kv;
+        __syncwarp();
       }
-      // Drain every MMA this thread issued before TMEM is released.
+      it += n_kv;
+    }
+    // Drain every MMA this warp issued before TMEM is released.
+    if (leader) {
       umma_commit(&sh.drain);
       mbar_wait(&sh.drain, 0);
     }
+    __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warpgroups
     const int hb = warp >> 2;                                   // 0: keys 0-63, 1: keys 64-127
@@ -288,6 +319,19 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int k = 0; k < 32; ++k)
           if (col0 + k > lim) r[k] = 0xff800000u;
+      };
+      auto mask16 = [&](uint32_t (&r)[16], int col0, int lim) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          if (col0 + k > lim) r[k] = 0xff800000u;
+      };
+      auto max16 = [&](float (&mx4)[4], const uint32_t (&r)[16]) {
+#pragma unroll
+        for (int k = 0; k < 16; k += 8) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            mx4[e] = max3f(mx4[e], __uint_as_float(r[k + e]), __uint_as_float(r[k + e + 4]));
+        }
       };
       auto max32 = [&](float (&mx4)[4], const uint32_t (&r)[32]) {
 #pragma unroll
@@ -323,6 +367,7 @@ __global__ void __launch_bounds__(352, 1)
           uint32_t r[32];
           tmem_ld32(lane_base + sb * 128 + hb * 64 + cc * 32, r);
           tmem_wait_ld();
+          reg_fence(r);
           if (msk) mask32(r, cc * 32, lim);
           max32(mx4, r);
         }
@@ -359,16 +404,26 @@ __global__ void __launch_bounds__(352, 1)
         const bool mskn = __any_sync(0xffffffffu, limn < 63);
         const uint64_t nm2 = f2pack(-m_used, -m_used);
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // Four chunks of 16 columns; the TMEM loads of chunk cc+1 are in flight
+        // while chunk cc is exponentiated.  P chunk cc goes to columns 8cc..8cc+7
+        // of this group's half, all below the S columns still to be read.
+        const uint32_t s_col = lane_base + sb * 128 + hb * 64;
+        const uint32_t sn_col = lane_base + sbn * 128 + hb * 64;
+        uint32_t ra[16], rb[16], rna[16], rnb[16];
+        tmem_ld16(s_col, ra);
+        if (has_next) tmem_ld16(sn_col, rna);
+        tmem_wait_ld();
+        reg_fence(ra);
+        if (has_next) reg_fence(rna);
+        auto chunk = [&](int cc, uint32_t (&r)[16], uint32_t (&rn)[16], uint32_t (&r2)[16], uint32_t (&rn2)[16]) {
+          if (cc < 3) {
+            tmem_ld16(s_col + (cc + 1) * 16, r2);
+            if (has_next) tmem_ld16(sn_col + (cc + 1) * 16, rn2);
+          }
+          if (msk) mask16(r, cc * 16, lim);
+          uint32_t pk[8];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t r[32], rn[32];
-          tmem_ld32(lane_base + sb * 128 + hb * 64 + cc * 32, r);
-          if (has_next) tmem_ld32(lane_base + sbn * 128 + hb * 64 + cc * 32, rn);
-          tmem_wait_ld();
-          if (msk) mask32(r, cc * 32, lim);
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < 8; ++k) {
             const uint64_t x = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
             float x0, x1, a, b;
             f2unpack(x, x0, x1);
@@ -381,12 +436,21 @@ __global__ void __launch_bounds__(352, 1)
             lsum = fadd2(lsum, f2pack(a, b));
             pk[k] = pack_bf16x2(a, b);
           }
-          tmem_st16(lane_base + sb * 128 + hb * 64 + cc * 16, pk);
+          tmem_st8(s_col + cc * 8, pk);
           if (has_next) {
-            if (mskn) mask32(rn, cc * 32, limn);
-            max32(mx4, rn);
+            if (mskn) mask16(rn, cc * 16, limn);
+            max16(mx4, rn);
           }
-        }
+          if (cc < 3) {
+            tmem_wait_ld();
+            reg_fence(r2);
+            if (has_next) reg_fence(rn2);
+          }
+        };
+        chunk(0, ra, rna, rb, rnb);
+        chunk(1, rb, rnb, ra, rna);
+        chunk(2, ra, rna, rb, rnb);
+        chunk(3, rb, rnb, ra, rna);
         if (has_next) {
           ok = post(j + 1, mx4);
           if (!ok) break;
@@ -402,6 +466,7 @@ __global__ void __launch_bounds__(352, 1)
             uint32_t o[32];
             tmem_ld32(o_base + q4 * 32, o);
             tmem_wait_ld();
+            reg_fence(o);
 #pragma unroll
             for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
             tmem_st32(o_base + q4 * 32, o);
@@ -437,6 +502,7 @@ __global__ void __launch_bounds__(352, 1)
         uint32_t o[32];
         tmem_ld32(o_base + q4 * 32, o);
         tmem_wait_ld();
+        reg_fence(o);
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
