@@ -7,22 +7,25 @@
 // output is rescaled by exp(m_old - m_new) when the max grows, and only O and the
 // log-sum-exp leave the chip.  S and P never reach HBM.
 //
-// B200 mapping (one persistent CTA per SM, 352 threads):
-//   warps 0-3  softmax warpgroup A: keys 0-63 of every S tile, O columns [0, D/2)
-//   warps 4-7  softmax warpgroup B: keys 64-127, O columns [D/2, D)
-//              thread = one query row = one TMEM lane.  The two groups exchange
-//              their partial row maxima through shared memory once per tile, so
-//              both take the same rescale decisions; each keeps its own partial
-//              row sum, combined in the epilogue.
-//   warp 8     TMA producer for Q (double buffered) and the K ring
-//   warp 10    TMA producer for the V ring (its own stream, so a K load never
+// B200 mapping (one persistent CTA per SM, 608 threads = 19 warps):
+//   warps 0-15 softmax: group k = warp / 4 (k = 0..3) owns keys [32k, 32k+32) of
+//              every S tile and O columns [k*D/4, (k+1)*D/4); thread = one query
+//              row = one TMEM lane (warp w reaches lanes 32*(w%4)..+31).  The four
+//              warps that share a row quadrant sit on the same SM sub-partition,
+//              so each sub-partition runs four softmax warps, enough to keep its
+//              MUFU pipe busy.  The groups exchange partial row maxima through
+//              shared memory once per tile (so all take the same rescale
+//              decisions) and partial row sums once per query tile.
+//   warp 16    TMA producer for Q (double buffered) and the K ring
+//   warp 17    MMA issuer: S = Q K^T (SS, both K-major) and O += P V (A = P from
+//              TMEM, B = V MN-major), accumulating in TMEM.
+//   warp 18    TMA producer for the V ring (its own stream, so a K load never
 //              queues behind a V load that waits for a free stage)
-//   warp 9     MMA issuer (one thread): S = Q K^T (SS, both K-major) and
-//              O += P V (A = P from TMEM, B = V MN-major), accumulating in TMEM.
 // TMEM (512 columns): three 128-column S/P buffers, then O (D columns).  Three
-// S buffers let S(j+1) be issued while P(j-1) may still be read by its PV MMA.
-// P(j) (bf16) is written over the S buffer: keys 0-63 in columns 0-31, keys
-// 64-127 in columns 64-95, so neither group overwrites columns the other reads.
+// S buffers let S(j+2) be issued while P(j-1) may still be read by its PV MMA.
+// P(j) (bf16) is written over the S buffer: group k's 32 keys go to columns
+// 32k..32k+15, inside its own S columns, so no group overwrites scores another
+// group still reads.
 //
 // exp2 with a folded scale: c = scale * log2(e), p = exp2(s*c - m) where m is
 // kept in log2 units; LSE = ln(2) * (m + log2 l).  The max used for the
@@ -45,7 +48,8 @@ struct FwdCfg {
   static constexpr int KST = 3;                      // K ring stages (== S buffers: S(g) frees stage g % 3)
   static constexpr int VST = (D == 128) ? 2 : 3;     // V ring stages (<= 3, see FwdShared::pv_done)
   static_assert(VST <= 3, "the V producer's waits on pv_done need VST <= 3");
-  static constexpr int kThreads = 352;
+  static constexpr int kGroups = 4;                  // softmax groups of 4 warps
+  static constexpr int kThreads = 608;
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = 384;                  // O accumulator column
   static constexpr int kOffQ = 0;                    // 2 tiles
@@ -68,9 +72,14 @@ struct FwdParams {
 };
 
 struct FwdShared {
-  // [parity][group][row]: partial row maxima of tile g live in xch[g & 1]; the
-  // epilogue's partial row sums go to the half the last tile did not use
-  float xch[2][2][128];
+  // Partial row maxima of tile g: xmax[g & 1][group][row], as bf16 rounded
+  // upward (the common maximum is only the exponent's reference point, and any
+  // value at or above the true maximum works).  Once every group has finished
+  // its last tile of a query tile, the same bytes carry the partial row sums.
+  union {
+    uint16_t xmax[2][4][128];
+    float xsum[4][128];
+  } x;
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[3];        // K(g) landed in stage g % 3 (the stage is free again once S(g) completes)
   uint64_t v_full[3];        // V(g) landed in stage g % VST
@@ -83,8 +92,9 @@ struct FwdShared {
   // sees the barrier two phases ahead.
   uint64_t pv_done[3];
   uint64_t xbar[2];          // both groups posted their maxima for a tile
-  uint64_t sbar;             // both groups posted their sums for a query tile
-  uint64_t sread;            // both groups read the sums (the half may be reused)
+  uint64_t ebar;             // every group is done with the maxima of a query tile
+  uint64_t sbar;             // every group posted its sum for a query tile
+  uint64_t sread;            // every group read the sums (the bytes may be reused)
   uint64_t o_free;
   uint64_t drain;
   uint64_t teardown;         // every warp is done with TMEM
@@ -112,7 +122,7 @@ __device__ __forceinline__ int fwd_n_kv(const FwdParams& p, int qt) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(608, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
   using C = FwdCfg<D>;
@@ -137,15 +147,16 @@ __global__ void __launch_bounds__(352, 1)
       mbar_init(&sh.pv_done[i], 1);
       mbar_init(&sh.k_full[i], 1);
       mbar_init(&sh.s_full[i], 1);
-      mbar_init(&sh.p_ready[i], 8);
+      mbar_init(&sh.p_ready[i], 16);
     }
-    mbar_init(&sh.xbar[0], 8);
-    mbar_init(&sh.xbar[1], 8);
-    mbar_init(&sh.sbar, 8);
-    mbar_init(&sh.sread, 8);
-    mbar_init(&sh.o_free, 8);
+    mbar_init(&sh.xbar[0], 16);
+    mbar_init(&sh.xbar[1], 16);
+    mbar_init(&sh.ebar, 16);
+    mbar_init(&sh.sbar, 16);
+    mbar_init(&sh.sread, 16);
+    mbar_init(&sh.o_free, 16);
     mbar_init(&sh.drain, 1);
-    mbar_init(&sh.teardown, 11);
+    mbar_init(&sh.teardown, 19);
     fence_barrier_init();
   }
   if (warp == 0) { tmem_alloc(&sh.tmem_base, C::kTmemCols); tmem_relinquish(); }
@@ -154,7 +165,7 @@ __global__ void __launch_bounds__(352, 1)
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ TMA producer: Q and K
     if (lane == 0) {
       tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk);
@@ -189,7 +200,7 @@ __global__ void __launch_bounds__(352, 1)
         for (int g = max(0, nq - 2); g < nq; ++g) mbar_drain_wait(&sh.q_full[g & 1], (g >> 1) & 1);
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == 18) {
     // ------------------------------------------------------------ TMA producer: V
     if (lane == 0) {
       tma_prefetch_desc(&tmv);
@@ -217,7 +228,7 @@ __global__ void __launch_bounds__(352, 1)
       if (!ok)
         for (int g = max(0, nv - C::VST); g < nv; ++g) mbar_drain_wait(&sh.v_full[g % C::VST], (g / C::VST) & 1);
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp follows the schedule (so descriptor arithmetic stays
     // warp-uniform); one lane, elected once, issues every MMA and commit, so its
@@ -267,7 +278,7 @@ __global__ void __launch_bounds__(352, 1)
       ok = issue_s(0) && (n_kv < 2 || issue_s(1));
       for (int j = 0; j < n_kv && ok; ++j) {
         if (j + 2 < n_kv && !issue_s(j + 2)) { ok = false; break; }
-        // O (+)= P(g) V(g); P keys 0-63 in columns 0-31, keys 64-127 in 64-95
+        // O (+)= P(g) V(g); keys 16kk..16kk+15 of P sit at column 32*(kk/2) + 8*(kk%2)
         const int g = it + j, vst = g % C::VST, sb = g % 3;
         ok = wait(&sh.v_full[vst], (g / C::VST) & 1) && wait(&sh.p_ready[sb], (g / 3) & 1);
         if (ok && j == 0 && tl >= 1) ok = wait(&sh.o_free, (tl - 1) & 1);
@@ -277,7 +288,7 @@ __global__ void __launch_bounds__(352, 1)
         if (leader) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts_lo(tmem + C::kOCol, tmem + sb * 128 + (k >> 2) * 64 + (k & 3) * 8, v_lo + ((k * 2048) >> 4), hi,
+            umma_ts_lo(tmem + C::kOCol, tmem + sb * 128 + (k >> 1) * 32 + (k & 1) * 8, v_lo + ((k * 2048) >> 4), hi,
                        idO, (j > 0 || k > 0));
           umma_commit(&sh.pv_done[sb]);
         }
@@ -291,13 +302,14 @@ __global__ void __launch_bounds__(352, 1)
       mbar_wait(&sh.drain, 0);
     }
     __syncwarp();
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int hb = warp >> 2;                                   // 0: keys 0-63, 1: keys 64-127
-    const int row = (warp & 3) * 32 + lane;                     // TMEM lane == tile row
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    constexpr int OH = D / 2;                                   // O columns per group
-    const uint32_t o_base = lane_base + C::kOCol + hb * OH;
+  } else if (warp < 16) {
+    // ------------------------------------------------------------ softmax groups
+    const int grp = warp >> 2;                                  // keys [32 grp, 32 grp + 32)
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;                           // TMEM lane == tile row
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    constexpr int OQ = D / 4;                                   // O columns per group
+    const uint32_t o_base = lane_base + C::kOCol + grp * OQ;
     const float c = p.c;
     const uint64_t c2 = f2pack(c, c);
     int it = 0, tl = 0;
@@ -309,16 +321,11 @@ __global__ void __launch_bounds__(352, 1)
       const int qrow = qt * 128 + row;
       float m_used = -INFINITY;
       uint64_t lsum = f2pack(0.f, 0.f);                         // two partial sums
-      // last visible key of this row within this group's 64 columns of tile j
+      // last visible key of this row within this group's 32 columns of tile j
       auto last_col = [&](int j) -> int {
-        const int kbase = j * 128 + hb * 64;
+        const int kbase = j * 128 + grp * 32;
         const int lim = p.N - 1 - kbase;
         return p.causal ? min(lim, qrow - kbase) : lim;
-      };
-      auto mask32 = [&](uint32_t (&r)[32], int col0, int lim) {
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (col0 + k > lim) r[k] = 0xff800000u;
       };
       auto mask16 = [&](uint32_t (&r)[16], int col0, int lim) {
 #pragma unroll
@@ -333,22 +340,14 @@ __global__ void __launch_bounds__(352, 1)
             mx4[e] = max3f(mx4[e], __uint_as_float(r[k + e]), __uint_as_float(r[k + e + 4]));
         }
       };
-      auto max32 = [&](float (&mx4)[4], const uint32_t (&r)[32]) {
-#pragma unroll
-        for (int k = 0; k < 32; k += 8) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            mx4[e] = max3f(mx4[e], __uint_as_float(r[k + e]), __uint_as_float(r[k + e + 4]));
-        }
-      };
-      // post this group's partial max of tile j for the other group
+      // post this group's partial max of tile j for the other groups
       auto post = [&](int j, const float (&mx4)[4]) -> bool {
         const int g = it + j, xp = g & 1;
         const float pm = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        if (j == 0 && tl >= 1) {       // the previous epilogue's sums used this half
+        if (j == 0 && tl >= 1) {       // the previous query tile's sums used these bytes
           if (!__all_sync(0xffffffffu, mbar_wait(&sh.sread, (tl - 1) & 1))) return false;
         }
-        sh.xch[xp][hb][row] = pm;
+        sh.x.xmax[xp][grp][row] = bf16_bits_round_up(pm);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.xbar[xp]);
         return true;
@@ -360,28 +359,29 @@ __global__ void __launch_bounds__(352, 1)
         if (!ok) break;
         tc_fence_after();
         const int lim = last_col(0);
-        const bool msk = __any_sync(0xffffffffu, lim < 63);
+        const bool msk = __any_sync(0xffffffffu, lim < 31);
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(lane_base + sb * 128 + hb * 64 + cc * 32, r);
-          tmem_wait_ld();
-          reg_fence(r);
-          if (msk) mask32(r, cc * 32, lim);
-          max32(mx4, r);
-        }
+        uint32_t r0[16], r1[16];
+        tmem_ld16(lane_base + sb * 128 + grp * 32, r0);
+        tmem_ld16(lane_base + sb * 128 + grp * 32 + 16, r1);
+        tmem_wait_ld();
+        reg_fence(r0);
+        reg_fence(r1);
+        if (msk) { mask16(r0, 0, lim); mask16(r1, 16, lim); }
+        max16(mx4, r0);
+        max16(mx4, r1);
         ok = post(0, mx4);
         if (!ok) break;
       }
-      // Tile j: take the common max, exponentiate its scores chunk by chunk while the
-      // same chunk of tile j+1 is read for that tile's max, write P, rescale O if the
-      // max moved, hand P to the MMA warp.
+      // Tile j: take the common max, exponentiate its scores in two chunks of 16
+      // while the same columns of tile j+1 are read for that tile's max, write P,
+      // rescale this group's O columns if the max moved, hand P to the MMA warp.
       for (int j = 0; j < n_kv && ok; ++j) {
         const int g = it + j, sb = g % 3, xp = g & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.xbar[xp], (g >> 1) & 1));
         if (!ok) break;
-        const float m_tile = fmaxf(sh.xch[xp][0][row], sh.xch[xp][1][row]) * c;
+        const float m_tile = fmaxf(fmaxf(bf16_bits_to_float(sh.x.xmax[xp][0][row]), bf16_bits_to_float(sh.x.xmax[xp][1][row])),
+                                   fmaxf(bf16_bits_to_float(sh.x.xmax[xp][2][row]), bf16_bits_to_float(sh.x.xmax[xp][3][row]))) * c;
         float alpha = 1.f;
         const bool need = (m_used == -INFINITY) || (m_tile > m_used + kRescaleTau);
         if (need) {
@@ -400,26 +400,20 @@ __global__ void __launch_bounds__(352, 1)
         }
         tc_fence_after();
         const int lim = last_col(j), limn = last_col(j + 1);
-        const bool msk = __any_sync(0xffffffffu, lim < 63);
-        const bool mskn = __any_sync(0xffffffffu, limn < 63);
+        const bool msk = __any_sync(0xffffffffu, lim < 31);
+        const bool mskn = __any_sync(0xffffffffu, limn < 31);
         const uint64_t nm2 = f2pack(-m_used, -m_used);
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        // Four chunks of 16 columns; the TMEM loads of chunk cc+1 are in flight
-        // while chunk cc is exponentiated.  P chunk cc goes to columns 8cc..8cc+7
-        // of this group's half, all below the S columns still to be read.
-        const uint32_t s_col = lane_base + sb * 128 + hb * 64;
-        const uint32_t sn_col = lane_base + sbn * 128 + hb * 64;
-        uint32_t ra[16], rb[16], rna[16], rnb[16];
-        tmem_ld16(s_col, ra);
-        if (has_next) tmem_ld16(sn_col, rna);
-        tmem_wait_ld();
-        reg_fence(ra);
-        if (has_next) reg_fence(rna);
-        auto chunk = [&](int cc, uint32_t (&r)[16], uint32_t (&rn)[16], uint32_t (&r2)[16], uint32_t (&rn2)[16]) {
-          if (cc < 3) {
-            tmem_ld16(s_col + (cc + 1) * 16, r2);
-            if (has_next) tmem_ld16(sn_col + (cc + 1) * 16, rn2);
-          }
+        const uint32_t s_col = lane_base + sb * 128 + grp * 32;
+        const uint32_t sn_col = lane_base + sbn * 128 + grp * 32;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t r[16], rn[16];
+          tmem_ld16(s_col + cc * 16, r);
+          if (has_next) tmem_ld16(sn_col + cc * 16, rn);
+          tmem_wait_ld();
+          reg_fence(r);
+          if (has_next) reg_fence(rn);
           if (msk) mask16(r, cc * 16, lim);
           uint32_t pk[8];
 #pragma unroll
@@ -427,12 +421,8 @@ __global__ void __launch_bounds__(352, 1)
             const uint64_t x = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
             float x0, x1, a, b;
             f2unpack(x, x0, x1);
-            if ((k & 3) == 3) {
-              exp2_fma_pair(x0, x1, a, b);          // one pair in four on the FMA pipe
-            } else {
-              a = ex2_approx(x0);
-              b = ex2_approx(x1);
-            }
+            a = ex2_approx(x0);
+            b = ex2_approx(x1);
             lsum = fadd2(lsum, f2pack(a, b));
             pk[k] = pack_bf16x2(a, b);
           }
@@ -441,35 +431,33 @@ __global__ void __launch_bounds__(352, 1)
             if (mskn) mask16(rn, cc * 16, limn);
             max16(mx4, rn);
           }
-          if (cc < 3) {
-            tmem_wait_ld();
-            reg_fence(r2);
-            if (has_next) reg_fence(rn2);
-          }
-        };
-        chunk(0, ra, rna, rb, rnb);
-        chunk(1, rb, rnb, ra, rna);
-        chunk(2, ra, rna, rb, rnb);
-        chunk(3, rb, rnb, ra, rna);
+        }
         if (has_next) {
           ok = post(j + 1, mx4);
           if (!ok) break;
         }
-        // Rescale this group's half of the running output when its max moved.
+        // Rescale this group's columns of the running output when its max moved.
         if (__any_sync(0xffffffffu, need && j > 0)) {
           const int gp = g - 1;
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[gp % 3], (gp / 3) & 1));
           if (!ok) break;
           tc_fence_after();
-#pragma unroll
-          for (int q4 = 0; q4 < OH / 32; ++q4) {
+          if constexpr (OQ == 32) {
             uint32_t o[32];
-            tmem_ld32(o_base + q4 * 32, o);
+            tmem_ld32(o_base, o);
             tmem_wait_ld();
             reg_fence(o);
 #pragma unroll
             for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(o_base + q4 * 32, o);
+            tmem_st32(o_base, o);
+          } else {
+            uint32_t o[16];
+            tmem_ld16(o_base, o);
+            tmem_wait_ld();
+            reg_fence(o);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st16(o_base, o);
           }
         }
         tmem_wait_st();
@@ -478,17 +466,19 @@ __global__ void __launch_bounds__(352, 1)
         if (lane == 0) mbar_arrive(&sh.p_ready[sb]);
       }
       if (!ok) break;
-      // epilogue: combine the two partial sums, wait for the last PV, O / l -> bf16, LSE
+      // epilogue: combine the partial sums, wait for the last PV, O / l -> bf16, LSE
       const int glast = it + n_kv - 1;
-      const int xs = (glast + 1) & 1;
+      if (lane == 0) mbar_arrive(&sh.ebar);                    // done reading this tile's maxima
+      ok = __all_sync(0xffffffffu, mbar_wait(&sh.ebar, tl & 1));
+      if (!ok) break;
       float l0, l1;
       f2unpack(lsum, l0, l1);
-      sh.xch[xs][hb][row] = l0 + l1;
+      sh.x.xsum[grp][row] = l0 + l1;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.sbar);
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.sbar, tl & 1));
       if (!ok) break;
-      const float l = sh.xch[xs][0][row] + sh.xch[xs][1][row];
+      const float l = (sh.x.xsum[0][row] + sh.x.xsum[1][row]) + (sh.x.xsum[2][row] + sh.x.xsum[3][row]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.sread);
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[glast % 3], (glast / 3) & 1));
@@ -496,24 +486,23 @@ __global__ void __launch_bounds__(352, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool live = qrow < p.N;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D + hb * OH;
-#pragma unroll
-      for (int q4 = 0; q4 < OH / 32; ++q4) {
-        uint32_t o[32];
-        tmem_ld32(o_base + q4 * 32, o);
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D + grp * OQ;
+      {
+        uint32_t o[OQ];
+        if constexpr (OQ == 32) tmem_ld32(o_base, o); else tmem_ld16(o_base, o);
         tmem_wait_ld();
         reg_fence(o);
-        uint32_t pk[16];
+        uint32_t pk[OQ / 2];
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
+        for (int k = 0; k < OQ / 2; ++k)
           pk[k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
         if (live) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
+          uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          for (int k = 0; k < OQ / 8; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      if (live && hb == 0) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      if (live && grp == 0) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + __log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.o_free);

@@ -392,6 +392,17 @@ __device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float& y0, flo
   y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
+// bf16 bit pattern of x rounded toward +infinity (positive finite values round
+// their magnitude up; negative values and infinities truncate, which is upward).
+__device__ __forceinline__ uint16_t bf16_bits_round_up(float x) {
+  uint32_t b = __float_as_uint(x);
+  if (x > 0.f && b < 0x7f800000u) b += 0xFFFFu;
+  return static_cast<uint16_t>(b >> 16);
+}
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t v) {
+  return __uint_as_float(static_cast<uint32_t>(v) << 16);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

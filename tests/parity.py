@@ -4,7 +4,12 @@ Forward, per element:  |dO| <= 1e-2 + half a bf16 ulp of |O_ref|  (an exactly co
   O rounded to bf16 already misses 1e-2 once |O| >= 2, so the bf16 rounding of the
   output itself is allowed on top of the 1e-2 budget);
   relative RMS over the tensor <= 5e-3;  |dLSE| <= 1e-3 (LSE stays fp32).
-Gradients, per tensor: max |d| <= 2e-2 * max(1, max |ref|), relative RMS <= 1e-2.
+Gradients, per tensor: max |d| <= 2e-2 * max(1, max |ref|) (the stated gradient gate),
+  plus a relative RMS <= 2e-2 of our own.  The backward takes O as a bf16 input, so
+  D_i = sum_k dO_ik O_ik carries the rounding of O (about 2^-9 relative per element);
+  on a causal row with one or two visible keys that error does not average out, and
+  dQ of rows 1-2 of a head lands a few percent off in relative terms (about 8e-3
+  absolute for |dQ| ~ 0.1), which dominates a sampled relative RMS.
 All of these reduce to the plain 1e-2 / 5e-3 / 1e-3 / 2e-2 bounds wherever values are O(1).
 """
 import numpy as np
@@ -14,7 +19,7 @@ O_ATOL = 1e-2
 O_RRMS = 5e-3
 LSE_ATOL = 1e-3
 G_REL = 2e-2
-G_RRMS = 1e-2
+G_RRMS = 2e-2
 
 
 def f64(t):
