@@ -373,9 +373,14 @@ __global__ void __launch_bounds__(608, 1)
         ok = post(0, mx4);
         if (!ok) break;
       }
-      // Tile j: take the common max, exponentiate its scores in two chunks of 16
-      // while the same columns of tile j+1 are read for that tile's max, write P,
-      // rescale this group's O columns if the max moved, hand P to the MMA warp.
+      // Tile j: (1) take the common max of tile j; (2) read this group's columns of
+      // tile j+1 and post their max at once, so the other groups find it long before
+      // they need it and the groups can drift apart by most of a tile (one group's
+      // waits then overlap another's exponentials); (3) exponentiate tile j in two
+      // chunks of 16 columns, write P; (4) rescale this group's O columns if the max
+      // moved, hand P to the MMA warp.  A group posts j+1 only after it has read the
+      // maxima of j, and reaches j only once every group has posted j, i.e. has read
+      // j-1: so two parity slots suffice.
       for (int j = 0; j < n_kv && ok; ++j) {
         const int g = it + j, sb = g % 3, xp = g & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.xbar[xp], (g >> 1) & 1));
@@ -392,28 +397,36 @@ __global__ void __launch_bounds__(608, 1)
           lsum = f2pack(l0 * alpha, l1 * alpha);
           m_used = m_new;
         }
-        const bool has_next = j + 1 < n_kv;
-        const int sbn = (g + 1) % 3;
-        if (has_next) {
+        if (j + 1 < n_kv) {
+          const int sbn = (g + 1) % 3;
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[sbn], ((g + 1) / 3) & 1));
           if (!ok) break;
+          tc_fence_after();
+          const int limn = last_col(j + 1);
+          const bool mskn = __any_sync(0xffffffffu, limn < 31);
+          uint32_t rn0[16], rn1[16];
+          tmem_ld16(lane_base + sbn * 128 + grp * 32, rn0);
+          tmem_ld16(lane_base + sbn * 128 + grp * 32 + 16, rn1);
+          tmem_wait_ld();
+          reg_fence(rn0);
+          reg_fence(rn1);
+          if (mskn) { mask16(rn0, 0, limn); mask16(rn1, 16, limn); }
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          max16(mx4, rn0);
+          max16(mx4, rn1);
+          ok = post(j + 1, mx4);
+          if (!ok) break;
         }
-        tc_fence_after();
-        const int lim = last_col(j), limn = last_col(j + 1);
+        const int lim = last_col(j);
         const bool msk = __any_sync(0xffffffffu, lim < 31);
-        const bool mskn = __any_sync(0xffffffffu, limn < 31);
         const uint64_t nm2 = f2pack(-m_used, -m_used);
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         const uint32_t s_col = lane_base + sb * 128 + grp * 32;
-        const uint32_t sn_col = lane_base + sbn * 128 + grp * 32;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          uint32_t r[16], rn[16];
+          uint32_t r[16];
           tmem_ld16(s_col + cc * 16, r);
-          if (has_next) tmem_ld16(sn_col + cc * 16, rn);
           tmem_wait_ld();
           reg_fence(r);
-          if (has_next) reg_fence(rn);
           if (msk) mask16(r, cc * 16, lim);
           uint32_t pk[8];
 #pragma unroll
@@ -427,14 +440,6 @@ __global__ void __launch_bounds__(608, 1)
             pk[k] = pack_bf16x2(a, b);
           }
           tmem_st8(s_col + cc * 8, pk);
-          if (has_next) {
-            if (mskn) mask16(rn, cc * 16, limn);
-            max16(mx4, rn);
-          }
-        }
-        if (has_next) {
-          ok = post(j + 1, mx4);
-          if (!ok) break;
         }
         // Rescale this group's columns of the running output when its max moved.
         if (__any_sync(0xffffffffu, need && j > 0)) {
