@@ -272,81 +272,102 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ MMA issuer
     // Order per step g:  dV(g) S^T(g+1) dK(g) dP^T(g+1).  The exps of step g+1
     // (phase A) run under dK(g) and dP^T(g+1); dS of step g (phase B) under dV(g)
-    // and S^T(g+1).
-    if (lane == 0) {
-      constexpr uint32_t idST = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
-      constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);      // dV, dK
-      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      int gs = 0, it = 0;
-      bool ok = true;
-      auto issue_st = [&](int g) -> bool {   // S^T(g) = K Q(g)^T
-        const int st = g & 1;
-        if (!mbar_wait(&sh.qdo_full[st], (g >> 1) & 1)) return false;
-        if (g >= 1 && !mbar_wait(&sh.v_done, (g - 1) & 1)) return false;      // P^T(g-1) consumed
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ + st * C::kTile);
+    // and S^T(g+1).  The whole warp follows the schedule (descriptor arithmetic
+    // stays warp-uniform); one lane, elected once, issues every MMA and commit.
+    const bool leader = elect_one();
+    constexpr uint32_t idST = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+    constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);      // dV, dK
+    constexpr uint32_t hi = sdesc_hi_sw128(1024);
+    const uint32_t k_lo = sdesc_lo(smem_u32(sK), 16), v_lo = sdesc_lo(smem_u32(sV), 16);
+    const uint32_t q_lo0 = sdesc_lo(smem_u32(sQ), 16), do_lo0 = sdesc_lo(smem_u32(sDO), 16);
+    const uint32_t q_mn0 = sdesc_lo(smem_u32(sQ), C::kBox), do_mn0 = sdesc_lo(smem_u32(sDO), C::kBox);
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    };
+    int gs = 0, it = 0;
+    bool ok = true;
+    auto issue_st = [&](int g) -> bool {   // S^T(g) = K Q(g)^T
+      const int st = g & 1;
+      if (!wait(&sh.qdo_full[st], (g >> 1) & 1)) return false;
+      if (g >= 1 && !wait(&sh.v_done, (g - 1) & 1)) return false;      // P^T(g-1) consumed
+      tc_fence_after();
+      if (leader) {
+        const uint32_t q_lo = q_lo0 + st * (C::kTile >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-          umma_ss(tmem + C::kS, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idST,
-                  k > 0);
+          const uint32_t off = ((k >> 2) * C::kBox + (k & 3) * 32) >> 4;
+          umma_ss_lo(tmem + C::kS, k_lo + off, q_lo + off, hi, idST, k > 0);
         }
         umma_commit(&sh.s_full);
-        return true;
-      };
-      auto issue_dp = [&](int g) -> bool {   // dP^T(g) = V dO(g)^T
-        const int st = g & 1;
-        if (g >= 1 && !mbar_wait(&sh.k_done, (g - 1) & 1)) return false;      // dS^T(g-1) consumed
-        tc_fence_after();
-        const uint32_t do_addr = smem_u32(sDO + st * C::kTile);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_dp = [&](int g) -> bool {   // dP^T(g) = V dO(g)^T
+      const int st = g & 1;
+      if (g >= 1 && !wait(&sh.k_done, (g - 1) & 1)) return false;      // dS^T(g-1) consumed
+      tc_fence_after();
+      if (leader) {
+        const uint32_t do_lo = do_lo0 + st * (C::kTile >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-          umma_ss(tmem + C::kDP, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
-                  idST, k > 0);
+          const uint32_t off = ((k >> 2) * C::kBox + (k & 3) * 32) >> 4;
+          umma_ss_lo(tmem + C::kDP, v_lo + off, do_lo + off, hi, idST, k > 0);
         }
         umma_commit(&sh.dp_full);
-        return true;
-      };
-      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
-        int bhkv, j;
-        kv_item(p, t, bhkv, j);
-        ok = mbar_wait(&sh.kv_full, it & 1);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
+      int bhkv, j;
+      kv_item(p, t, bhkv, j);
+      ok = wait(&sh.kv_full, it & 1);
+      if (!ok) break;
+      const int n_steps = p.G * (p.nt - kv_first_q(p, j));
+      ok = issue_st(gs) && issue_dp(gs);
+      for (int u = 0; u < n_steps && ok; ++u, ++gs) {
+        const int st = gs & 1;
+        // dV += P^T dO  (A = P^T in TMEM, K = queries; B = dO MN-major)
+        ok = wait(&sh.p_ready, gs & 1);
+        if (ok && u == 0 && it >= 1) ok = wait(&sh.acc_free, (it - 1) & 1);
         if (!ok) break;
-        const int n_steps = p.G * (p.nt - kv_first_q(p, j));
-        ok = issue_st(gs) && issue_dp(gs);
-        for (int u = 0; u < n_steps && ok; ++u, ++gs) {
-          const int st = gs & 1;
-          const uint32_t q_addr = smem_u32(sQ + st * C::kTile), do_addr = smem_u32(sDO + st * C::kTile);
-          // dV += P^T dO  (A = P^T in TMEM, K = queries; B = dO MN-major)
-          ok = mbar_wait(&sh.p_ready, gs & 1);
-          if (ok && u == 0 && it >= 1) ok = mbar_wait(&sh.acc_free, (it - 1) & 1);
-          if (!ok) break;
-          tc_fence_after();
+        tc_fence_after();
+        if (leader) {
+          const uint32_t do_mn = do_mn0 + st * (C::kTile >> 4);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + C::kDV, tmem + C::kS + (k >> 2) * 64 + (k & 3) * 8,
-                    sdesc_sw128(do_addr + k * 2048, C::kBox, 1024), idKV, !(u == 0 && k == 0));
+            umma_ts_lo(tmem + C::kDV, tmem + C::kS + (k >> 2) * 64 + (k & 3) * 8, do_mn + ((k * 2048) >> 4), hi,
+                       idKV, !(u == 0 && k == 0));
           umma_commit(&sh.v_done);
-          if (u + 1 < n_steps && !issue_st(gs + 1)) { ok = false; break; }
-          // dK += dS^T Q  (A = dS^T in TMEM; B = Q MN-major)
-          ok = mbar_wait(&sh.ds_ready, gs & 1);
-          if (!ok) break;
-          tc_fence_after();
+        }
+        __syncwarp();
+        if (u + 1 < n_steps && !issue_st(gs + 1)) { ok = false; break; }
+        // dK += dS^T Q  (A = dS^T in TMEM; B = Q MN-major)
+        ok = wait(&sh.ds_ready, gs & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (leader) {
+          const uint32_t q_mn = q_mn0 + st * (C::kTile >> 4);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + C::kDK, tmem + C::kDP + (k >> 2) * 64 + (k & 3) * 8,
-                    sdesc_sw128(q_addr + k * 2048, C::kBox, 1024), idKV, !(u == 0 && k == 0));
+            umma_ts_lo(tmem + C::kDK, tmem + C::kDP + (k >> 2) * 64 + (k & 3) * 8, q_mn + ((k * 2048) >> 4), hi,
+                       idKV, !(u == 0 && k == 0));
           umma_commit(&sh.k_done);
           umma_commit(&sh.qdo_empty[st]);
-          if (u + 1 < n_steps && !issue_dp(gs + 1)) { ok = false; break; }
         }
-        if (!ok) break;
-        umma_commit(&sh.kv_empty);
+        __syncwarp();
+        if (u + 1 < n_steps && !issue_dp(gs + 1)) { ok = false; break; }
       }
+      if (!ok) break;
+      if (leader) umma_commit(&sh.kv_empty);
+      __syncwarp();
+    }
+    if (leader) {
       umma_commit(&sh.drain);
       mbar_wait(&sh.drain, 0);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ dS warpgroups (rows = keys)
     // warps 0-3: queries 0-63 of every step and the dV epilogue; warps 4-7: queries
@@ -617,79 +638,92 @@ __global__ void __launch_bounds__(352, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     // Order per step j:  S(j+1)  [dS(j)] dQ(j)  dP(j+1).  The warpgroups' exps of step
-    // j+1 run under dQ(j) and dP(j+1); dS of step j needs dP(j).
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);   // S, dP
-      constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);      // dQ += dS K
-      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
-      int gj = 0, it = 0;
-      bool ok = true;
-      auto issue_s = [&](int g) -> bool {     // S(g) = Q K(g)^T into buffer g % 2
-        const int st = g % C::KVST, sb = g & 1;
-        if (!mbar_wait(&sh.k_full[st], (g / C::KVST) & 1)) return false;
-        if (g >= 2 && !mbar_wait(&sh.q_done[sb], ((g >> 1) - 1) & 1)) return false;   // dS(g-2) consumed
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + st * C::kTile);
+    // j+1 run under dQ(j) and dP(j+1); dS of step j needs dP(j).  The whole warp
+    // follows the schedule; one lane, elected once, issues every MMA and commit.
+    const bool leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);   // S, dP
+    constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);      // dQ += dS K
+    constexpr uint32_t hi = sdesc_hi_sw128(1024);
+    const uint32_t q_lo = sdesc_lo(smem_u32(sQ), 16), do_lo = sdesc_lo(smem_u32(sDO), 16);
+    const uint32_t k_lo0 = sdesc_lo(smem_u32(sK), 16), v_lo0 = sdesc_lo(smem_u32(sV), 16);
+    const uint32_t k_mn0 = sdesc_lo(smem_u32(sK), C::kBox);
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    };
+    int gj = 0, it = 0;
+    bool ok = true;
+    auto issue_s = [&](int g) -> bool {     // S(g) = Q K(g)^T into buffer g % 2
+      const int st = g % C::KVST, sb = g & 1;
+      if (!wait(&sh.k_full[st], (g / C::KVST) & 1)) return false;
+      if (g >= 2 && !wait(&sh.q_done[sb], ((g >> 1) - 1) & 1)) return false;   // dS(g-2) consumed
+      tc_fence_after();
+      if (leader) {
+        const uint32_t k_lo = k_lo0 + st * (C::kTile >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-          umma_ss(tmem + (sb ? C::kS1 : C::kS0), sdesc_sw128(q_addr + off, 16, 1024),
-                  sdesc_sw128(k_addr + off, 16, 1024), idS, k > 0);
+          const uint32_t off = ((k >> 2) * C::kBox + (k & 3) * 32) >> 4;
+          umma_ss_lo(tmem + (sb ? C::kS1 : C::kS0), q_lo + off, k_lo + off, hi, idS, k > 0);
         }
         umma_commit(&sh.s_full[sb]);
-        return true;
-      };
-      auto issue_dp = [&](int g) -> bool {    // dP(g) = dO V(g)^T
-        const int st = g % C::KVST;
-        if (!mbar_wait(&sh.v_full[st], (g / C::KVST) & 1)) return false;
-        if (g >= 1 && !mbar_wait(&sh.dp_free, (g - 1) & 1)) return false;       // dP(g-1) read
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sV + st * C::kTile);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_dp = [&](int g) -> bool {    // dP(g) = dO V(g)^T
+      const int st = g % C::KVST;
+      if (!wait(&sh.v_full[st], (g / C::KVST) & 1)) return false;
+      if (g >= 1 && !wait(&sh.dp_free, (g - 1) & 1)) return false;       // dP(g-1) read
+      tc_fence_after();
+      if (leader) {
+        const uint32_t v_lo = v_lo0 + st * (C::kTile >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-          umma_ss(tmem + C::kDP, sdesc_sw128(do_addr + off, 16, 1024), sdesc_sw128(v_addr + off, 16, 1024),
-                  idS, k > 0);
+          const uint32_t off = ((k >> 2) * C::kBox + (k & 3) * 32) >> 4;
+          umma_ss_lo(tmem + C::kDP, do_lo + off, v_lo + off, hi, idS, k > 0);
         }
         umma_commit(&sh.dp_full);
         umma_commit(&sh.v_empty[st]);
-        return true;
-      };
-      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
-        int bhq, i;
-        q_item(p, t, bhq, i);
-        const int n_kv = q_n_kv(p, i);
-        ok = mbar_wait(&sh.qdo_full, it & 1);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
+      int bhq, i;
+      q_item(p, t, bhq, i);
+      const int n_kv = q_n_kv(p, i);
+      ok = wait(&sh.qdo_full, it & 1);
+      if (!ok) break;
+      ok = issue_s(gj) && issue_dp(gj);
+      for (int u = 0; u < n_kv && ok; ++u) {
+        const int g = gj + u, st = g % C::KVST, sb = g & 1;
+        if (u + 1 < n_kv && !issue_s(g + 1)) { ok = false; break; }
+        // dQ += dS K  (A = dS in TMEM, M = queries, K = keys; B = K MN-major)
+        ok = wait(&sh.ds_ready, g & 1);
+        if (ok && u == 0 && it >= 1) ok = wait(&sh.acc_free, (it - 1) & 1);
         if (!ok) break;
-        ok = issue_s(gj) && issue_dp(gj);
-        for (int u = 0; u < n_kv && ok; ++u) {
-          const int g = gj + u, st = g % C::KVST, sb = g & 1;
-          if (u + 1 < n_kv && !issue_s(g + 1)) { ok = false; break; }
-          // dQ += dS K  (A = dS in TMEM, M = queries, K = keys; B = K MN-major)
-          ok = mbar_wait(&sh.ds_ready, g & 1);
-          if (ok && u == 0 && it >= 1) ok = mbar_wait(&sh.acc_free, (it - 1) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sK + st * C::kTile);
+        tc_fence_after();
+        if (leader) {
+          const uint32_t k_mn = k_mn0 + st * (C::kTile >> 4);
           const uint32_t sbase = tmem + (sb ? C::kS1 : C::kS0);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + C::kDQ, sbase + (k >> 2) * 64 + (k & 3) * 8, sdesc_sw128(k_addr + k * 2048, C::kBox, 1024),
-                    idQ, !(u == 0 && k == 0));
+            umma_ts_lo(tmem + C::kDQ, sbase + (k >> 2) * 64 + (k & 3) * 8, k_mn + ((k * 2048) >> 4), hi, idQ,
+                       !(u == 0 && k == 0));
           umma_commit(&sh.q_done[sb]);
           umma_commit(&sh.k_empty[st]);
-          if (u + 1 < n_kv) {
-            if (!issue_dp(g + 1)) { ok = false; break; }
-          } else {
-            umma_commit(&sh.qdo_empty);     // the item's last reads of Q and dO are issued
-          }
+          if (u + 1 == n_kv) umma_commit(&sh.qdo_empty);     // the item's last reads of Q and dO are issued
         }
-        if (!ok) break;
-        gj += n_kv;
+        __syncwarp();
+        if (u + 1 < n_kv && !issue_dp(g + 1)) { ok = false; break; }
       }
+      if (!ok) break;
+      gj += n_kv;
+    }
+    if (leader) {
       umma_commit(&sh.drain);
       mbar_wait(&sh.drain, 0);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ dS warpgroups (rows = queries)
     // warps 0-3: keys 0-63 of every step, warps 4-7: keys 64-127.  The row's LSE and D
