@@ -49,6 +49,12 @@ struct FwdCfg {
   static constexpr int VST = (D == 128) ? 2 : 3;     // V ring stages (<= 3, see FwdShared::pv_done)
   static_assert(VST <= 3, "the V producer's waits on pv_done need VST <= 3");
   static constexpr int kGroups = 4;                  // softmax groups of 4 warps
+  // Of every 8 score pairs, how many are exponentiated on the FMA pipe instead of
+  // MUFU (16 ex2 per SM per clock, so one exp per score costs as much MUFU time as
+  // the d = 128 tile's two MMAs).  Measured on B200 with four softmax warps per
+  // sub-partition: 0 is fastest or within noise of 1-3 at d = 64 and d = 128, so
+  // the issue slots the polynomial takes cost more than the MUFU time it saves.
+  static constexpr int kFmaPairs = 0;
   static constexpr int kThreads = 608;
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = 384;                  // O accumulator column
@@ -434,8 +440,12 @@ __global__ void __launch_bounds__(608, 1)
             const uint64_t x = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
             float x0, x1, a, b;
             f2unpack(x, x0, x1);
-            a = ex2_approx(x0);
-            b = ex2_approx(x1);
+            if (k >= 8 - C::kFmaPairs) {
+              exp2_fma_pair(x0, x1, a, b);
+            } else {
+              a = ex2_approx(x0);
+              b = ex2_approx(x1);
+            }
             lsum = fadd2(lsum, f2pack(a, b));
             pk[k] = pack_bf16x2(a, b);
           }
