@@ -13,11 +13,11 @@
 
 #include "attn.h"
 #include "fwd.cuh"
+#include "fwd_pp.cuh"
 #include "bwd.cuh"
 
 namespace {
 
-using attn::FwdCfg;
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -83,16 +83,18 @@ int check_common(int B, int Hq, int Hkv, int N, int d, float scale, int causal) 
   return ATTN_OK;
 }
 
+
+// Forward: two query tiles per CTA (fwd_pp.cuh).
 template <int D>
-int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                int N, float scale, int causal, cudaStream_t stream, const DeviceInfo& di) {
-  using C = FwdCfg<D>;
+  using C = attn::PpCfg<D>;
   static std::once_flag attr_once[64];
   static bool attr_ok[64];
   int dev = 0;
   cudaGetDevice(&dev);
   std::call_once(attr_once[dev], [&] {
-    attr_ok[dev] = cudaFuncSetAttribute(attn::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_ok[dev] = cudaFuncSetAttribute(attn::attn_fwd_pp_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::kSmem) == cudaSuccess;
   });
   if (!attr_ok[dev]) return ATTN_ERR_LAUNCH;
@@ -113,8 +115,9 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.total_tiles = p.n_qtiles * B * Hq;
   p.c = scale * 1.4426950408889634f;
   p.causal = causal;
-  const int grid = p.total_tiles < di.sms ? p.total_tiles : di.sms;
-  attn::attn_fwd_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  const int units = B * Hkv * ((p.G * p.n_qtiles + 1) / 2);
+  const int grid = units < di.sms ? units : di.sms;
+  attn::attn_fwd_pp_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -228,8 +231,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   DeviceInfo* di = nullptr;
   if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_fwd<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, *di);
-  return launch_fwd<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, *di);
+  if (d == 64) return launch_fwd_pp<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, *di);
+  return launch_fwd_pp<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, *di);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int causal) {

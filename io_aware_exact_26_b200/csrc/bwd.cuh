@@ -231,6 +231,7 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv); tma_prefetch_desc(&tmdo);
+      const uint64_t pol_reuse = l2_policy_evict_last(), pol_once = l2_policy_evict_first();
       int gs = 0, it = 0, nq = 0, nkv = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
@@ -239,22 +240,28 @@ __global__ void __launch_bounds__(320, 1)
         if (it >= 1) ok = mbar_wait(&sh.kv_empty, (it - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&sh.kv_full, 2 * C::kTile);
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(sK + c * C::kBox, &tmk, &sh.kv_full, c * 64, j * 128, bhkv);
-          tma_load_3d(sV + c * C::kBox, &tmv, &sh.kv_full, c * 64, j * 128, bhkv);
+        for (int c = 0; c < D / 64; ++c) {                  // K_j, V_j: read by this item only
+          tma_load_3d_hint(sK + c * C::kBox, &tmk, &sh.kv_full, c * 64, j * 128, bhkv, pol_once);
+          tma_load_3d_hint(sV + c * C::kBox, &tmv, &sh.kv_full, c * 64, j * 128, bhkv, pol_once);
         }
         nkv = it + 1;
         const int b = bhkv / p.Hkv, hk = bhkv - b * p.Hkv;
-        for (int h = 0; h < p.G && ok; ++h) {
-          const int bhq = b * p.Hq + hk * p.G + h;
-          for (int i = kv_first_q(p, j); i < p.nt; ++i, ++gs) {
+        // Query tiles from the last down to the first visible one, the G heads of
+        // the group inside: every item of a head group starts at the same tile, so
+        // the CTAs working on that group read each Q/dO tile at about the same
+        // time and HBM delivers it about once.
+        for (int i = p.nt - 1; i >= kv_first_q(p, j) && ok; --i) {
+          for (int h = 0; h < p.G; ++h, ++gs) {
+            const int bhq = b * p.Hq + hk * p.G + h;
             const int st = gs & 1;
             if (gs >= 2) ok = mbar_wait(&sh.qdo_empty[st], ((gs >> 1) - 1) & 1);
             if (!ok) break;
             mbar_arrive_expect_tx(&sh.qdo_full[st], 2 * C::kTile + 1024);
-            for (int c = 0; c < D / 64; ++c) {
-              tma_load_3d(sQ + st * C::kTile + c * C::kBox, &tmq, &sh.qdo_full[st], c * 64, i * 128, bhq);
-              tma_load_3d(sDO + st * C::kTile + c * C::kBox, &tmdo, &sh.qdo_full[st], c * 64, i * 128, bhq);
+            for (int c = 0; c < D / 64; ++c) {              // Q_i, dO_i: read by every key tile's item
+              tma_load_3d_hint(sQ + st * C::kTile + c * C::kBox, &tmq, &sh.qdo_full[st], c * 64, i * 128, bhq,
+                               pol_reuse);
+              tma_load_3d_hint(sDO + st * C::kTile + c * C::kBox, &tmdo, &sh.qdo_full[st], c * 64, i * 128, bhq,
+                               pol_reuse);
             }
             const size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + i * 128;
             bulk_load(sVec + st * 256, p.lse2 + vrow, 512, &sh.qdo_full[st]);
@@ -383,8 +390,8 @@ __global__ void __launch_bounds__(320, 1)
       kv_item(p, t, bhkv, j);
       const int key = j * 128 + r;
       const bool key_live = key < p.N;
-      for (int h = 0; h < p.G && ok; ++h) {
-        for (int i = kv_first_q(p, j); i < p.nt && ok; ++i, ++gs) {
+      for (int i = p.nt - 1; i >= kv_first_q(p, j) && ok; --i) {
+        for (int h = 0; h < p.G && ok; ++h, ++gs) {
           const int st = gs & 1;
           const float* sLse = sVec + st * 256 + 64 * hb;
           const float* sDd = sLse + 128;

@@ -1,0 +1,464 @@
+// Forward exact attention for sm_100a, two query tiles per CTA ("ping-pong").
+//
+// Method (page "attention 的显存线性化" §三; page "attn-efficient", online-softmax
+// section): per 128-row query tile, stream 128-key tiles of K/V, form S on chip,
+// keep a running row max m and sum l, rescale the partial output when the max
+// grows, write only O and the log-sum-exp.  S and P never reach HBM.
+//
+// B200 mapping.  A work unit is a pair of query tiles A and B that read the same
+// KV head (two heads of a GQA group at one query tile, or two adjacent query
+// tiles of one head); each K/V tile is loaded once for both.  Team A (warps 0-7)
+// owns tile A, team B (warps 8-15) tile B; the MMA warp interleaves the two
+// teams' products, so while one team exponentiates, the tensor cores work on the
+// other team's S or PV, and the two teams' MUFU phases alternate.
+//   warps 0-7, 8-15  softmax teams; inside a team, group k = (warp % 8) / 4 owns
+//                    keys [64k, 64k+64) of each S tile and O columns
+//                    [k*D/2, (k+1)*D/2); thread = query row = TMEM lane.
+//   warp 16          TMA producer: Q_A, Q_B (one buffer each), K and V rings (2
+//                    stages each), loaded as K(0) V(0) K(1) V(1) ..., the order in
+//                    which the MMA warp releases their stages
+//   warp 17          MMA issuer
+// TMEM: S_A at 0, S_B at 128 (P written over S as bf16: keys 0-63 in columns
+// 0-31, keys 64-127 in 64-95), O_A at 256, O_B at 256 + D.
+// Per team the loop is S(j) -> softmax(j) -> PV(j) -> S(j+1): one S buffer per
+// tile, so S(j+1) is issued only after PV(j) has completed (no reliance on the
+// order in which the tensor cores retire MMAs for the aliasing of P and S).
+// Each step a team's two groups exchange partial row maxima of the tile in
+// shared memory; the exp2 with folded scale and the lazy rescale threshold are
+// described in fwd.cuh.
+#pragma once
+#include "fwd.cuh"
+
+namespace attn {
+
+template <int D>
+struct PpCfg {
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kBox = 128 * 128;
+  static constexpr int KST = 2;
+  static constexpr int VST = 2;
+  static constexpr int kThreads = 576;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
+  static constexpr int kOffQ = 0;                       // Q_A, Q_B
+  static constexpr int kOffK = 2 * kTile;
+  static constexpr int kOffV = kOffK + KST * kTile;
+  static constexpr int kOffSh = kOffV + VST * kTile;
+  static constexpr int kLayout = kOffSh + 8192;
+  static constexpr int kSmem = kLayout + 1024;
+  static_assert(kSmem <= 232448, "shared memory layout exceeds 227 KB");
+};
+
+struct PpShared {
+  float xmax[2][2][2][128];   // [team][parity][group][row] partial row maxima of a step
+  float xsum[2][2][128];      // [team][group][row] partial row sums of a unit
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2];         // per team: S of its current step complete
+  uint64_t p_ready[2];        // per team: P written by its 8 warps
+  uint64_t pv_done[2];        // per team: PV of its step complete
+  uint64_t xbar[2][2];        // [team][parity]: both groups posted their maxima
+  uint64_t sbar[2];           // per team: both groups posted their sums
+  uint64_t o_free[2];         // per team: O read out by the epilogue
+  uint64_t drain;
+  uint64_t teardown;
+  uint32_t tmem_base;
+};
+static_assert(sizeof(PpShared) <= 8192, "PpShared does not fit its slot");
+
+struct PpUnit {
+  int bh0, qt0, n0;           // tile A
+  int bh1, qt1, n1;           // tile B (n1 = 0: no tile B)
+  int bkv;
+  __device__ __forceinline__ int n(int x) const { return x ? n1 : n0; }
+  __device__ __forceinline__ int qt(int x) const { return x ? qt1 : qt0; }
+  __device__ __forceinline__ int bh(int x) const { return x ? bh1 : bh0; }
+};
+
+// Unit u -> two query tiles of one KV head.  The tiles of a KV head group are
+// listed query-tile-major, longest first under causal masking, the G heads
+// inside; consecutive list entries are paired, so under causal masking tile A
+// sees as many key tiles as tile B or one more.
+__device__ __forceinline__ PpUnit pp_unit(const FwdParams& p, int u) {
+  const int per_group = p.G * p.n_qtiles;
+  const int upg = (per_group + 1) >> 1;
+  const int gk = u / upg;
+  const int m = u - gk * upg;
+  PpUnit r;
+  r.bkv = gk;
+  auto tile = [&](int l, int& bh, int& qt, int& n) {
+    if (l < per_group) {
+      const int rq = l / p.G;
+      const int h = l - rq * p.G;
+      qt = p.causal ? (p.n_qtiles - 1 - rq) : rq;
+      bh = (gk / p.Hkv) * p.Hq + (gk % p.Hkv) * p.G + h;
+      n = fwd_n_kv(p, qt);
+    } else {
+      bh = 0; qt = 0; n = 0;
+    }
+  };
+  tile(2 * m, r.bh0, r.qt0, r.n0);
+  tile(2 * m + 1, r.bh1, r.qt1, r.n1);
+  return r;
+}
+
+__device__ __forceinline__ int pp_units(const FwdParams& p) {
+  return p.B * p.Hkv * ((p.G * p.n_qtiles + 1) >> 1);
+}
+
+template <int D>
+__global__ void __launch_bounds__(576, 1)
+    attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
+  using C = PpCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  PpShared& sh = *reinterpret_cast<PpShared*>(smem + C::kOffSh);
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_units = pp_units(p);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.q_full[i], 1);
+      mbar_init(&sh.q_empty[i], 1);
+      mbar_init(&sh.k_full[i], 1);
+      mbar_init(&sh.k_empty[i], 1);
+      mbar_init(&sh.v_full[i], 1);
+      mbar_init(&sh.v_empty[i], 1);
+      mbar_init(&sh.s_full[i], 1);
+      mbar_init(&sh.p_ready[i], 8);
+      mbar_init(&sh.pv_done[i], 1);
+      mbar_init(&sh.xbar[i][0], 8);
+      mbar_init(&sh.xbar[i][1], 8);
+      mbar_init(&sh.sbar[i], 8);
+      mbar_init(&sh.o_free[i], 8);
+    }
+    mbar_init(&sh.drain, 1);
+    mbar_init(&sh.teardown, 18);
+    fence_barrier_init();
+  }
+  if (warp == 0) { tmem_alloc(&sh.tmem_base, C::kTmemCols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 16) {
+    // ------------------------------------------------------------ TMA producer: Q_A, Q_B, K, V
+    if (lane == 0) {
+      tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv);
+      int kc = 0, uq0 = 0, uq1 = 0;
+      int nk = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const PpUnit w = pp_unit(p, u);
+        auto load_q = [&](int x, int uq) -> bool {     // Q of team x, its uq-th unit
+          if (uq >= 1 && !mbar_wait(&sh.q_empty[x], (uq - 1) & 1)) return false;
+          mbar_arrive_expect_tx(&sh.q_full[x], C::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sQ + x * C::kTile + c * C::kBox, &tmq, &sh.q_full[x], c * 64, w.qt(x) * 128, w.bh(x));
+          return true;
+        };
+        ok = load_q(0, uq0++);
+        if (ok && w.n1 > 0) ok = load_q(1, uq1++);
+        for (int j = 0; j < w.n0 && ok; ++j, ++kc) {
+          const int st = kc & 1;
+          if (kc >= 2) ok = mbar_wait(&sh.k_empty[st], ((kc >> 1) - 1) & 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, j * 128, w.bkv);
+          if (kc >= 2) ok = mbar_wait(&sh.v_empty[st], ((kc >> 1) - 1) & 1);
+          if (!ok) { nk = kc + 1; break; }
+          mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sV + st * C::kTile + c * C::kBox, &tmv, &sh.v_full[st], c * 64, j * 128, w.bkv);
+          nk = kc + 1;
+        }
+      }
+      if (!ok)
+        for (int g = max(0, nk - 2); g < nk; ++g) {
+          mbar_drain_wait(&sh.k_full[g & 1], (g >> 1) & 1);
+          mbar_drain_wait(&sh.v_full[g & 1], (g >> 1) & 1);
+        }
+    }
+  } else if (warp == 17) {
+    // ------------------------------------------------------------ MMA issuer
+    // Per step j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_X(j+1) waits for PV_X(j)
+    // (the P it overwrites); meanwhile the tensor cores run the other team's work.
+    const bool leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
+    constexpr uint32_t hi = sdesc_hi_sw128(1024);
+    const uint32_t q_lo0 = sdesc_lo(smem_u32(sQ), 16);
+    const uint32_t k_lo0 = sdesc_lo(smem_u32(sK), 16);
+    const uint32_t v_lo0 = sdesc_lo(smem_u32(sV), C::kBox);
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    };
+    int kc = 0, vc = 0;
+    int gs0 = 0, gs1 = 0;        // steps issued per team
+    int uu0 = 0, uu1 = 0;        // units per team
+    bool ok = true;
+    // S_X = Q_X K^T for team x from K stage st
+    auto issue_s = [&](int x, int st, bool last) {
+      if (leader) {
+        const uint32_t q_lo = q_lo0 + x * (C::kTile >> 4);
+        const uint32_t k_lo = k_lo0 + st * (C::kTile >> 4);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = ((k >> 2) * C::kBox + (k & 3) * 32) >> 4;
+          umma_ss_lo(tmem + (x ? C::kS1 : C::kS0), q_lo + off, k_lo + off, hi, idS, k > 0);
+        }
+        umma_commit(&sh.s_full[x]);
+        if (last) umma_commit(&sh.q_empty[x]);
+      }
+      __syncwarp();
+    };
+    // O_X (+)= P_X V for team x from V stage st
+    auto issue_pv = [&](int x, int st, bool first) {
+      if (leader) {
+        const uint32_t v_lo = v_lo0 + st * (C::kTile >> 4);
+        const uint32_t sbase = tmem + (x ? C::kS1 : C::kS0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ts_lo(tmem + (x ? C::kO1 : C::kO0), sbase + (k >> 2) * 64 + (k & 3) * 8, v_lo + ((k * 2048) >> 4), hi,
+                     idO, !(first && k == 0));
+        umma_commit(&sh.pv_done[x]);
+      }
+      __syncwarp();
+    };
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const PpUnit w = pp_unit(p, u);
+      // first S of each team
+      {
+        const int st = kc & 1;
+        ok = wait(&sh.k_full[st], (kc >> 1) & 1);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int gsx = x ? gs1 : gs0, uux = x ? uu1 : uu0;
+          if (!ok || w.n(x) == 0) continue;
+          ok = wait(&sh.q_full[x], uux & 1);
+          if (ok && gsx >= 1) ok = wait(&sh.pv_done[x], (gsx - 1) & 1);   // previous unit's last PV
+          if (!ok) continue;
+          tc_fence_after();
+          issue_s(x, st, w.n(x) == 1);
+        }
+        if (!ok) break;
+        if (leader) umma_commit(&sh.k_empty[st]);
+        __syncwarp();
+        ++kc;
+      }
+      for (int j = 0; j < w.n0 && ok; ++j, ++vc) {
+        const int vst = vc & 1;
+        ok = wait(&sh.v_full[vst], (vc >> 1) & 1);
+        const bool next_k = j + 1 < w.n0;
+        bool k_ready = false;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int gsx = x ? gs1 : gs0, uux = x ? uu1 : uu0, nx = w.n(x);
+          if (!ok || j >= nx) continue;
+          const int g = gsx + j;
+          ok = wait(&sh.p_ready[x], g & 1);
+          if (ok && j == 0 && uux >= 1) ok = wait(&sh.o_free[x], (uux - 1) & 1);
+          if (!ok) continue;
+          tc_fence_after();
+          issue_pv(x, vst, j == 0);
+          if (j + 1 < nx) {
+            if (!k_ready) {
+              ok = wait(&sh.k_full[kc & 1], (kc >> 1) & 1);
+              k_ready = true;
+            }
+            if (ok) ok = wait(&sh.pv_done[x], g & 1);     // P_X(j) read: the S buffer may be overwritten
+            if (!ok) continue;
+            tc_fence_after();
+            issue_s(x, kc & 1, j + 2 == nx);
+          }
+        }
+        if (!ok) break;
+        if (leader) {
+          umma_commit(&sh.v_empty[vst]);
+          if (next_k) umma_commit(&sh.k_empty[kc & 1]);
+        }
+        __syncwarp();
+        if (next_k) ++kc;
+      }
+      gs0 += w.n0; ++uu0;
+      if (w.n1 > 0) { gs1 += w.n1; ++uu1; }
+    }
+    if (leader) {
+      umma_commit(&sh.drain);
+      mbar_wait(&sh.drain, 0);
+    }
+    __syncwarp();
+  } else if (warp < 16) {
+    // ------------------------------------------------------------ softmax teams
+    const int x = warp >> 3;                                    // team
+    const int grp = (warp >> 2) & 1;                            // keys [64 grp, 64 grp + 64)
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t s_base = lane_base + (x ? C::kS1 : C::kS0) + grp * 64;
+    constexpr int OH = D / 2;
+    const uint32_t o_base = lane_base + (x ? C::kO1 : C::kO0) + grp * OH;
+    const float c = p.c;
+    const uint64_t c2 = f2pack(c, c);
+    int gs = 0, uu = 0;
+    bool ok = true;
+    auto mask16 = [&](uint32_t (&r)[16], int col0, int lim) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        if (col0 + k > lim) r[k] = 0xff800000u;
+    };
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const PpUnit w = pp_unit(p, u);
+      const int n = w.n(x);
+      if (n == 0) continue;
+      const int qrow = w.qt(x) * 128 + row;
+      const int bh = w.bh(x);
+      float m_used = -INFINITY;
+      uint64_t lsum = f2pack(0.f, 0.f);
+      for (int j = 0; j < n && ok; ++j) {
+        const int g = gs + j, xp = g & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[x], g & 1));
+        if (!ok) break;
+        tc_fence_after();
+        const int kbase = j * 128 + grp * 64;
+        const int lim = p.causal ? min(p.N - 1, qrow) - kbase : p.N - 1 - kbase;   // last visible column
+        const bool msk = __any_sync(0xffffffffu, lim < 63);
+        // pass 1: this group's partial row max of the 64 columns
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t r0[16], r1[16];
+          tmem_ld16(s_base + hh * 32, r0);
+          tmem_ld16(s_base + hh * 32 + 16, r1);
+          tmem_wait_ld();
+          reg_fence(r0);
+          reg_fence(r1);
+          if (msk) { mask16(r0, hh * 32, lim); mask16(r1, hh * 32 + 16, lim); }
+#pragma unroll
+          for (int k = 0; k < 16; k += 8) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              mx4[e] = max3f(mx4[e], __uint_as_float(r0[k + e]), __uint_as_float(r0[k + e + 4]));
+              mx4[e] = max3f(mx4[e], __uint_as_float(r1[k + e]), __uint_as_float(r1[k + e + 4]));
+            }
+          }
+        }
+        sh.xmax[x][xp][grp][row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.xbar[x][xp]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&sh.xbar[x][xp], (g >> 1) & 1));
+        if (!ok) break;
+        const float m_tile = fmaxf(sh.xmax[x][xp][0][row], sh.xmax[x][xp][1][row]) * c;
+        float alpha = 1.f;
+        const bool need = (m_used == -INFINITY) || (m_tile > m_used + kRescaleTau);
+        if (need) {
+          const float m_new = fmaxf(m_used, m_tile);
+          alpha = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
+          float l0, l1;
+          f2unpack(lsum, l0, l1);
+          lsum = f2pack(l0 * alpha, l1 * alpha);
+          m_used = m_new;
+        }
+        // Rescale this group's O columns if the max moved.  S_X(j) was issued only
+        // after PV_X(j-1) completed, so O already holds every step before j; the
+        // wait below is then immediate.
+        if (__any_sync(0xffffffffu, need && j > 0)) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[x], (g - 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int q4 = 0; q4 < OH / 16; ++q4) {
+            uint32_t o[16];
+            tmem_ld16(o_base + q4 * 16, o);
+            tmem_wait_ld();
+            reg_fence(o);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st16(o_base + q4 * 16, o);
+          }
+        }
+        // pass 2: exponentiate, P (bf16) over the columns already read
+        const uint64_t nm2 = f2pack(-m_used, -m_used);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t r[16];
+          tmem_ld16(s_base + cc * 16, r);
+          tmem_wait_ld();
+          reg_fence(r);
+          if (msk) mask16(r, cc * 16, lim);
+          uint32_t pk[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t xx = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
+            float x0, x1;
+            f2unpack(xx, x0, x1);
+            const float a = ex2_approx(x0), b = ex2_approx(x1);
+            lsum = fadd2(lsum, f2pack(a, b));
+            pk[k] = pack_bf16x2(a, b);
+          }
+          tmem_st8(s_base + cc * 8, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.p_ready[x]);
+      }
+      if (!ok) break;
+      // epilogue: combine the two groups' sums, wait for the last PV, O / l, LSE
+      const int glast = gs + n - 1;
+      float l0, l1;
+      f2unpack(lsum, l0, l1);
+      sh.xsum[x][grp][row] = l0 + l1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.sbar[x]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sh.sbar[x], uu & 1));
+      if (!ok) break;
+      const float l = sh.xsum[x][0][row] + sh.xsum[x][1][row];
+      ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[x], glast & 1));
+      if (!ok) break;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool live = qrow < p.N;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D + grp * OH;
+#pragma unroll 1
+      for (int q4 = 0; q4 < OH / 16; ++q4) {
+        uint32_t o[16];
+        tmem_ld16(o_base + q4 * 16, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        uint32_t pk[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          pk[k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 16);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+      if (live && grp == 0) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.o_free[x]);
+      gs += n;
+      ++uu;
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sh.teardown);
+  if (warp == 0) {
+    mbar_wait(&sh.teardown, 0);
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace attn
