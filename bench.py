@@ -350,7 +350,7 @@ def main():
             "roofline": roofline,
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
-            "gpu_launches": args.steps * (4 if has_bwd else 1),   # fwd; bwd = prep + dK/dV + dQ
+            "gpu_launches": args.steps * (5 if has_bwd else 2),   # fwd = counter reset + kernel; bwd = prep + dK/dV + dQ
             "clocks": clocks}
     if has_bwd:
         line["bwd"] = {"ms": round(bwd_avg, 4), "tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 1),

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -84,6 +85,13 @@ int check_common(int B, int Hq, int Hkv, int N, int d, float scale, int causal) 
 }
 
 
+// Work-unit counter slot for the next dynamically scheduled launch (rotates over
+// attn::kSchedSlots; concurrent launches in flight take different slots).
+int next_sched_slot() {
+  static std::atomic<unsigned> n{0};
+  return static_cast<int>(n.fetch_add(1, std::memory_order_relaxed) % attn::kSchedSlots);
+}
+
 // Forward: two query tiles per CTA (fwd_pp.cuh).
 template <int D>
 int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -117,6 +125,8 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   p.causal = causal;
   const int units = B * Hkv * ((p.G * p.n_qtiles + 1) / 2);
   const int grid = units < di.sms ? units : di.sms;
+  p.sched_slot = next_sched_slot();
+  attn::sched_reset_kernel<<<1, 32, 0, stream>>>(p.sched_slot);
   attn::attn_fwd_pp_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }

@@ -23,6 +23,7 @@ struct FwdParams {
   int n_qtiles, total_tiles;
   float c;          // scale * log2(e)
   int causal;
+  int sched_slot;   // g_sched slot this launch claims work units from
 };
 
 // Key tiles a query tile sees: all of them, or (causal) those up to its diagonal.

@@ -5,6 +5,11 @@
 // keep a running row max m and sum l, rescale the partial output when the max
 // grows, write only O and the log-sum-exp.  S and P never reach HBM.
 //
+// Scheduling: CTAs claim work units from a global counter (g_sched) in the
+// order pp_unit numbers them, so a CTA that drew short causal units takes more;
+// the producer warp claims and passes each unit index to the other warps through
+// a small ring in shared memory.
+//
 // B200 mapping.  A work unit is a pair of query tiles A and B that read the same
 // KV head (two heads of a GQA group at one query tile, or two adjacent query
 // tiles of one head); each K/V tile is loaded once for both.  Team A (warps 0-7)
@@ -38,6 +43,9 @@ struct PpCfg {
   static constexpr int KST = 2;
   static constexpr int VST = 2;
   static constexpr int kThreads = 576;
+  // Of every 8 score pairs, how many are exponentiated on the FMA pipe instead of
+  // MUFU (16 ex2 per SM per clock).
+  static constexpr int kFmaPairs = 0;
   static constexpr int kTmemCols = 512;
   static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
   static constexpr int kOffQ = 0;                       // Q_A, Q_B
@@ -60,11 +68,25 @@ struct PpShared {
   uint64_t xbar[2][2];        // [team][parity]: both groups posted their maxima
   uint64_t sbar[2];           // per team: both groups posted their sums
   uint64_t o_free[2];         // per team: O read out by the epilogue
+  uint64_t unit_full[4];      // unit index posted by the producer
+  uint64_t unit_empty[4];     // unit index read by the MMA warp and the 16 softmax warps
+  int unit_ring[4];
   uint64_t drain;
   uint64_t teardown;
   uint32_t tmem_base;
 };
 static_assert(sizeof(PpShared) <= 8192, "PpShared does not fit its slot");
+
+// The k-th unit this CTA processes (-1: none left), as posted by the producer.
+__device__ __forceinline__ int pp_next_unit(PpShared& sh, int k, int lane, bool& ok) {
+  const int slot = k & 3;
+  ok = __all_sync(0xffffffffu, mbar_wait(&sh.unit_full[slot], (k >> 2) & 1));
+  if (!ok) return -1;
+  const int u = *reinterpret_cast<volatile int*>(&sh.unit_ring[slot]);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sh.unit_empty[slot]);
+  return u;
+}
 
 struct PpUnit {
   int bh0, qt0, n0;           // tile A
@@ -136,6 +158,10 @@ __global__ void __launch_bounds__(576, 1)
       mbar_init(&sh.sbar[i], 8);
       mbar_init(&sh.o_free[i], 8);
     }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&sh.unit_full[i], 1);
+      mbar_init(&sh.unit_empty[i], 17);
+    }
     mbar_init(&sh.drain, 1);
     mbar_init(&sh.teardown, 18);
     fence_barrier_init();
@@ -153,7 +179,15 @@ __global__ void __launch_bounds__(576, 1)
       int kc = 0, uq0 = 0, uq1 = 0;
       int nk = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      for (int k = 0; ok; ++k) {
+        const int slot = k & 3;
+        if (k >= 4) ok = mbar_wait(&sh.unit_empty[slot], ((k >> 2) - 1) & 1);
+        if (!ok) break;
+        int u = static_cast<int>(atomicAdd(&g_sched[p.sched_slot], 1u));
+        if (u >= n_units) u = -1;
+        sh.unit_ring[slot] = u;
+        mbar_arrive(&sh.unit_full[slot]);                  // release: the index is visible first
+        if (u < 0) break;
         const PpUnit w = pp_unit(p, u);
         auto load_q = [&](int x, int uq) -> bool {     // Q of team x, its uq-th unit
           if (uq >= 1 && !mbar_wait(&sh.q_empty[x], (uq - 1) & 1)) return false;
@@ -231,7 +265,9 @@ __global__ void __launch_bounds__(576, 1)
       }
       __syncwarp();
     };
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+      const int u = pp_next_unit(sh, k, lane, ok);
+      if (u < 0) break;
       const PpUnit w = pp_unit(p, u);
       // first S of each team
       {
@@ -313,7 +349,9 @@ __global__ void __launch_bounds__(576, 1)
       for (int k = 0; k < 16; ++k)
         if (col0 + k > lim) r[k] = 0xff800000u;
     };
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+      const int u = pp_next_unit(sh, k, lane, ok);
+      if (u < 0) break;
       const PpUnit w = pp_unit(p, u);
       const int n = w.n(x);
       if (n == 0) continue;
@@ -398,7 +436,13 @@ __global__ void __launch_bounds__(576, 1)
             const uint64_t xx = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
             float x0, x1;
             f2unpack(xx, x0, x1);
-            const float a = ex2_approx(x0), b = ex2_approx(x1);
+            float a, b;
+            if (k >= 8 - C::kFmaPairs) {
+              exp2_fma_pair(x0, x1, a, b);
+            } else {
+              a = ex2_approx(x0);
+              b = ex2_approx(x1);
+            }
             lsum = fadd2(lsum, f2pack(a, b));
             pk[k] = pack_bf16x2(a, b);
           }

@@ -17,6 +17,17 @@ namespace attn {
 //        3 = shared memory could not be aligned for the swizzled tiles.
 __device__ int g_attn_status = 0;
 
+// Work-unit counters for dynamically scheduled kernels: each launch takes one
+// slot (rotated by the host), zeroed by sched_reset_kernel on the same stream
+// just before the launch, so launches in flight on different streams never share
+// a counter and a launch that ended early cannot leave a stale count behind.
+constexpr int kSchedSlots = 128;
+__device__ unsigned int g_sched[kSchedSlots];
+
+__global__ void sched_reset_kernel(int slot) {
+  if (threadIdx.x == 0) g_sched[slot] = 0u;
+}
+
 __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
