@@ -68,25 +68,13 @@ struct PpShared {
   uint64_t xbar[2][2];        // [team][parity]: both groups posted their maxima
   uint64_t sbar[2];           // per team: both groups posted their sums
   uint64_t o_free[2];         // per team: O read out by the epilogue
-  uint64_t unit_full[4];      // unit index posted by the producer
-  uint64_t unit_empty[4];     // unit index read by the MMA warp and the 16 softmax warps
-  int unit_ring[4];
+  UnitRing ring;              // unit indices for the MMA warp and the 16 softmax warps
   uint64_t drain;
   uint64_t teardown;
   uint32_t tmem_base;
 };
 static_assert(sizeof(PpShared) <= 8192, "PpShared does not fit its slot");
 
-// The k-th unit this CTA processes (-1: none left), as posted by the producer.
-__device__ __forceinline__ int pp_next_unit(PpShared& sh, int k, int lane, bool& ok) {
-  const int slot = k & 3;
-  ok = __all_sync(0xffffffffu, mbar_wait(&sh.unit_full[slot], (k >> 2) & 1));
-  if (!ok) return -1;
-  const int u = *reinterpret_cast<volatile int*>(&sh.unit_ring[slot]);
-  __syncwarp();
-  if (lane == 0) mbar_arrive(&sh.unit_empty[slot]);
-  return u;
-}
 
 struct PpUnit {
   int bh0, qt0, n0;           // tile A
@@ -158,10 +146,7 @@ __global__ void __launch_bounds__(576, 1)
       mbar_init(&sh.sbar[i], 8);
       mbar_init(&sh.o_free[i], 8);
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&sh.unit_full[i], 1);
-      mbar_init(&sh.unit_empty[i], 17);
-    }
+    unit_ring_init(sh.ring, 17);
     mbar_init(&sh.drain, 1);
     mbar_init(&sh.teardown, 18);
     fence_barrier_init();
@@ -179,14 +164,11 @@ __global__ void __launch_bounds__(576, 1)
       int kc = 0, uq0 = 0, uq1 = 0;
       int nk = 0;
       bool ok = true;
+      // A unit is claimed only when the producer is ready to load it: claiming
+      // ahead leaves units reserved by busy CTAs at the tail (measured slower).
+      int u = 0;
       for (int k = 0; ok; ++k) {
-        const int slot = k & 3;
-        if (k >= 4) ok = mbar_wait(&sh.unit_empty[slot], ((k >> 2) - 1) & 1);
-        if (!ok) break;
-        int u = static_cast<int>(atomicAdd(&g_sched[p.sched_slot], 1u));
-        if (u >= n_units) u = -1;
-        sh.unit_ring[slot] = u;
-        mbar_arrive(&sh.unit_full[slot]);                  // release: the index is visible first
+        u = unit_ring_claim(sh.ring, k, p.sched_slot, n_units);
         if (u < 0) break;
         const PpUnit w = pp_unit(p, u);
         auto load_q = [&](int x, int uq) -> bool {     // Q of team x, its uq-th unit
@@ -213,6 +195,7 @@ __global__ void __launch_bounds__(576, 1)
           nk = kc + 1;
         }
       }
+      if (u == -2) ok = false;
       if (!ok)
         for (int g = max(0, nk - 2); g < nk; ++g) {
           mbar_drain_wait(&sh.k_full[g & 1], (g >> 1) & 1);
@@ -266,7 +249,7 @@ __global__ void __launch_bounds__(576, 1)
       __syncwarp();
     };
     for (int k = 0; ok; ++k) {
-      const int u = pp_next_unit(sh, k, lane, ok);
+      const int u = unit_ring_take(sh.ring, k, lane, ok);
       if (u < 0) break;
       const PpUnit w = pp_unit(p, u);
       // first S of each team
@@ -350,7 +333,7 @@ __global__ void __launch_bounds__(576, 1)
         if (col0 + k > lim) r[k] = 0xff800000u;
     };
     for (int k = 0; ok; ++k) {
-      const int u = pp_next_unit(sh, k, lane, ok);
+      const int u = unit_ring_take(sh.ring, k, lane, ok);
       if (u < 0) break;
       const PpUnit w = pp_unit(p, u);
       const int n = w.n(x);
@@ -369,21 +352,26 @@ __global__ void __launch_bounds__(576, 1)
         const bool msk = __any_sync(0xffffffffu, lim < 63);
         // pass 1: this group's partial row max of the 64 columns
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t r0[16], r1[16];
-          tmem_ld16(s_base + hh * 32, r0);
-          tmem_ld16(s_base + hh * 32 + 16, r1);
+        {
+          uint32_t r0[16], r1[16], r2[16], r3[16];
+          tmem_ld16(s_base, r0);
+          tmem_ld16(s_base + 16, r1);
+          tmem_ld16(s_base + 32, r2);
+          tmem_ld16(s_base + 48, r3);
           tmem_wait_ld();
           reg_fence(r0);
           reg_fence(r1);
-          if (msk) { mask16(r0, hh * 32, lim); mask16(r1, hh * 32 + 16, lim); }
+          reg_fence(r2);
+          reg_fence(r3);
+          if (msk) { mask16(r0, 0, lim); mask16(r1, 16, lim); mask16(r2, 32, lim); mask16(r3, 48, lim); }
 #pragma unroll
           for (int k = 0; k < 16; k += 8) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               mx4[e] = max3f(mx4[e], __uint_as_float(r0[k + e]), __uint_as_float(r0[k + e + 4]));
               mx4[e] = max3f(mx4[e], __uint_as_float(r1[k + e]), __uint_as_float(r1[k + e + 4]));
+              mx4[e] = max3f(mx4[e], __uint_as_float(r2[k + e]), __uint_as_float(r2[k + e + 4]));
+              mx4[e] = max3f(mx4[e], __uint_as_float(r3[k + e]), __uint_as_float(r3[k + e + 4]));
             }
           }
         }

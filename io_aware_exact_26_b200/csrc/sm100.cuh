@@ -133,6 +133,55 @@ __device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity) 
     if (globaltimer_ns() - t0 > 100000000ull) return;
 }
 
+// Ring of work-unit indices: one producer thread claims units from g_sched and
+// posts them; each consumer warp takes them in the same order.  A posted -1 ends
+// the sequence.
+struct UnitRing {
+  uint64_t full[4];     // count 1: the producer posted slot k & 3
+  uint64_t empty[4];    // count = number of consumer warps
+  int idx[4];
+};
+
+__device__ __forceinline__ void unit_ring_init(UnitRing& r, uint32_t consumers) {
+  for (int i = 0; i < 4; ++i) {
+    mbar_init(&r.full[i], 1);
+    mbar_init(&r.empty[i], consumers);
+  }
+}
+
+// Producer (one thread): claim the k-th unit of this CTA from counter `slot`,
+// post it (or -1 once u >= n), return it; -2 if a wait failed.
+__device__ __forceinline__ int unit_ring_claim(UnitRing& r, int k, int slot, int n) {
+  const int i = k & 3;
+  if (k >= 4 && !mbar_wait(&r.empty[i], ((k >> 2) - 1) & 1)) return -2;
+  int u = static_cast<int>(atomicAdd(&g_sched[slot], 1u));
+  if (u >= n) u = -1;
+  r.idx[i] = u;
+  mbar_arrive(&r.full[i]);              // release: the index is visible before the arrival
+  return u;
+}
+
+// Consumer (one thread standing for its warp): the k-th unit, -1 when none is left.
+__device__ __forceinline__ int unit_ring_take1(UnitRing& r, int k, bool& ok) {
+  const int i = k & 3;
+  ok = mbar_wait(&r.full[i], (k >> 2) & 1);
+  if (!ok) return -1;
+  const int u = *reinterpret_cast<volatile int*>(&r.idx[i]);
+  mbar_arrive(&r.empty[i]);
+  return u;
+}
+
+// Consumer (whole warp): the k-th unit of this CTA, -1 when none is left.
+__device__ __forceinline__ int unit_ring_take(UnitRing& r, int k, int lane, bool& ok) {
+  const int i = k & 3;
+  ok = __all_sync(0xffffffffu, mbar_wait(&r.full[i], (k >> 2) & 1));
+  if (!ok) return -1;
+  const int u = *reinterpret_cast<volatile int*>(&r.idx[i]);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&r.empty[i]);
+  return u;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
