@@ -104,6 +104,16 @@ int attn_get_device_status(void* stream);
 /* Static, human-readable text for a status code. */
 const char* attn_status_string(int status);
 
+/* Diagnostic (no counterpart on the pages): exercises the device-side failure
+ * path that every kernel of this library uses.  Launches one CTA on `stream`
+ * that waits on an mbarrier nothing will ever arrive on, through the same bounded
+ * wait as the kernels but with a limit of `limit_ns` nanoseconds (1 ns .. 1 s).
+ * The wait gives up, records the timeout in the error word and the CTA returns:
+ * nothing hangs, traps or faults.  A following attn_get_device_status() returns
+ * ATTN_ERR_DEVICE_TIMEOUT and clears the word.  Returns ATTN_ERR_INVALID_ARG for
+ * a limit out of range, ATTN_ERR_LAUNCH if the launch is refused, else ATTN_OK. */
+int attn_selftest_timeout(long long limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

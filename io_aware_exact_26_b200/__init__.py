@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     attn_bwd_workspace_size,
     attn_fwd,
     attn_get_device_status,
+    attn_selftest_timeout,
     attn_status_string,
     lib,
     library_path,

@@ -48,6 +48,8 @@ def lib():
     L.attn_get_device_status.restype = i
     L.attn_status_string.argtypes = [i]
     L.attn_status_string.restype = ctypes.c_char_p
+    L.attn_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
+    L.attn_selftest_timeout.restype = i
     _lib = L
     return L
 
@@ -150,6 +152,13 @@ def attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, *, scale=None, causal=Fals
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd_noalloc")
     return dq, dk, dv
+
+
+def attn_selftest_timeout(limit_ns: int, stream=None) -> None:
+    """Launch the bounded-wait self-test (one CTA waits on a barrier nothing arrives on)."""
+    st = int(lib().attn_selftest_timeout(int(limit_ns), _stream_ptr(stream)))
+    if st != 0:
+        raise AttnError(st, "attn_selftest_timeout")
 
 
 def attn_get_device_status(stream=None) -> int:

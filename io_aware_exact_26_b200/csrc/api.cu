@@ -282,6 +282,31 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                   kNoAllocScratchBytes, stream);
 }
 
+}  // extern "C"
+
+namespace {
+// Waits on an mbarrier that nothing arrives on, with the kernels' bounded-wait
+// code and a short limit: the wait gives up, records the timeout in the error
+// word and the kernel returns.
+__global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    attn::mbar_init(&bar, 1);
+    attn::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)attn::mbar_wait_for(&bar, 0, limit_ns);
+}
+}  // namespace
+
+extern "C" {
+
+int attn_selftest_timeout(long long limit_ns, void* stream) {
+  if (limit_ns <= 0 || limit_ns > 1000000000LL) return ATTN_ERR_INVALID_ARG;
+  selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<unsigned long long>(limit_ns));
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
 int attn_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_LAUNCH;
   int v = 0, zero = 0;

@@ -111,19 +111,22 @@ constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
 // Bounded wait for the mbarrier phase with the given parity to complete.  Gives
 // up (returns false) after kWaitTimeoutNs, recording error 1, or as soon as any
 // CTA has recorded an error.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 0) {
       if (status_set()) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         record_error(&g_attn_status, 1);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitTimeoutNs);
 }
 
 // Bounded wait used only on error paths, to let copies already in flight land.

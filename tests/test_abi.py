@@ -27,7 +27,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
-         "attn_status_string"])
+         "attn_status_string", "attn_selftest_timeout"])
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -88,3 +88,9 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "library_path", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         binding.lib()
+
+
+def test_selftest_timeout_rejects_out_of_range_limits(L):
+    assert L.attn_selftest_timeout(0, None) == -1
+    assert L.attn_selftest_timeout(-5, None) == -1
+    assert L.attn_selftest_timeout(2_000_000_000, None) == -1
