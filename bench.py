@@ -176,6 +176,25 @@ def config_dict(w: Workload, n_gpus):
             "l2": "inputs larger than L2 (126 MB); no flush"}
 
 
+def rank_seed(w: Workload, rank: int) -> int:
+    """Each rank times its own replica of the workload on its own synthetic inputs."""
+    return w.seed + 101 * rank
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of per-rank timings (the slowest rank sets the job's time)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_tflops(flops_per_rank, world, ms):
+    """Whole-job throughput: every rank processes flops_per_rank in ms (the max over ranks)."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def run_reference(args, rank, world):
     """The reference arm: the fp64 oracle on the host cores, bounded samples per step."""
     if rank != 0:
@@ -235,7 +254,7 @@ def main():
     w = WORKLOADS[args.workload]
     has_bwd = "bwd" in w.passes
     dev = torch.device("cuda", local)
-    x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed + 101 * rank, qk_std=w.qk_std, vo_std=w.vo_std,
+    x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=rank_seed(w, rank), qk_std=w.qk_std, vo_std=w.vo_std,
                     boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=has_bwd)
     q, k, v = x["q"], x["k"], x["v"]
     do = x.get("do")
@@ -286,14 +305,11 @@ def main():
     total_ms = start.elapsed_time(stop)
     fwd_ms = [a.elapsed_time(b) for a, b, _ in evs]
     bwd_ms = [b.elapsed_time(c) for _, b, c in evs] if has_bwd else []
-    t = torch.tensor([total_ms, statistics.mean(fwd_ms), statistics.mean(bwd_ms) if bwd_ms else 0.0],
-                     dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_avg, bwd_avg = t.tolist()
+    total_ms, fwd_avg, bwd_avg = max_over_ranks(
+        [total_ms, statistics.mean(fwd_ms), statistics.mean(bwd_ms) if bwd_ms else 0.0], dist, dev)
     ms_per_step = total_ms / args.steps
     f_fwd, f_bwd = step_flops(w)
-    value = (f_fwd + f_bwd) * world / (ms_per_step * 1e-3) / 1e12
+    value = weak_scaling_tflops(f_fwd + f_bwd, world, ms_per_step)
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     host = {n: x[n].cpu().pin_memory() for n in x}
@@ -319,11 +335,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = te.item() / args.e2e_steps
-    e2e_value = (f_fwd + f_bwd) * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0] / args.e2e_steps
+    e2e_value = weak_scaling_tflops(f_fwd + f_bwd, world, e2e_ms)
 
     # ---- roofline of the dominant kernel (backward when present)
     peaks, peaks_kind = load_peaks()
