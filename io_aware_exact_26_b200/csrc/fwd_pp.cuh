@@ -25,9 +25,11 @@
 //   warp 17          MMA issuer
 // TMEM: S_A at 0, S_B at 128 (P written over S as bf16: keys 0-63 in columns
 // 0-31, keys 64-127 in 64-95), O_A at 256, O_B at 256 + D.
-// Per team the loop is S(j) -> softmax(j) -> PV(j) -> S(j+1): one S buffer per
-// tile, so S(j+1) is issued only after PV(j) has completed (no reliance on the
-// order in which the tensor cores retire MMAs for the aliasing of P and S).
+// Per team the loop is S(j) -> softmax(j) -> PV(j) -> S(j+1), one S buffer per
+// tile with P written over it.  S(j+1) is issued right behind PV(j): MMAs issued
+// by one thread are performed in issue order, so PV(j) has read P(j) before
+// S(j+1) writes those columns, and the commit that signals S(j+1) also covers
+// PV(j).
 // Each step a team's two groups exchange partial row maxima of the tile in
 // shared memory; the exp2 with folded scale and the lazy rescale threshold are
 // described in fwd.cuh.
@@ -261,7 +263,6 @@ __global__ void __launch_bounds__(576, 1)
           const int gsx = x ? gs1 : gs0, uux = x ? uu1 : uu0;
           if (!ok || w.n(x) == 0) continue;
           ok = wait(&sh.q_full[x], uux & 1);
-          if (ok && gsx >= 1) ok = wait(&sh.pv_done[x], (gsx - 1) & 1);   // previous unit's last PV
           if (!ok) continue;
           tc_fence_after();
           issue_s(x, st, w.n(x) == 1);
@@ -291,10 +292,9 @@ __global__ void __launch_bounds__(576, 1)
               ok = wait(&sh.k_full[kc & 1], (kc >> 1) & 1);
               k_ready = true;
             }
-            if (ok) ok = wait(&sh.pv_done[x], g & 1);     // P_X(j) read: the S buffer may be overwritten
             if (!ok) continue;
             tc_fence_after();
-            issue_s(x, kc & 1, j + 2 == nx);
+            issue_s(x, kc & 1, j + 2 == nx);             // in issue order behind PV_X(j)
           }
         }
         if (!ok) break;
@@ -391,8 +391,8 @@ __global__ void __launch_bounds__(576, 1)
           lsum = f2pack(l0 * alpha, l1 * alpha);
           m_used = m_new;
         }
-        // Rescale this group's O columns if the max moved.  S_X(j) was issued only
-        // after PV_X(j-1) completed, so O already holds every step before j; the
+        // Rescale this group's O columns if the max moved.  The commit that signalled
+        // S_X(j) also covers PV_X(j-1), so O already holds every step before j; the
         // wait below is then immediate.
         if (__any_sync(0xffffffffu, need && j > 0)) {
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[x], (g - 1) & 1));
