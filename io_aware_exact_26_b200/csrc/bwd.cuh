@@ -296,7 +296,8 @@ __global__ void __launch_bounds__(320, 1)
     auto issue_st = [&](int g) -> bool {   // S^T(g) = K Q(g)^T
       const int st = g & 1;
       if (!wait(&sh.qdo_full[st], (g >> 1) & 1)) return false;
-      if (g >= 1 && !wait(&sh.v_done, (g - 1) & 1)) return false;      // P^T(g-1) consumed
+      // S^T(g) overwrites P^T(g-1): issued behind dV(g-1) by this thread, which the
+      // tensor cores perform first (MMAs of one thread run in issue order).
       tc_fence_after();
       if (leader) {
         const uint32_t q_lo = q_lo0 + st * (C::kTile >> 4);
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(320, 1)
     };
     auto issue_dp = [&](int g) -> bool {   // dP^T(g) = V dO(g)^T
       const int st = g & 1;
-      if (g >= 1 && !wait(&sh.k_done, (g - 1) & 1)) return false;      // dS^T(g-1) consumed
+      // dP^T(g) overwrites dS^T(g-1): issued behind dK(g-1), performed after it.
       tc_fence_after();
       if (leader) {
         const uint32_t do_lo = do_lo0 + st * (C::kTile >> 4);
@@ -662,7 +663,7 @@ __global__ void __launch_bounds__(352, 1)
     auto issue_s = [&](int g) -> bool {     // S(g) = Q K(g)^T into buffer g % 2
       const int st = g % C::KVST, sb = g & 1;
       if (!wait(&sh.k_full[st], (g / C::KVST) & 1)) return false;
-      if (g >= 2 && !wait(&sh.q_done[sb], ((g >> 1) - 1) & 1)) return false;   // dS(g-2) consumed
+      // S(g) overwrites dS(g-2): issued behind dQ(g-2), performed after it.
       tc_fence_after();
       if (leader) {
         const uint32_t k_lo = k_lo0 + st * (C::kTile >> 4);

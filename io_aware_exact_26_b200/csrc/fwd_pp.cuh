@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(576, 1)
         ok = wait(&sh.k_full[st], (kc >> 1) & 1);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          const int gsx = x ? gs1 : gs0, uux = x ? uu1 : uu0;
+          const int uux = x ? uu1 : uu0;
           if (!ok || w.n(x) == 0) continue;
           ok = wait(&sh.q_full[x], uux & 1);
           if (!ok) continue;
