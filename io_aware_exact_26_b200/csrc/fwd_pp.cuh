@@ -50,8 +50,12 @@ struct PpCfg {
   static constexpr int kFmaPairs = 0;
   static constexpr int kTmemCols = 512;
   static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
-  static constexpr int kOffQ = 0;                       // Q_A, Q_B
-  static constexpr int kOffK = 2 * kTile;
+  // Q buffers per team: two at d = 64, so the next unit's Q loads while the current
+  // unit still reads its own (short units, e.g. N = 1024, would wait for it); one
+  // at d = 128, where shared memory has no room and units are longer.
+  static constexpr int QST = (D == 64) ? 2 : 1;
+  static constexpr int kOffQ = 0;                       // Q slots [team][QST]
+  static constexpr int kOffK = 2 * QST * kTile;
   static constexpr int kOffV = kOffK + KST * kTile;
   static constexpr int kOffSh = kOffV + VST * kTile;
   static constexpr int kLayout = kOffSh + 8192;
@@ -62,7 +66,7 @@ struct PpCfg {
 struct PpShared {
   float xmax[2][2][2][128];   // [team][parity][group][row] partial row maxima of a step
   float xsum[2][2][128];      // [team][group][row] partial row sums of a unit
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2][2], q_empty[2][2];   // [team][Q slot]
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t s_full[2];         // per team: S of its current step complete
   uint64_t p_ready[2];        // per team: P written by its 8 warps
@@ -134,8 +138,10 @@ __global__ void __launch_bounds__(576, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.q_full[i], 1);
-      mbar_init(&sh.q_empty[i], 1);
+      for (int q = 0; q < C::QST; ++q) {
+        mbar_init(&sh.q_full[i][q], 1);
+        mbar_init(&sh.q_empty[i][q], 1);
+      }
       mbar_init(&sh.k_full[i], 1);
       mbar_init(&sh.k_empty[i], 1);
       mbar_init(&sh.v_full[i], 1);
@@ -174,10 +180,12 @@ __global__ void __launch_bounds__(576, 1)
         if (u < 0) break;
         const PpUnit w = pp_unit(p, u);
         auto load_q = [&](int x, int uq) -> bool {     // Q of team x, its uq-th unit
-          if (uq >= 1 && !mbar_wait(&sh.q_empty[x], (uq - 1) & 1)) return false;
-          mbar_arrive_expect_tx(&sh.q_full[x], C::kTile);
+          const int qs = uq % C::QST;
+          if (uq >= C::QST && !mbar_wait(&sh.q_empty[x][qs], ((uq / C::QST) - 1) & 1)) return false;
+          mbar_arrive_expect_tx(&sh.q_full[x][qs], C::kTile);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ + x * C::kTile + c * C::kBox, &tmq, &sh.q_full[x], c * 64, w.qt(x) * 128, w.bh(x));
+            tma_load_3d(sQ + (x * C::QST + qs) * C::kTile + c * C::kBox, &tmq, &sh.q_full[x][qs], c * 64,
+                        w.qt(x) * 128, w.bh(x));
           return true;
         };
         ok = load_q(0, uq0++);
@@ -223,9 +231,9 @@ __global__ void __launch_bounds__(576, 1)
     int uu0 = 0, uu1 = 0;        // units per team
     bool ok = true;
     // S_X = Q_X K^T for team x from K stage st
-    auto issue_s = [&](int x, int st, bool last) {
+    auto issue_s = [&](int x, int qs, int st, bool last) {
       if (leader) {
-        const uint32_t q_lo = q_lo0 + x * (C::kTile >> 4);
+        const uint32_t q_lo = q_lo0 + (x * C::QST + qs) * (C::kTile >> 4);
         const uint32_t k_lo = k_lo0 + st * (C::kTile >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
@@ -233,7 +241,7 @@ __global__ void __launch_bounds__(576, 1)
           umma_ss_lo(tmem + (x ? C::kS1 : C::kS0), q_lo + off, k_lo + off, hi, idS, k > 0);
         }
         umma_commit(&sh.s_full[x]);
-        if (last) umma_commit(&sh.q_empty[x]);
+        if (last) umma_commit(&sh.q_empty[x][qs]);
       }
       __syncwarp();
     };
@@ -262,10 +270,10 @@ __global__ void __launch_bounds__(576, 1)
         for (int x = 0; x < 2; ++x) {
           const int uux = x ? uu1 : uu0;
           if (!ok || w.n(x) == 0) continue;
-          ok = wait(&sh.q_full[x], uux & 1);
+          ok = wait(&sh.q_full[x][uux % C::QST], (uux / C::QST) & 1);
           if (!ok) continue;
           tc_fence_after();
-          issue_s(x, st, w.n(x) == 1);
+          issue_s(x, uux % C::QST, st, w.n(x) == 1);
         }
         if (!ok) break;
         if (leader) umma_commit(&sh.k_empty[st]);
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(576, 1)
             }
             if (!ok) continue;
             tc_fence_after();
-            issue_s(x, kc & 1, j + 2 == nx);             // in issue order behind PV_X(j)
+            issue_s(x, uux % C::QST, kc & 1, j + 2 == nx);   // in issue order behind PV_X(j)
           }
         }
         if (!ok) break;
