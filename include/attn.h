@@ -55,7 +55,11 @@ typedef enum {
 } attn_status_t;
 
 /* Forward: O and LSE for every (b, h, i).
- * Reads q, k, v; writes o and lse.  Returns ATTN_OK or a negative status. */
+ * Reads q, k, v; writes o and lse.  Returns ATTN_OK or a negative status.
+ * Enqueues two kernels on `stream`: a one-thread kernel that zeroes this call's
+ * work counter, then the forward, whose persistent CTAs claim work units from
+ * that counter.  Each call takes the next of 128 counters (rotating), so up to
+ * 128 forward calls may be in flight at once, on any streams. */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
              void* stream);
