@@ -120,7 +120,6 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   p.N = N;
   p.G = Hq / Hkv;
   p.n_qtiles = (N + 127) / 128;
-  p.total_tiles = p.n_qtiles * B * Hq;
   p.c = scale * 1.4426950408889634f;
   p.causal = causal;
   const int units = B * Hkv * ((p.G * p.n_qtiles + 1) / 2);

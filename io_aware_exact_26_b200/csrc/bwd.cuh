@@ -171,7 +171,7 @@ struct KvShared {
   uint64_t qdo_full[2], qdo_empty[2];
   uint64_t s_full, dp_full;     // S^T / dP^T of the step in TMEM
   uint64_t p_ready, ds_ready;   // P^T / dS^T (bf16) written back by both dS warpgroups
-  uint64_t v_done, k_done;      // dV / dK MMA of the step complete
+  uint64_t k_done;              // dK MMA of the step complete (the item's last one ends it)
   uint64_t acc_free;            // dV / dK of the previous item read out
   uint64_t drain;
   uint32_t tmem_base;
@@ -215,7 +215,6 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(&sh.dp_full, 1);
     mbar_init(&sh.p_ready, 8);
     mbar_init(&sh.ds_ready, 8);
-    mbar_init(&sh.v_done, 1);
     mbar_init(&sh.k_done, 1);
     mbar_init(&sh.acc_free, 8);
     mbar_init(&sh.drain, 1);
@@ -347,7 +346,6 @@ __global__ void __launch_bounds__(320, 1)
           for (int k = 0; k < 8; ++k)
             umma_ts_lo(tmem + C::kDV, tmem + C::kS + (k >> 2) * 64 + (k & 3) * 8, do_mn + ((k * 2048) >> 4), hi,
                        idKV, !(u == 0 && k == 0));
-          umma_commit(&sh.v_done);
         }
         __syncwarp();
         if (u + 1 < n_steps && !issue_st(gs + 1)) { ok = false; break; }

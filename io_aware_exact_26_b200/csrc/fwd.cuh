@@ -20,7 +20,7 @@ struct FwdParams {
   void* o;
   float* lse;
   int B, Hq, Hkv, N, G;
-  int n_qtiles, total_tiles;
+  int n_qtiles;
   float c;          // scale * log2(e)
   int causal;
   int sched_slot;   // g_sched slot this launch claims work units from

@@ -13,8 +13,7 @@ namespace attn {
 
 // Device status word of the library (the whole device side is one translation
 // unit): 0 = ok; otherwise the first error code recorded.
-// Codes: 1 = an mbarrier wait timed out, 2 = a dQ ordering wait timed out,
-//        3 = shared memory could not be aligned for the swizzled tiles.
+// Code 1 = an mbarrier wait timed out (the only code the kernels record).
 __device__ int g_attn_status = 0;
 
 // Work-unit counters for dynamically scheduled kernels: each launch takes one
@@ -36,7 +35,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 // One lane of a converged warp (elect.sync); the others get false.
 __device__ __forceinline__ bool elect_one() {
@@ -164,15 +162,6 @@ __device__ __forceinline__ int unit_ring_claim(UnitRing& r, int k, int slot, int
   return u;
 }
 
-// Consumer (one thread standing for its warp): the k-th unit, -1 when none is left.
-__device__ __forceinline__ int unit_ring_take1(UnitRing& r, int k, bool& ok) {
-  const int i = k & 3;
-  ok = mbar_wait(&r.full[i], (k >> 2) & 1);
-  if (!ok) return -1;
-  const int u = *reinterpret_cast<volatile int*>(&r.idx[i]);
-  mbar_arrive(&r.empty[i]);
-  return u;
-}
 
 // Consumer (whole warp): the k-th unit of this CTA, -1 when none is left.
 __device__ __forceinline__ int unit_ring_take(UnitRing& r, int k, int lane, bool& ok) {
@@ -244,27 +233,7 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both described by UMMA smem descriptors.
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
-// D[tmem] (+)= A[tmem] * B[smem]^T; A is M x K, 16-bit elements packed two per column.
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 // Split shared-memory descriptors (128B swizzle): the low word holds the start
 // address and the leading byte offset, the high word the stride byte offset,
@@ -353,18 +322,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -373,38 +330,7 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Register reallocation between warpgroups (all four warps of a warpgroup must
-// execute the same instruction).  The sum over warpgroups must not exceed the
-// registers the block was launched with.
-template <uint32_t N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
 
-// ---------------------------------------------------------------- descriptors
-// UMMA shared-memory matrix descriptor (sm_100 layout):
-//   [0,14) start address >> 4, [16,30) leading byte offset >> 4,
-//   [32,46) stride byte offset >> 4, [46,48) version = 1,
-//   [49,52) base offset = 0, [52] LBO mode = 0, [61,64) swizzle (2 = 128-byte).
-// K-major, 128B swizzle: rows are 128 bytes (64 bf16 of K), 8-row groups are
-//   1024 bytes apart (SBO); LBO is unused.  Advancing K by 16 elements inside the
-//   swizzle atom is a +32 byte start address.
-// MN-major, 128B swizzle: 64 MN-contiguous elements per 128-byte row, 8 K-rows
-//   per 1024-byte atom (SBO between K groups), LBO between 64-wide MN blocks.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(2) << 61;
-  return d;
-}
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulate:
 //   [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),
@@ -478,16 +404,6 @@ __device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float& y0, flo
   y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-// bf16 bit pattern of x rounded toward +infinity (positive finite values round
-// their magnitude up; negative values and infinities truncate, which is upward).
-__device__ __forceinline__ uint16_t bf16_bits_round_up(float x) {
-  uint32_t b = __float_as_uint(x);
-  if (x > 0.f && b < 0x7f800000u) b += 0xFFFFu;
-  return static_cast<uint16_t>(b >> 16);
-}
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t v) {
-  return __uint_as_float(static_cast<uint32_t>(v) << 16);
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
