@@ -19,9 +19,9 @@
 //   warps 0-7, 8-15  softmax teams; inside a team, group k = (warp % 8) / 4 owns
 //                    keys [64k, 64k+64) of each S tile and O columns
 //                    [k*D/2, (k+1)*D/2); thread = query row = TMEM lane.
-//   warp 16          TMA producer: Q_A, Q_B (one buffer each), K and V rings (2
-//                    stages each), loaded as K(0) V(0) K(1) V(1) ..., the order in
-//                    which the MMA warp releases their stages
+//   warp 16          TMA producer: Q_A, Q_B (one buffer per team at d = 128, two
+//                    at d = 64), K and V rings (2 stages each), loaded as K(0) V(0)
+//                    K(1) V(1) ..., the order in which the MMA warp releases them
 //   warp 17          MMA issuer
 // TMEM: S_A at 0, S_B at 128 (P written over S as bf16: keys 0-63 in columns
 // 0-31, keys 64-127 in 64-95), O_A at 256, O_B at 256 + D.
