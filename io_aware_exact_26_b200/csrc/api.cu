@@ -184,7 +184,8 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   p.c = scale * 1.4426950408889634f;
   p.scale = scale;
   // dK, dV: one item per (b, kv-head, key tile)
-  p.total_items = B * Hkv * nt;
+  p.npair = (nt + 1) / 2;
+  p.total_items = B * Hkv * (causal ? p.npair : nt);
   int grid = p.total_items < sms ? p.total_items : sms;
   attn_bwd_kv_kernel<D><<<grid, KvCfg<D>::kThreads, KvCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
   if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;

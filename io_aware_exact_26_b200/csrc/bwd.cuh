@@ -116,6 +116,7 @@ struct BwdParams {
   const float* dd;
   int B, Hq, Hkv, N, G;
   int nt;           // number of 128-row tiles along N
+  int npair;        // (nt + 1) / 2: key-tile pairs per KV head (causal dK/dV units)
   int total_items;
   int causal;
   float c;          // scale * log2(e)
@@ -177,14 +178,36 @@ struct KvShared {
   uint32_t tmem_base;
 };
 
-// item t -> (bh_kv, key tile j); key tile outermost, so the key tiles with the most
-// query tiles (causal) come first
-// Items are numbered KV head by KV head, so the CTAs running at the same time
-// stream the Q/dO of the same few head groups (L2 hits); within a head, key tile
-// j ascending (causal: the item of key tile j sees nt - j query tiles, longest first).
-__device__ __forceinline__ void kv_item(const BwdParams& p, int t, int& bhkv, int& j) {
-  bhkv = t / p.nt;
-  j = t - bhkv * p.nt;
+// Work units of the dK/dV kernel, numbered KV head by KV head, so the CTAs running at
+// the same time stream the Q/dO of the same few head groups.
+//  - Non-causal: unit t is key tile j = t mod nt, one item.
+//  - Causal: unit t is the pair of key tiles (pr, nt-1-pr), two items (one for the
+//    middle tile when nt is odd). Together they see nt+1 query tiles whatever pr is,
+//    so units cost the same and the CTAs that start them together stay in step.
+//    The first item walks its query tiles from the last one down, the second from
+//    its diagonal tile up: at step T of a unit the CTAs of one head group read
+//    query tile nt-1-T or T-1, so each Q/dO tile reaches L2 from HBM about twice
+//    per group instead of once per key tile.
+__device__ __forceinline__ int kv_halves(const BwdParams& p, int t) {
+  if (!p.causal) return 1;
+  const int pr = t % p.npair;
+  return 2 * pr + 1 == p.nt ? 1 : 2;
+}
+__device__ __forceinline__ void kv_item(const BwdParams& p, int t, int hf, int& bhkv, int& j, bool& up) {
+  if (!p.causal) {
+    bhkv = t / p.nt;
+    j = t - bhkv * p.nt;
+    up = false;
+    return;
+  }
+  bhkv = t / p.npair;
+  const int pr = t - bhkv * p.npair;
+  j = hf ? p.nt - 1 - pr : pr;
+  up = hf != 0;
+}
+// s-th query tile an item visits, s in [0, nt - first)
+__device__ __forceinline__ int kv_q_tile(const BwdParams& p, int first, bool up, int s) {
+  return up ? first + s : p.nt - 1 - s;
 }
 __device__ __forceinline__ int kv_first_q(const BwdParams& p, int j) { return p.causal ? j : 0; }
 
@@ -233,9 +256,11 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t pol_reuse = l2_policy_evict_last(), pol_once = l2_policy_evict_first();
       int gs = 0, it = 0, nq = 0, nkv = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
+      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
+      for (int hf = 0; hf < kv_halves(p, t) && ok; ++hf, ++it) {
         int bhkv, j;
-        kv_item(p, t, bhkv, j);
+        bool up;
+        kv_item(p, t, hf, bhkv, j, up);
         if (it >= 1) ok = mbar_wait(&sh.kv_empty, (it - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&sh.kv_full, 2 * C::kTile);
@@ -245,11 +270,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         nkv = it + 1;
         const int b = bhkv / p.Hkv, hk = bhkv - b * p.Hkv;
-        // Query tiles from the last down to the first visible one, the G heads of
-        // the group inside: every item of a head group starts at the same tile, so
-        // the CTAs working on that group read each Q/dO tile at about the same
-        // time and HBM delivers it about once.
-        for (int i = p.nt - 1; i >= kv_first_q(p, j) && ok; --i) {
+        // Query tiles in the item's order, the G heads of the group inside.
+        const int first = kv_first_q(p, j);
+        for (int s = 0; s < p.nt - first && ok; ++s) {
+          const int i = kv_q_tile(p, first, up, s);
           for (int h = 0; h < p.G; ++h, ++gs) {
             const int bhq = b * p.Hq + hk * p.G + h;
             const int st = gs & 1;
@@ -326,9 +350,11 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       return true;
     };
-    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
+    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
+    for (int hf = 0; hf < kv_halves(p, t) && ok; ++hf, ++it) {
       int bhkv, j;
-      kv_item(p, t, bhkv, j);
+      bool up;
+      kv_item(p, t, hf, bhkv, j, up);
       ok = wait(&sh.kv_full, it & 1);
       if (!ok) break;
       const int n_steps = p.G * (p.nt - kv_first_q(p, j));
@@ -384,12 +410,16 @@ __global__ void __launch_bounds__(320, 1)
     const float c = p.c;
     int gs = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x) {
+    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
+    for (int hf = 0; hf < kv_halves(p, t) && ok; ++hf) {
       int bhkv, j;
-      kv_item(p, t, bhkv, j);
+      bool up;
+      kv_item(p, t, hf, bhkv, j, up);
       const int key = j * 128 + r;
       const bool key_live = key < p.N;
-      for (int i = p.nt - 1; i >= kv_first_q(p, j) && ok; --i) {
+      const int first = kv_first_q(p, j);
+      for (int s = 0; s < p.nt - first && ok; ++s) {
+        const int i = kv_q_tile(p, first, up, s);
         for (int h = 0; h < p.G && ok; ++h, ++gs) {
           const int st = gs & 1;
           const float* sLse = sVec + st * 256 + 64 * hb;
