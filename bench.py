@@ -220,9 +220,12 @@ def run_reference(args, rank, world):
             total_heads += heads
     value = statistics.median(vals) if vals else None
     sample = f"{total_heads} whole heads (B=1,H=1 slices of {w.name}) over {args.steps} timed steps"
+    # ms_per_step: one whole step of the workload (all heads) at the sampled rate
+    ms = sum(step_flops(w)) / (value * 1e12) * 1e3 if value else None
     line = {"impl": "reference", "metric": "attention fwd+bwd TFLOPS" if "bwd" in w.passes else "attention fwd TFLOPS",
             "value": value, "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "higher_is_better": True, "dtype": "f64", "data": "synthetic", "config": config_dict(w, args.gpus),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": config_dict(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

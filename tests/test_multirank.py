@@ -74,3 +74,11 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     bench.run_reference(Args, rank=0, world=2)
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    # the same keys as the main arm's line, plus the baseline description
+    for key in ("metric", "unit", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    # ms_per_step is one whole step of the workload at the measured rate
+    f, fb = bench.step_flops(bench.WORKLOADS[Args.workload])
+    assert abs(line["ms_per_step"] - (f + fb) / (line["value"] * 1e12) * 1e3) <= 1e-9 * line["ms_per_step"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
