@@ -63,6 +63,27 @@ WORKLOADS = {
         qk_std=3.0, boost_frac=0.01, boost=8.0, seed=1004),
 }
 
+# Sequence-length sweep: a fixed number of tokens B*N and a fixed model width Hq*d,
+# so the work per token grows with N and the FLOP/byte of each head is ~N/4.  At
+# N = 32768 one sequence already exceeds the token budget, so B stays 1 there.
+SWEEP_TOKENS = 16384
+SWEEP_WIDTH = 2048
+SWEEP_N = (1024, 2048, 4096, 8192, 16384, 32768)
+SWEEP_D = (64, 128)
+
+
+def sweep_workloads():
+    """Workloads of the sequence-length sweep, non-causal and causal, both head sizes; seeds 2000+k."""
+    out = []
+    for d in SWEEP_D:
+        for causal in (False, True):
+            for n in SWEEP_N:
+                B = max(1, SWEEP_TOKENS // n)
+                H = SWEEP_WIDTH // d
+                name = f"sweep_{'causal' if causal else 'full'}_b{B}_h{H}_n{n}_d{d}"
+                out.append(Workload(name, B, H, H, n, d, causal, "fwd+bwd", seed=2000 + len(out)))
+    return out
+
 
 def _normal_bf16(shape, std, gen, device):
     x = torch.randn(shape, generator=gen, dtype=torch.float32, device=device)

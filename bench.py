@@ -1,6 +1,7 @@
 """Benchmark: exact attention forward + backward TFLOPS on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py --sweep [--sweep-reps R] [--warmup W]
 
 One step = one pass of the whole hot path over one batch: attn_fwd (O, LSE) then
 attn_bwd (dQ, dK, dV) for workloads that train, attn_fwd alone for forward-only
@@ -13,6 +14,10 @@ and the max time over ranks is reported.
 
 Printed as one JSON line by rank 0.  ``--impl reference`` times the fp64 CPU
 oracle instead (the reference arm), on a bounded sample of the same workload.
+``--sweep`` times attn_fwd and attn_bwd separately over the sequence-length sweep
+(B*N and Hq*d fixed, N from 1K to 32K, d 64 and 128, causal and not) on one GPU
+and prints one JSON line per point: the median of R timed calls after W warm-up
+calls, each call's inputs larger than L2.
 """
 from __future__ import annotations
 
@@ -30,7 +35,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from attn_inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+from attn_inputs import WORKLOADS, Workload, make_inputs, sweep_workloads  # noqa: E402
 from io_aware_exact_26_b200 import accounting as acc  # noqa: E402
 
 DEFAULT_WORKLOAD = "gpt2_medium_b64_h16_n1024_d64"
@@ -231,6 +236,58 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """One JSON line per sweep point: forward and backward timed apart, median over calls."""
+    import torch
+    import io_aware_exact_26_b200 as attn
+
+    peaks, peaks_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    for w in sweep_workloads():
+        x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, device=dev, with_grad=True)
+        q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(attn.attn_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.N, w.d, w.causal), dtype=torch.uint8,
+                         device=dev)
+
+        def fwd():
+            attn.attn_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal)
+
+        def bwd():
+            attn.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale=w.scale, causal=w.causal, workspace=ws)
+
+        f_fwd, f_bwd = step_flops(w)
+        point = {"sweep": "B*N=16384, Hq*d=2048", "workload": w.name, "B": w.B, "Hq": w.Hq, "N": w.N, "d": w.d,
+                 "causal": w.causal, "reps": args.sweep_reps, "warmup": args.warmup,
+                 "peak": peak, "peak_source": f"{peaks_kind} bf16 dense (burst)"}
+        sampler = ClockSampler(0)
+        sampler.start()
+        for name, fn, flops in (("fwd", fwd, f_fwd), ("bwd", bwd, f_bwd)):
+            for _ in range(args.warmup):
+                fn()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.sweep_reps)]
+            for a, b in evs:
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            if attn.attn_get_device_status() != 0:
+                raise SystemExit(f"device-side error in the sweep at {w.name} ({name})")
+            ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+            tf = flops / (ms * 1e-3) / 1e12
+            point[name] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4)}
+        point["clocks"] = sampler.stop()
+        print(json.dumps(point), flush=True)
+        del x, q, k, v, do, o, lse, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -241,8 +298,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="time the sequence-length sweep, one line per point")
+    ap.add_argument("--sweep-reps", type=int, default=50)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.sweep:
+        run_sweep(args)
+        return
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
