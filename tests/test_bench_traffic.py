@@ -71,3 +71,12 @@ def test_entries_are_stamped_and_read_back_only_for_the_same_sources(tmp_path, m
 def test_forward_only_workloads_get_no_backward_entry(tmp_path):
     entry = bench_traffic.update("causal_b8_h16_n4096_d128", sample_csv(), str(tmp_path), revision="abc1234")
     assert set(entry) == {"fwd"}
+
+
+def test_source_fingerprint_ignores_comments_and_layout_but_not_code():
+    src = "int f(int x) {\n  // scale\n  return 2 * x; /* twice */\n}\n"
+    same = "int f(int x) { return 2 * x; }  // reformatted\n"
+    other = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench.code_text(src) == bench.code_text(same)
+    assert bench.code_text(src) != bench.code_text(other)
+    assert "scale" not in bench.code_text(src) and "twice" not in bench.code_text(src)
