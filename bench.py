@@ -38,7 +38,8 @@ sys.path.insert(0, ROOT)
 from attn_inputs import WORKLOADS, Workload, make_inputs, sweep_workloads  # noqa: E402
 from io_aware_exact_26_b200 import accounting as acc  # noqa: E402
 
-DEFAULT_WORKLOAD = "gpt2_medium_b64_h16_n1024_d64"
+# The largest single-GPU workload (forward + backward, causal, d = 128, N = 32768).
+DEFAULT_WORKLOAD = "long_causal_b1_h32_n32768_d128"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -142,40 +143,93 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def time_oracle(w: Workload, budget_s: float, max_heads=None):
-    """Time the fp64 oracle on whole heads of the workload until the budget is spent.
+def cpu_info():
+    """The host the oracle runs on: CPU model, logical CPUs, CPUs this process may use."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count()
+    return {"model": model, "logical_cpus": os.cpu_count(), "usable_cpus": usable}
 
-    Returns (TFLOPS, seconds, heads, threads).  Test infrastructure: only this
-    baseline leg of the benchmark runs the oracle.
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+ORACLE_BLOCK = 1024
+
+
+def time_oracle(w: Workload, budget_s: float, max_blocks=None, min_blocks=1, seed_offset=0):
+    """Time the fp64 oracle on 1024-row blocks of one head of the workload.
+
+    Rows are independent, so the oracle's cost for a whole step is the cost of one
+    row block times the number of row blocks in the step (B * Hq * ceil(N / 1024));
+    the oracle materialises the full masked score block whatever the mask, so every
+    block of a head costs the same.  Blocks are drawn from one synthetic head of the
+    workload's shape and distribution until ``budget_s`` seconds are spent (at least
+    ``min_blocks``).  Returns a dict with the extrapolated step time and rate.
+    Test infrastructure: only the baseline legs of the benchmark run the oracle.
     """
     import numpy as np
     from attn_inputs import to_f64
     from oracle import reference as ref
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"),
-                      default=1)
-    except Exception:
-        threads = os.cpu_count() or 1
-    heads, spent, flops = 0, 0.0, 0.0
-    b = h = 0
+    has_bwd = "bwd" in w.passes
+    x = make_inputs(1, 1, 1, w.N, w.d, seed=w.seed + 17 + seed_offset, qk_std=w.qk_std, vo_std=w.vo_std,
+                    boost_frac=w.boost_frac, boost=w.boost, with_grad=has_bwd)
+    qh, kh, vh = to_f64(x["q"][0, 0]), to_f64(x["k"][0, 0]), to_f64(x["v"][0, 0])
+    doh = to_f64(x["do"][0, 0]) if has_bwd else None
+    nblk = (w.N + ORACLE_BLOCK - 1) // ORACLE_BLOCK
+    order = np.random.default_rng(w.seed + seed_offset).permutation(nblk)
+    spent, blocks, rows = 0.0, 0, 0
     while True:
-        x = make_inputs(1, 1, 1, w.N, w.d, seed=w.seed + 17 * heads, qk_std=w.qk_std, vo_std=w.vo_std,
-                        boost_frac=w.boost_frac, boost=w.boost, with_grad="bwd" in w.passes)
-        q, k, v = to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"])
+        a = int(order[blocks % nblk]) * ORACLE_BLOCK
+        r = np.arange(a, min(w.N, a + ORACLE_BLOCK))
         t0 = time.perf_counter()
-        ref.ref_fwd(q, k, v, w.scale, w.causal)
-        f = acc.flops_fwd(1, 1, w.N, w.d, w.causal)
-        if "bwd" in w.passes:
-            ref.ref_bwd(q, k, v, to_f64(x["do"]), w.scale, w.causal)
-            f += acc.flops_bwd(1, 1, w.N, w.d, w.causal)
+        ref.attend_head(qh, kh, vh, w.scale, w.causal, rows=r)
+        if has_bwd:
+            ref.grad_rows(qh, kh, vh, doh, w.scale, w.causal, r)
         spent += time.perf_counter() - t0
-        flops += f
-        heads += 1
-        if spent >= budget_s or (max_heads and heads >= max_heads):
+        blocks += 1
+        rows += len(r)
+        if (spent >= budget_s and blocks >= min_blocks) or (max_blocks and blocks >= max_blocks):
             break
-    del b, h, np
-    return flops / spent / 1e12, spent, heads, threads
+    # step time at the sampled per-row cost (rows of the last block may be fewer)
+    step_rows = w.B * w.Hq * w.N
+    step_s = spent / rows * step_rows
+    return {"tflops": sum(step_flops(w)) / step_s / 1e12, "step_ms": step_s * 1e3, "seconds": spent,
+            "blocks": blocks, "rows": rows, "step_rows": step_rows, "threads": blas_threads()}
+
+
+def single_thread_oracle(budget_s=2.0):
+    """The oracle forward with one BLAS thread on the single-head N=256 d=64 workload."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        return None
+    w = WORKLOADS["single_head_n256_d64"]
+    with threadpool_limits(limits=1, user_api="blas"):
+        r = time_oracle(w, budget_s)
+    return {"workload": w.name, "tflops": round(r["tflops"], 6), "seconds": round(r["seconds"], 2),
+            "calls": r["blocks"], "threads": 1}
+
+
+def oracle_sample_text(w: Workload, r):
+    return (f"{r['blocks']} row blocks of {ORACLE_BLOCK} ({r['rows']} query rows, "
+            f"{'forward + backward' if 'bwd' in w.passes else 'forward'}) of one synthetic head of {w.name}, "
+            f"{r['seconds']:.1f} s; the step's {r['step_rows']} rows are extrapolated at that per-row cost")
 
 
 def step_flops(w: Workload):
@@ -210,29 +264,37 @@ def weak_scaling_tflops(flops_per_rank, world, ms):
 
 
 def run_reference(args, rank, world):
-    """The reference arm: the fp64 oracle on the host cores, bounded samples per step."""
+    """The reference arm: the fp64 oracle on the host cores, a bounded sample per step."""
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
     budget = min(2.0, max(0.2, 90.0 / max(1, args.steps + args.warmup)))
-    vals = []
-    total_heads = 0
+    t_run = time.perf_counter()
+    vals, step_ms, blocks, rows, secs = [], [], 0, 0, 0.0
     threads = 1
     for i in range(args.warmup + args.steps):
-        v, spent, heads, threads = time_oracle(w, budget)
+        r = time_oracle(w, budget, seed_offset=i)
+        threads = r["threads"]
         if i >= args.warmup:
-            vals.append(v)
-            total_heads += heads
+            vals.append(r["tflops"])
+            step_ms.append(r["step_ms"])
+            blocks += r["blocks"]
+            rows += r["rows"]
+            secs += r["seconds"]
     value = statistics.median(vals) if vals else None
-    sample = f"{total_heads} whole heads (B=1,H=1 slices of {w.name}) over {args.steps} timed steps"
-    # ms_per_step: one whole step of the workload (all heads) at the sampled rate
-    ms = sum(step_flops(w)) / (value * 1e12) * 1e3 if value else None
+    ms = statistics.median(step_ms) if step_ms else None
+    sample = (f"{blocks} row blocks of {ORACLE_BLOCK} ({rows} query rows) of synthetic heads shaped like "
+              f"{w.name}, {secs:.1f} s over {args.steps} timed steps; each step's time is extrapolated from "
+              f"its own sample at the sampled per-row cost")
     line = {"impl": "reference", "metric": "attention fwd+bwd TFLOPS" if "bwd" in w.passes else "attention fwd TFLOPS",
             "value": value, "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "config": config_dict(w, args.gpus),
-            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle", "sample": sample},
-            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "ms_per_step": ms, "ms_per_step_extrapolated": True, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_dict(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                             "extrapolated": True, "sample": sample, "host": cpu_info()},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+                    "note": "the oracle reads and writes host memory; no copies"},
+            "run_seconds": round(time.perf_counter() - t_run, 1)}
     print(json.dumps(line), flush=True)
 
 
@@ -291,8 +353,8 @@ def run_sweep(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -387,7 +449,8 @@ def main():
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     host = {n: x[n].cpu().pin_memory() for n in x}
-    outs_dev = {"dq": dq, "dk": dk, "dv": dv} if has_bwd else {"o": o}
+    # the step's results: the forward's O and LSE, and the gradients when it trains
+    outs_dev = {"o": o, "lse": lse, **({"dq": dq, "dk": dk, "dv": dv} if has_bwd else {})}
     out_host = {n: torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for n, t_ in outs_dev.items()}
     h2d = sum(t_.numel() * t_.element_size() for t_ in host.values())
     d2h = sum(t_.numel() * t_.element_size() for t_ in out_host.values())
@@ -443,9 +506,11 @@ def main():
         line["bwd"] = {"ms": round(bwd_avg, 4), "tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 1),
                        "frac_of_peak": round(f_bwd / (bwd_avg * 1e-3) / 1e12 / peak, 4)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, spent, heads, threads = time_oracle(w, args.cpu_budget)
-        line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
-                                "sample": f"{heads} whole heads (B=1,H=1 slices of the workload), {spent:.1f} s"}
+        r = time_oracle(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(r["tflops"], 6), "unit": "TFLOPS", "cores": r["threads"],
+                                "kind": "oracle", "extrapolated": True, "step_ms": round(r["step_ms"], 1),
+                                "sample": oracle_sample_text(w, r), "host": cpu_info(),
+                                "single_thread": single_thread_oracle()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -1,30 +1,43 @@
-"""DRAM traffic of one bench.py run, from an ncu launch list.
+"""Launch lists and DRAM traffic of the benchmark workloads, from narrow ncu captures.
 
-Turns the CSV of an ncu launch list into ``profiles/launches_<workload>.md`` (per kernel:
-launches, time, share, DRAM bytes per launch) and into the workload's entry in
-``profiles/dram_traffic.json``, which bench.py reports as ``roofline.traffic``.
+Two kinds of capture feed ``profiles/``; both run on one GPU, each only after the
+same command line has exited 0 without ncu, always with ``--clock-control none``.
 
-The capture runs on one GPU, after the same command has exited 0 without ncu:
+1. Launch list (time only, one pass per launch) of the full-size bench command:
 
-    python bench.py --workload W --steps 1 --warmup 3 --no-cpu-baseline --e2e-steps 1 > plain.log 2>&1 && \\
-    ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum --clock-control none \\
-        -c 200 --csv --log-file launches.csv \\
-        python bench.py --workload W --steps 1 --warmup 3 --no-cpu-baseline --e2e-steps 1
+       python bench.py --workload W --steps 2 --warmup 3 --no-cpu-baseline --e2e-steps 1 > plain.log 2>&1 && \\
+       ncu --metrics gpu__time_duration.sum --clock-control none -c 60 --csv --log-file launches.csv \\
+           python bench.py --workload W --steps 2 --warmup 3 --no-cpu-baseline --e2e-steps 1
 
-and then, on the same source tree:
+   ``python bench_traffic.py launches --workload W launches.csv`` writes
+   ``profiles/launches_<W>.md`` (per kernel: launches, time, share).
 
-    python bench_traffic.py --workload W launches.csv
+2. DRAM bytes, one kernel per capture (``-k``, ``-c 1``), on a reduced case of the
+   same workload: B (or the head counts, keeping Hq/Hkv) divided by ``--div`` so the
+   inputs stay a few hundred MB but larger than the 126 MB L2:
 
-Each entry is stamped with ``bench.kernel_source_hash()`` of the tree it runs on, so
-bench.py uses it only while the kernels are the ones that were captured.  ncu replays
-every launch serially with cold caches: compare the time SHARES with a live run, not
-the absolute times.
+       python bench_traffic.py run --workload W --div 4 > plain.log 2>&1 && \\
+       ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum --clock-control none \\
+           -k regex:attn_bwd_kv -s 1 -c 1 --csv --log-file dram_bwd_kv.csv \\
+           python bench_traffic.py run --workload W --div 4
+
+   (one such capture per kernel).  ``python bench_traffic.py dram --workload W --div 4
+   dram_*.csv`` scales each kernel's bytes by ``div`` -- every kernel's traffic is a sum
+   over independent (b, kv-head) units, so it grows in proportion to their number --
+   and writes the workload's entry of ``profiles/dram_traffic.json`` and
+   ``profiles/dram_<W>.md``.
+
+Each traffic entry is stamped with ``bench.kernel_source_hash()`` of the tree it runs
+on, so bench.py reports it only while the kernels are the ones that were captured.
+ncu replays launches serially with cold caches: compare time SHARES with a live run,
+not absolute times.
 """
 from __future__ import annotations
 
 import argparse
 import collections
 import csv
+import dataclasses
 import io
 import json
 import os
@@ -36,16 +49,40 @@ sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
 
-METRICS = "gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum"
+DRAM_METRICS = "dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum"
+# kernel name pattern for -k, per kernel of the path, and the pass it belongs to
+KERNELS = {"fwd": ("attn_fwd_pp", "fwd"), "bwd_prep": ("attn_bwd_prep", "bwd"),
+           "bwd_kv": ("attn_bwd_kv", "bwd"), "bwd_q": ("attn_bwd_q", "bwd")}
 _MS = {"nsecond": 1e-6, "ns": 1e-6, "usecond": 1e-3, "us": 1e-3, "msecond": 1.0, "ms": 1.0, "second": 1e3, "s": 1e3}
 _BYTES = {"byte": 1.0, "B": 1.0, "Kbyte": 1e3, "KB": 1e3, "Mbyte": 1e6, "MB": 1e6, "Gbyte": 1e9, "GB": 1e9}
 
 
-def capture_command(workload: str) -> str:
-    sel = "" if workload == bench.DEFAULT_WORKLOAD else f" --workload {workload}"
-    run = f"python bench.py{sel} --steps 1 --warmup 3 --no-cpu-baseline --e2e-steps 1"
-    return (f"{run} > plain.log 2>&1 && \\\nncu --metrics {METRICS} --clock-control none -c 200 --csv "
+def bench_run(workload: str) -> str:
+    return f"python bench.py --workload {workload} --steps 2 --warmup 3 --no-cpu-baseline --e2e-steps 1"
+
+
+def launches_command(workload: str) -> str:
+    run = bench_run(workload)
+    return (f"{run} > plain.log 2>&1 && \\\nncu --metrics gpu__time_duration.sum --clock-control none -c 60 --csv "
             f"--log-file launches.csv {run}")
+
+
+def dram_command(workload: str, div: int, kernel: str) -> str:
+    run = f"python bench_traffic.py run --workload {workload} --div {div}"
+    pat = KERNELS[kernel][0]
+    return (f"{run} > plain.log 2>&1 && \\\nncu --metrics {DRAM_METRICS} --clock-control none -k regex:{pat} "
+            f"-s 1 -c 1 --csv --log-file dram_{kernel}.csv {run}")
+
+
+def reduced(w, div: int):
+    """The workload with its independent (b, kv-head) units divided by ``div``."""
+    if div == 1:
+        return w
+    if w.B % div == 0:
+        return dataclasses.replace(w, B=w.B // div)
+    if w.Hkv % div == 0:
+        return dataclasses.replace(w, Hq=w.Hq // div, Hkv=w.Hkv // div)
+    raise ValueError(f"cannot divide {w.name} by {div}")
 
 
 def kernel_label(name: str) -> str:
@@ -54,7 +91,8 @@ def kernel_label(name: str) -> str:
 
 
 def parse_launches(text: str):
-    """Per kernel (in first-seen order): launches, total ms, DRAM bytes read and written."""
+    """Per kernel (in first-seen order): launches, total ms, and DRAM bytes read and
+    written when the capture has them (None otherwise)."""
     rows = list(csv.reader(io.StringIO("\n".join(l for l in text.splitlines() if l.startswith('"')))))
     if not rows:
         raise ValueError("no CSV rows in the ncu log")
@@ -65,22 +103,15 @@ def parse_launches(text: str):
         per_launch.setdefault(r[idi], {"name": r[ki]})[r[mi]] = (float(r[vi].replace(",", "")), r[ui])
     agg = collections.OrderedDict()
     for launch in per_launch.values():
-        a = agg.setdefault(kernel_label(launch["name"]), {"n": 0, "ms": 0.0, "rd": 0.0, "wr": 0.0})
+        a = agg.setdefault(kernel_label(launch["name"]), {"n": 0, "ms": 0.0, "rd": None, "wr": None})
         a["n"] += 1
         v, u = launch["gpu__time_duration.sum"]
         a["ms"] += v * _MS[u]
         for key, tag in (("dram__bytes_read.sum", "rd"), ("dram__bytes_write.sum", "wr")):
-            v, u = launch[key]
-            a[tag] += v * _BYTES[u]
+            if key in launch:
+                v, u = launch[key]
+                a[tag] = (a[tag] or 0.0) + v * _BYTES[u]
     return agg
-
-
-def pass_bytes(agg):
-    """DRAM bytes per call of each pass: the forward's kernels, the backward's kernels."""
-    def per_call(pred):
-        return round(sum((a["rd"] + a["wr"]) / a["n"] for k, a in agg.items() if pred(k)))
-    return {"fwd": per_call(lambda k: "attn_fwd" in k or "sched_reset" in k),
-            "bwd": per_call(lambda k: "attn_bwd" in k)}
 
 
 def launch_table(workload: str, agg, note: str) -> str:
@@ -88,16 +119,16 @@ def launch_table(workload: str, agg, note: str) -> str:
     total = sum(a["ms"] for a in agg.values())
     total_ours = sum(agg[k]["ms"] for k in ours) or 1.0
     out = [f"# Launch list: {workload}", "",
-           "Command (ncu replays each launch serially with cold caches: compare shares, not absolute times):", "",
-           "```", capture_command(workload), "```", "",
-           f"Summarised by `python bench_traffic.py --workload {workload} launches.csv`.", "", note, "",
-           "| kernel | launches | total ms | share of all | share of attention kernels | ms / launch | "
-           "DRAM read MB / launch | DRAM write MB / launch |",
-           "|---|---|---|---|---|---|---|---|"]
+           "Command (time only, one pass per launch; ncu replays each launch serially with cold caches: "
+           "compare shares, not absolute times):", "",
+           "```", launches_command(workload), "```", "",
+           f"Summarised by `python bench_traffic.py launches --workload {workload} launches.csv`.", "", note, "",
+           "| kernel | launches | total ms | share of all | share of attention kernels | ms / launch |",
+           "|---|---|---|---|---|---|"]
     for k, a in agg.items():
         share_ours = f"{100 * a['ms'] / total_ours:.1f}%" if k in ours else "-"
         out.append(f"| `{k}` | {a['n']} | {a['ms']:.3f} | {100 * a['ms'] / total:.1f}% | {share_ours} | "
-                   f"{a['ms'] / a['n']:.3f} | {a['rd'] / a['n'] / 1e6:.1f} | {a['wr'] / a['n'] / 1e6:.1f} |")
+                   f"{a['ms'] / a['n']:.3f} |")
     return "\n".join(out) + "\n"
 
 
@@ -109,43 +140,138 @@ def git_revision() -> str:
         return "unknown"
 
 
-def update(workload: str, csv_text: str, profiles_dir: str, revision: str | None = None):
-    """Write the launch table and merge this workload's entry into dram_traffic.json."""
+def write_launches(workload: str, csv_text: str, profiles_dir: str, revision: str | None = None) -> str:
     agg = parse_launches(csv_text)
-    shash = bench.kernel_source_hash()
-    rev = revision or git_revision()
     w = bench.WORKLOADS[workload]
     passes = "one attn_fwd and one attn_bwd (prep + dK/dV + dQ kernels)" if "bwd" in w.passes else "one attn_fwd"
-    note = (f"Kernel sources: git revision {rev} (kernel source hash {shash}). The bench step is {passes}; "
-            "the run makes 6 of each (3 warm-up, 1 timed, 2 end-to-end); the at:: kernels are torch's "
-            "input generation and host-copy casts, outside the timed region.")
+    note = (f"Kernel sources: git revision {revision or git_revision()} (kernel source hash "
+            f"{bench.kernel_source_hash()}). The bench step is {passes}; the run makes 6 of each (3 warm-up, "
+            "2 timed, 1 end-to-end); the at:: kernels are torch's input generation and host-copy casts, "
+            "outside the timed region.")
     os.makedirs(profiles_dir, exist_ok=True)
-    with open(os.path.join(profiles_dir, f"launches_{workload}.md"), "w") as f:
+    path = os.path.join(profiles_dir, f"launches_{workload}.md")
+    with open(path, "w") as f:
         f.write(launch_table(workload, agg, note))
+    return path
+
+
+def dram_entry(workload: str, div: int, csv_texts, revision: str | None = None):
+    """Per kernel: DRAM bytes of one full-size launch (captured bytes x div) and the
+    source hash; per pass: the sum over its kernels."""
+    shash = bench.kernel_source_hash()
+    kernels = {}
+    for text in csv_texts:
+        for name, a in parse_launches(text).items():
+            if a["rd"] is None:
+                raise ValueError(f"{name}: capture has no DRAM metrics")
+            key = next((k for k, (pat, _) in KERNELS.items() if pat in name), None)
+            if key is None:
+                continue
+            kernels[key] = {"kernel": name, "captured_bytes": round((a["rd"] + a["wr"]) / a["n"]),
+                            "read_bytes_per_launch": round(a["rd"] / a["n"] * div),
+                            "write_bytes_per_launch": round(a["wr"] / a["n"] * div),
+                            "bytes_per_launch": round((a["rd"] + a["wr"]) / a["n"] * div)}
+    entry = {"div": div, "source_hash": shash, "revision": revision or git_revision(), "kernels": kernels}
+    for pas in ("fwd", "bwd"):
+        ks = [k for k, (_, p) in KERNELS.items() if p == pas]
+        if all(k in kernels for k in ks):
+            entry[pas] = {"bytes_per_launch": sum(kernels[k]["bytes_per_launch"] for k in ks), "source_hash": shash}
+    return entry
+
+
+def dram_table(workload: str, entry) -> str:
+    from io_aware_exact_26_b200 import accounting as acc
+    w = bench.WORKLOADS[workload]
+    alg = {"fwd": acc.min_bytes_fwd(w.B, w.Hq, w.Hkv, w.N, w.d), "bwd": acc.min_bytes_bwd(w.B, w.Hq, w.Hkv, w.N, w.d)}
+    rw = reduced(w, entry["div"])
+    out = [f"# DRAM traffic: {workload}", "",
+           f"Captured per kernel on the reduced case B={rw.B}, Hq={rw.Hq}, Hkv={rw.Hkv}, N={rw.N}, d={rw.d} "
+           f"(the workload's (b, kv-head) units divided by {entry['div']}), one launch each, and scaled by "
+           f"{entry['div']} to a full-size launch.  Kernel sources: git revision {entry['revision']} "
+           f"(kernel source hash {entry['source_hash']}).", "", "Commands, one per kernel:", ""]
+    for k in entry["kernels"]:
+        out += ["```", dram_command(workload, entry["div"], k), "```"]
+    out += ["", "| kernel | captured MB | read MB / full launch | write MB / full launch | total MB / full launch |",
+            "|---|---|---|---|---|"]
+    for k, e in entry["kernels"].items():
+        out.append(f"| `{e['kernel']}` | {e['captured_bytes'] / 1e6:.1f} | {e['read_bytes_per_launch'] / 1e6:.1f} | "
+                   f"{e['write_bytes_per_launch'] / 1e6:.1f} | {e['bytes_per_launch'] / 1e6:.1f} |")
+    out += ["", "| pass | DRAM MB / launch | algorithmic minimum MB | ratio |", "|---|---|---|---|"]
+    for pas in ("fwd", "bwd"):
+        if pas in entry:
+            b = entry[pas]["bytes_per_launch"]
+            out.append(f"| {pas} | {b / 1e6:.1f} | {alg[pas] / 1e6:.1f} | {b / alg[pas]:.2f} |")
+    return "\n".join(out) + "\n"
+
+
+def write_dram(workload: str, div: int, csv_texts, profiles_dir: str, revision: str | None = None):
+    entry = dram_entry(workload, div, csv_texts, revision)
     path = os.path.join(profiles_dir, "dram_traffic.json")
     try:
         with open(path) as f:
             traffic = json.load(f)
     except (OSError, ValueError):
         traffic = {}
-    per_pass = pass_bytes(agg)
-    traffic[workload] = {p: {"bytes_per_launch": b, "source_hash": shash} for p, b in per_pass.items()
-                         if b > 0 and (p == "fwd" or "bwd" in w.passes)}
+    traffic[workload] = entry
+    os.makedirs(profiles_dir, exist_ok=True)
     with open(path, "w") as f:
         json.dump(traffic, f, indent=1)
-    return traffic[workload]
+    with open(os.path.join(profiles_dir, f"dram_{workload}.md"), "w") as f:
+        f.write(dram_table(workload, entry))
+    return entry
+
+
+def run_case(workload: str, div: int, reps: int):
+    """The kernels of one bench step on the reduced case, ``reps`` times (for ncu -k/-s/-c)."""
+    import torch
+    import io_aware_exact_26_b200 as attn
+    from attn_inputs import make_inputs
+    w = reduced(bench.WORKLOADS[workload], div)
+    dev = torch.device("cuda", 0)
+    x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, qk_std=w.qk_std, vo_std=w.vo_std,
+                    boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=True)
+    ws = torch.empty(attn.attn_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.N, w.d, w.causal), dtype=torch.uint8,
+                     device=dev)
+    for _ in range(reps):
+        o, lse = attn.attn_fwd(x["q"], x["k"], x["v"], scale=w.scale, causal=w.causal)
+        attn.attn_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], scale=w.scale, causal=w.causal, workspace=ws)
+    torch.cuda.synchronize()
+    st = attn.attn_get_device_status()
+    print(json.dumps({"case": dataclasses.asdict(w), "reps": reps, "status": st}))
+    if st != 0:
+        raise SystemExit(1)
 
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("--workload", required=True, choices=sorted(bench.WORKLOADS))
-    ap.add_argument("--revision", default=None, help="git revision the capture was taken on (default: HEAD)")
-    ap.add_argument("--profiles", default=os.path.join(ROOT, "profiles"))
-    ap.add_argument("csv", help="the ncu --csv --log-file output")
+    sub = ap.add_subparsers(dest="cmd", required=True)
+    a = sub.add_parser("launches", help="launch table from a time-only ncu launch list")
+    a.add_argument("--workload", required=True, choices=sorted(bench.WORKLOADS))
+    a.add_argument("--revision", default=None)
+    a.add_argument("--profiles", default=os.path.join(ROOT, "profiles"))
+    a.add_argument("csv")
+    b = sub.add_parser("dram", help="DRAM bytes per full-size launch from per-kernel captures")
+    b.add_argument("--workload", required=True, choices=sorted(bench.WORKLOADS))
+    b.add_argument("--div", type=int, required=True)
+    b.add_argument("--revision", default=None)
+    b.add_argument("--profiles", default=os.path.join(ROOT, "profiles"))
+    b.add_argument("csv", nargs="+")
+    c = sub.add_parser("run", help="run one reduced case of the workload (the program ncu captures)")
+    c.add_argument("--workload", required=True, choices=sorted(bench.WORKLOADS))
+    c.add_argument("--div", type=int, default=1)
+    c.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
-    with open(args.csv) as f:
-        entry = update(args.workload, f.read(), args.profiles, args.revision)
-    print(json.dumps({args.workload: entry}))
+    if args.cmd == "launches":
+        with open(args.csv) as f:
+            print(write_launches(args.workload, f.read(), args.profiles, args.revision))
+    elif args.cmd == "dram":
+        texts = []
+        for p in args.csv:
+            with open(p) as f:
+                texts.append(f.read())
+        print(json.dumps({args.workload: write_dram(args.workload, args.div, texts, args.profiles, args.revision)}))
+    else:
+        run_case(args.workload, args.div, args.reps)
 
 
 if __name__ == "__main__":

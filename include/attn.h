@@ -51,7 +51,8 @@ typedef enum {
   ATTN_ERR_ALIGNMENT = -3,     /* a pointer is not 16-byte aligned */
   ATTN_ERR_LAUNCH = -4,        /* the CUDA runtime refused a launch or an attribute */
   ATTN_ERR_DEVICE_TIMEOUT = -5,/* a bounded device wait expired (see attn_get_device_status) */
-  ATTN_ERR_WORKSPACE = -6      /* backward workspace missing or too small */
+  ATTN_ERR_WORKSPACE = -6,     /* backward workspace too small (or beyond the no-alloc scratch) */
+  ATTN_ERR_ALLOC = -7          /* the library's own stream-ordered allocation failed */
 } attn_status_t;
 
 /* Forward: O and LSE for every (b, h, i).
@@ -64,16 +65,24 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
              void* stream);
 
-/* Bytes of device workspace attn_bwd needs for this shape (caller allocates;
- * contents need no initialisation).  Returns 0 for arguments attn_bwd would reject. */
+/* Bytes of device workspace attn_bwd needs for this shape (8 bytes per query row:
+ * the row's log-sum-exp in log2 units and D_i = sum_k dO_ik O_ik, both fp32; rows
+ * padded to a multiple of 128).  Contents need no initialisation.  Returns 0 for
+ * arguments attn_bwd would reject. */
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int causal);
 
 /* Backward: gradients of sum(O * dO) with respect to q, k, v.
  * Reads q, k, v, o (the forward output), lse (the forward log-sum-exp) and dO;
  * writes dq, dk, dv.  For GQA, dk and dv sum over the q-heads of each group.
  * The reduction order is fixed, so two calls on the same inputs give the same
- * bits.  `workspace` must hold attn_bwd_workspace_size(...) bytes, 16-byte
- * aligned; it is overwritten. */
+ * bits.
+ * Workspace ownership: if `workspace` is non-NULL it must hold
+ *   attn_bwd_workspace_size(...) bytes (else ATTN_ERR_WORKSPACE), 16-byte aligned
+ *   (else ATTN_ERR_ALIGNMENT); it is overwritten and stays the caller's.  If it is
+ *   NULL (`workspace_bytes` is then ignored), the library takes the workspace
+ *   with cudaMallocAsync on `stream` and releases it with cudaFreeAsync on
+ *   `stream` behind its kernels, so the call stays asynchronous; a failed
+ *   allocation returns ATTN_ERR_ALLOC with nothing launched. */
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
              const void* dO, void* dq, void* dk, void* dv,
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
@@ -90,7 +99,9 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
  *   - Shapes whose workspace (attn_bwd_workspace_size) exceeds 64 MiB
  *     (67108864 bytes) are rejected with ATTN_ERR_WORKSPACE before any launch.
  *   - The first call on each device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *     that device current); make that first call before any stream capture.  If
+ *     that lookup fails the call returns ATTN_ERR_LAUNCH and the next call
+ *     tries the lookup again.
  *   - All calls share the one array and leave their contents in it; everything
  *     that must start at zero is cleared by the call itself.  Calls that overlap
  *     on the GPU (different streams, or different host threads) race on the

@@ -107,7 +107,11 @@ def attn_bwd_workspace_size(B, Hq, Hkv, N, d, causal=False) -> int:
 
 def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale=None, causal=False,
              workspace=None, stream=None):
-    """Gradients of sum(O * dO) with respect to q, k, v; returns (dq, dk, dv)."""
+    """Gradients of sum(O * dO) with respect to q, k, v; returns (dq, dk, dv).
+
+    ``workspace``: a device tensor of at least attn_bwd_workspace_size(...) bytes, or
+    None to let the library allocate it on the stream.
+    """
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
         _check(t, n)
     _check(lse, "lse", torch.float32)
@@ -120,12 +124,12 @@ def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale=None, caus
         _check(t, n)
     if scale is None:
         scale = d ** -0.5
-    need = attn_bwd_workspace_size(B, Hq, Hkv, N, d, causal)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    # workspace=None passes NULL: the library then takes its workspace with a
+    # stream-ordered allocation (cudaMallocAsync / cudaFreeAsync on the stream).
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
                         _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
-                        _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_ptr(stream))
+                        _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream_ptr(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd")
     return dq, dk, dv

@@ -1,7 +1,8 @@
 // Host side of libattn_b200.so: the extern "C" entry points declared in
 // include/attn.h.  Validates arguments, encodes the TMA tensor maps, picks the
-// kernel instance and launches it on the caller's stream.  No allocation, no
-// synchronisation on the launch path.
+// kernel instance and launches it on the caller's stream.  No synchronisation on
+// the launch path; the only allocation is attn_bwd's stream-ordered workspace when
+// the caller passes none.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -120,7 +121,7 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   p.N = N;
   p.G = Hq / Hkv;
   p.n_qtiles = (N + 127) / 128;
-  p.c = scale * 1.4426950408889634f;
+  p.c = attn::folded_scale(scale);
   p.causal = causal;
   const int units = B * Hkv * ((p.G * p.n_qtiles + 1) / 2);
   const int grid = units < di.sms ? units : di.sms;
@@ -181,7 +182,7 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   p.G = Hq / Hkv;
   p.nt = nt;
   p.causal = causal;
-  p.c = scale * 1.4426950408889634f;
+  p.c = folded_scale(scale);
   p.scale = scale;
   // dK, dV: one item per (b, kv-head, key tile)
   p.npair = (nt + 1) / 2;
@@ -213,20 +214,30 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 static constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(64) << 20;   // 64 MiB
 static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
 
-// Device address of g_bwd_scratch on the current device, looked up once per device
-// with that device current.  In host code the array's name is only a host-side
-// stand-in, so kernels must be given this address instead.  Returns nullptr if
-// the lookup failed.
+// Device address of g_bwd_scratch on the current device, looked up with that device
+// current and cached once the lookup succeeds.  In host code the array's name is
+// only a host-side stand-in, so kernels must be given this address instead.
+// Returns nullptr if the lookup failed (e.g. tried during a stream capture); a
+// later call tries again.
 static void* noalloc_scratch_on_current_device() {
-  static std::once_flag once[64];
-  static void* addr[64];
+  static std::atomic<void*> addr[64];
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::call_once(once[dev], [dev] {
+  void* a = addr[dev].load(std::memory_order_acquire);
+  if (a) return a;
+  std::lock_guard<std::mutex> lock(mu);
+  a = addr[dev].load(std::memory_order_relaxed);
+  if (!a) {
     void* p = nullptr;
-    addr[dev] = cudaGetSymbolAddress(&p, g_bwd_scratch) == cudaSuccess ? p : nullptr;
-  });
-  return addr[dev];
+    if (cudaGetSymbolAddress(&p, g_bwd_scratch) == cudaSuccess && p) {
+      a = p;
+      addr[dev].store(p, std::memory_order_release);
+    } else {
+      (void)cudaGetLastError();
+    }
+  }
+  return a;
 }
 
 extern "C" {
@@ -260,12 +271,27 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return ATTN_ERR_ALIGNMENT;
   const size_t need = attn::bwd_workspace_bytes(B, Hq, Hkv, N, d);
-  if (need > 0 && (!workspace || workspace_bytes < need)) return ATTN_ERR_WORKSPACE;
+  if (workspace && workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   if (workspace && !aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
   DeviceInfo* di = nullptr;
   if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
-  return attn::launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, workspace,
-                          static_cast<cudaStream_t>(stream), di->sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // No caller workspace: a stream-ordered allocation, freed on the same stream right
+  // behind the kernels that use it (the memory returns to the device's pool once they end).
+  void* ws = workspace;
+  if (!ws) {
+    if (cudaMallocAsync(&ws, need, s) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return ATTN_ERR_ALLOC;
+    }
+  }
+  const int st2 = attn::launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, ws, s,
+                                   di->sms);
+  if (!workspace && cudaFreeAsync(ws, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return st2 != ATTN_OK ? st2 : ATTN_ERR_ALLOC;
+  }
+  return st2;
 }
 
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -324,7 +350,8 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case ATTN_ERR_LAUNCH: return "CUDA launch or attribute error";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
-    case ATTN_ERR_WORKSPACE: return "backward workspace missing or too small";
+    case ATTN_ERR_WORKSPACE: return "backward workspace too small";
+    case ATTN_ERR_ALLOC: return "stream-ordered allocation of the backward workspace failed";
     default: return "unknown status";
   }
 }

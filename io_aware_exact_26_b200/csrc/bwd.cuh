@@ -124,19 +124,18 @@ struct BwdParams {
 };
 
 // Exps of one 16-column slice of a score tile held by this thread: p = 2^(s c - l).
-// Masked columns (only on diagonal / ragged tiles) get s = -inf first, so p = 0
-// (or 2^-126.5 on the FMA-pipe path); the exp loop itself has no branch.
+// Masked columns (only on diagonal / ragged tiles) get an exponent argument of -inf
+// after scaling, so p = 0 for any c >= 0 (2^-126.5 on the FMA-pipe path).
 __device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const float (&lv)[16], float c, bool masked,
                                           int col0, int lo, int hi, float* pf) {
-  if (masked) {
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-      if (col0 + k < lo || col0 + k > hi) sr[k] = 0xff800000u;
-  }
 #pragma unroll
   for (int k = 0; k < 16; k += 2) {
-    const float x0 = fmaf(__uint_as_float(sr[k]), c, -lv[k]);
-    const float x1 = fmaf(__uint_as_float(sr[k + 1]), c, -lv[k + 1]);
+    float x0 = fmaf(__uint_as_float(sr[k]), c, -lv[k]);
+    float x1 = fmaf(__uint_as_float(sr[k + 1]), c, -lv[k + 1]);
+    if (masked) {
+      if (col0 + k < lo || col0 + k > hi) x0 = -INFINITY;
+      if (col0 + k + 1 < lo || col0 + k + 1 > hi) x1 = -INFINITY;
+    }
     if ((k & 6) == 6) {
       exp2_fma_pair(x0, x1, pf[k], pf[k + 1]);   // one pair in four on the FMA pipe
     } else {

@@ -16,6 +16,16 @@ namespace attn {
 
 constexpr float kRescaleTau = 8.0f;
 
+// Folded scale c = scale * log2(e), floored at 1e-30 so that a masked score (-inf)
+// times c stays -inf (with c = 0 it would be NaN).  The floor changes nothing else:
+// for any c <= 1e-30 every finite exponent argument s*c - m rounds to the same
+// fp32 value as with the exact c (|s| is far below 1e20 for bf16 inputs of this
+// size), so scale = 0 still gives uniform attention over the visible keys.
+__host__ __device__ inline float folded_scale(float scale) {
+  const float c = scale * 1.4426950408889634f;
+  return c > 1e-30f ? c : 1e-30f;
+}
+
 struct FwdParams {
   void* o;
   float* lse;

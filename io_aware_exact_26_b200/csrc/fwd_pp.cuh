@@ -388,7 +388,9 @@ __global__ void __launch_bounds__(576, 1)
         if (lane == 0) mbar_arrive(&sh.xbar[x][xp]);
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.xbar[x][xp], (g >> 1) & 1));
         if (!ok) break;
-        const float m_tile = fmaxf(sh.xmax[x][xp][0][row], sh.xmax[x][xp][1][row]) * c;
+        // tile max in log2 units; a row whose keys in this tile are all masked keeps -inf
+        const float mx = fmaxf(sh.xmax[x][xp][0][row], sh.xmax[x][xp][1][row]);
+        const float m_tile = mx == -INFINITY ? -INFINITY : mx * c;
         float alpha = 1.f;
         const bool need = (m_used == -INFINITY) || (m_tile > m_used + kRescaleTau);
         if (need) {
@@ -417,8 +419,11 @@ __global__ void __launch_bounds__(576, 1)
             tmem_st16(o_base + q4 * 16, o);
           }
         }
-        // pass 2: exponentiate, P (bf16) over the columns already read
-        const uint64_t nm2 = f2pack(-m_used, -m_used);
+        // pass 2: exponentiate, P (bf16) over the columns already read.  Masked columns
+        // hold -inf, and c > 0 (the host floors it at 1e-30), so their exponent argument
+        // is -inf and p = 0; the base is 0 while the row has seen no visible key.
+        const float mb = m_used == -INFINITY ? 0.f : m_used;
+        const uint64_t nm2 = f2pack(-mb, -mb);
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[16];

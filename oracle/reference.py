@@ -5,7 +5,7 @@ Definition followed (page "attention çš„æ˜¾å­˜çº¿æ€§åŒ–", Â§ä¸€, and page "æ³¨æ„
 The row softmax subtracts the row maximum first (same page 1, Â§1.1.8 formula):
 P_ij = exp(S_ij - m_i) / sum_j exp(S_ij - m_i).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * ``scale`` is an explicit argument; the intended value is 1/sqrt(d).
 * causal: query i sees keys j <= i (equal query and key lengths).
 * GQA (page "attn-efficient", table of the three families, row â‘¢): q-head h uses
@@ -72,22 +72,29 @@ def ref_fwd(q, k, v, scale, causal, block=1024):
     return o, lse
 
 
+def grad_rows(qh, kh, vh, doh, scale, causal, r):
+    """The part of the one-head gradient that comes from the query rows ``r``:
+    (dQ[r], that block's terms of dK, that block's terms of dV), fp64."""
+    p, _, _ = _softmax_rows(_scores(qh, kh, scale, causal, r))
+    o = p @ vh
+    dd = (doh[r] * o).sum(axis=1)              # D_i = sum_k dO_ik O_ik
+    dp = doh[r] @ vh.T                          # dP = dO V^T
+    ds = p * (dp - dd[:, None])                 # dS = P * (dP - D)
+    return scale * (ds @ kh), scale * (ds.T @ qh[r]), p.T @ doh[r]
+
+
 def grad_head(qh, kh, vh, doh, scale, causal, block=1024):
-    """Gradients of sum(O * dO) for one q-head against its kv-head: (dQ, dK, dV), fp64."""
+    """Gradients of sum(O * dO) for one q-head against its kv-head: (dQ, dK, dV), fp64.
+    dK and dV are sums over query rows, taken one row block at a time."""
     n = qh.shape[0]
     dq = np.empty_like(qh)
     dk = np.zeros_like(kh)
     dv = np.zeros_like(vh)
     for a in range(0, n, block):
         r = np.arange(a, min(n, a + block))
-        p, _, _ = _softmax_rows(_scores(qh, kh, scale, causal, r))
-        o = p @ vh
-        dd = (doh[r] * o).sum(axis=1)              # D_i = sum_k dO_ik O_ik
-        dp = doh[r] @ vh.T                          # dP = dO V^T
-        ds = p * (dp - dd[:, None])                 # dS = P * (dP - D)
-        dq[r] = scale * (ds @ kh)
-        dk += scale * (ds.T @ qh[r])
-        dv += p.T @ doh[r]
+        dq[r], dkr, dvr = grad_rows(qh, kh, vh, doh, scale, causal, r)
+        dk += dkr
+        dv += dvr
     return dq, dk, dv
 
 

@@ -11,7 +11,15 @@ Gradients, per tensor: max |d| <= 2e-2 * max(1, max |ref|) (the stated gradient 
   dQ of rows 1-2 of a head lands a few percent off in relative terms (about 8e-3
   absolute for |dQ| ~ 0.1), which dominates a sampled relative RMS.
 All of these reduce to the plain 1e-2 / 5e-3 / 1e-3 / 2e-2 bounds wherever values are O(1).
+
+With ATTN_PARITY_LOG=<file> every check appends its raw figures (max |err|, the
+bound it was held to, relative RMS) as one JSON line, and
+``python -m tests.parity <file>`` turns such a log into a markdown table.
 """
+import json
+import os
+import sys
+
 import numpy as np
 import torch
 
@@ -37,18 +45,31 @@ def rel_rms(got, ref):
     return float(np.sqrt(np.mean((got - ref) ** 2)) / max(den, 1e-30))
 
 
+def _record(kind, what, err, bound_text, rr, ref):
+    path = os.environ.get("ATTN_PARITY_LOG")
+    if not path:
+        return
+    rec = {"kind": kind, "what": what, "max_abs_err": float(err.max()) if err.size else 0.0,
+           "bound": bound_text, "rel_rms": rr, "max_abs_ref": float(np.abs(ref).max()) if ref.size else 0.0,
+           "n": int(err.size)}
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
 def check_o(got, ref, what="O"):
     got = np.asarray(got, np.float64)
     err = np.abs(got - ref)
     bound = O_ATOL + half_ulp_bf16(ref)
+    rr = rel_rms(got, ref)
+    _record("O", what, err, f"1e-2 + half ulp (max {bound.max():.3g})", rr, ref)
     worst = np.unravel_index(np.argmax(err - bound), err.shape)
     assert np.all(err <= bound), f"{what}: max |err| {err.max():.3g}, worst at {worst}: got {got[worst]} ref {ref[worst]}"
-    rr = rel_rms(got, ref)
     assert rr <= O_RRMS, f"{what}: relative RMS {rr:.3g}"
 
 
-def check_lse(got, ref):
+def check_lse(got, ref, what="LSE"):
     err = np.abs(np.asarray(got, np.float64) - ref)
+    _record("LSE", what, err, f"{LSE_ATOL:g}", None, ref)
     assert err.max() <= LSE_ATOL, f"LSE: max |err| {err.max():.3g} at {np.unravel_index(np.argmax(err), err.shape)}"
 
 
@@ -56,7 +77,27 @@ def check_grad(got, ref, what):
     got = np.asarray(got, np.float64)
     err = np.abs(got - ref)
     bound = G_REL * max(1.0, float(np.abs(ref).max()))
+    rr = rel_rms(got, ref)
+    _record("grad", what, err, f"{bound:.3g}", rr, ref)
     worst = np.unravel_index(np.argmax(err), err.shape)
     assert err.max() <= bound, f"{what}: max |err| {err.max():.3g} > {bound:.3g} at {worst}: got {got[worst]} ref {ref[worst]}"
-    rr = rel_rms(got, ref)
     assert rr <= G_RRMS, f"{what}: relative RMS {rr:.3g}"
+
+
+def render_report(lines):
+    """Markdown table of a parity log (one JSON object per line)."""
+    out = ["| check | tensor | elements | max abs ref | max abs err | bound on abs err | relative RMS |",
+           "|---|---|---|---|---|---|---|"]
+    for ln in lines:
+        if not ln.strip():
+            continue
+        r = json.loads(ln)
+        rr = "-" if r["rel_rms"] is None else f"{r['rel_rms']:.2e}"
+        out.append(f"| {r['what']} | {r['kind']} | {r['n']} | {r['max_abs_ref']:.3g} | {r['max_abs_err']:.3g} | "
+                   f"{r['bound']} | {rr} |")
+    return "\n".join(out) + "\n"
+
+
+if __name__ == "__main__":
+    with open(sys.argv[1]) as f:
+        sys.stdout.write(render_report(f.readlines()))

@@ -6,6 +6,8 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
+import pytest  # noqa: E402
+
 import bench  # noqa: E402
 import bench_traffic  # noqa: E402
 
@@ -39,6 +41,15 @@ def sample_csv():
     return "\n".join(lines)
 
 
+def time_only_csv():
+    lines = ["==PROF== Connected to process 1", HDR]
+    for i, (name, ns) in enumerate([("attn::sched_reset_kernel(int)", "2,000"),
+                                    ("void attn::attn_fwd_pp_kernel<128>(CUtensorMap, attn::FwdParams)", "7,000,000"),
+                                    ("void attn::attn_bwd_kv_kernel<128>(CUtensorMap)", "12,000,000")]):
+        lines.append(row(i, name, "gpu__time_duration.sum", "nsecond", ns))
+    return "\n".join(lines)
+
+
 def test_launches_are_grouped_per_kernel_with_units_converted():
     agg = bench_traffic.parse_launches(sample_csv())
     assert list(agg) == ["at::vectorized_elementwise_kernel<4>", "attn::sched_reset_kernel",
@@ -49,28 +60,52 @@ def test_launches_are_grouped_per_kernel_with_units_converted():
     assert fwd["rd"] == 400e6 + 0.6e9 and fwd["wr"] == 200e6
 
 
-def test_per_pass_bytes_are_per_call_sums_of_the_pass_kernels():
-    b = bench_traffic.pass_bytes(bench_traffic.parse_launches(sample_csv()))
-    assert b["fwd"] == round((400e6 + 600e6 + 200e6) / 2)          # reset kernels move nothing
-    assert b["bwd"] == round(275e6 + 770e6 + 650e6)
+def test_time_only_launch_lists_have_no_dram_figures(tmp_path):
+    agg = bench_traffic.parse_launches(time_only_csv())
+    assert all(a["rd"] is None and a["wr"] is None for a in agg.values())
+    path = bench_traffic.write_launches("long_causal_b1_h32_n32768_d128", time_only_csv(), str(tmp_path), "abc1234")
+    md = open(path).read()
+    assert "abc1234" in md and "--clock-control none" in md and "gpu__time_duration.sum --clock" in md
+    assert "dram__" not in md    # the full-size capture collects time only
 
 
-def test_entries_are_stamped_and_read_back_only_for_the_same_sources(tmp_path, monkeypatch):
-    entry = bench_traffic.update("gpt2_medium_b64_h16_n1024_d64", sample_csv(), str(tmp_path), revision="abc1234")
+def test_dram_commands_capture_one_kernel_one_launch():
+    for k in bench_traffic.KERNELS:
+        cmd = bench_traffic.dram_command("long_causal_b1_h32_n32768_d128", 4, k)
+        assert " -k regex:" in cmd and " -c 1 " in cmd and "--clock-control none" in cmd and "--div 4" in cmd
+
+
+def test_reduced_cases_divide_the_independent_units():
+    w = bench.WORKLOADS["long_causal_b1_h32_n32768_d128"]
+    r = bench_traffic.reduced(w, 4)
+    assert (r.B, r.Hq, r.Hkv, r.N, r.d) == (1, 8, 8, 32768, 128)
+    g = bench_traffic.reduced(bench.WORKLOADS["gqa_causal_b4_hq32_hkv8_n8192_d128"], 4)
+    assert (g.B, g.Hq, g.Hkv) == (1, 32, 8)
+    # still larger than L2 per input tensor set
+    assert 3 * r.B * r.Hq * r.N * r.d * 2 > 126e6
+
+
+def test_dram_entries_scale_to_full_launches_and_are_stamped(tmp_path, monkeypatch):
+    texts = [sample_csv()]
+    entry = bench_traffic.write_dram("long_causal_b1_h32_n32768_d128", 4, texts, str(tmp_path), revision="abc1234")
+    k = entry["kernels"]
+    assert k["fwd"]["bytes_per_launch"] == round((400e6 + 600e6 + 200e6) / 2 * 4)
+    assert k["bwd_kv"]["bytes_per_launch"] == round(770e6 * 4)
+    assert entry["bwd"]["bytes_per_launch"] == sum(k[x]["bytes_per_launch"] for x in ("bwd_prep", "bwd_kv", "bwd_q"))
     assert entry["fwd"]["source_hash"] == bench.kernel_source_hash()
-    md = (tmp_path / "launches_gpt2_medium_b64_h16_n1024_d64.md").read_text()
-    assert "abc1234" in md and "--clock-control none" in md and "`attn::attn_bwd_kv_kernel<64>`" in md
+    md = (tmp_path / "dram_long_causal_b1_h32_n32768_d128.md").read_text()
+    assert "abc1234" in md and "-k regex:attn_bwd_kv" in md
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "dram_traffic.json"))
-    assert bench.measured_traffic("gpt2_medium_b64_h16_n1024_d64", "bwd") == entry["bwd"]["bytes_per_launch"]
+    assert bench.measured_traffic("long_causal_b1_h32_n32768_d128", "bwd") == entry["bwd"]["bytes_per_launch"]
     data = json.loads((tmp_path / "dram_traffic.json").read_text())
-    data["gpt2_medium_b64_h16_n1024_d64"]["bwd"]["source_hash"] = "0" * 16    # kernels changed since
+    data["long_causal_b1_h32_n32768_d128"]["bwd"]["source_hash"] = "0" * 16    # kernels changed since
     (tmp_path / "dram_traffic.json").write_text(json.dumps(data))
-    assert bench.measured_traffic("gpt2_medium_b64_h16_n1024_d64", "bwd") is None
+    assert bench.measured_traffic("long_causal_b1_h32_n32768_d128", "bwd") is None
 
 
-def test_forward_only_workloads_get_no_backward_entry(tmp_path):
-    entry = bench_traffic.update("causal_b8_h16_n4096_d128", sample_csv(), str(tmp_path), revision="abc1234")
-    assert set(entry) == {"fwd"}
+def test_time_only_captures_are_refused_as_dram_evidence():
+    with pytest.raises(ValueError):
+        bench_traffic.dram_entry("long_causal_b1_h32_n32768_d128", 4, [time_only_csv()])
 
 
 def test_source_fingerprint_ignores_comments_and_layout_but_not_code():

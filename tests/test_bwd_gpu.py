@@ -62,3 +62,37 @@ def test_bwd_is_bitwise_deterministic(attn):
         torch.cuda.synchronize()
         for a, b in zip(g1, g2):
             assert torch.equal(a, b)
+
+
+def test_bwd_null_workspace_through_c_abi(attn):
+    """workspace = NULL: the library allocates on the stream; same bits as a caller workspace."""
+    import ctypes
+    B, Hq, Hkv, N, d = 1, 4, 2, 700, 128
+    x = make_inputs(B, Hq, Hkv, N, d, seed=77)
+    ins, ref_g, scale = run_fwd_bwd(attn, x, d, True)
+    q, k, v, do, o, lse = ins
+    outs = [torch.full_like(t, float("nan")) for t in (q, k, v)]
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = attn.lib().attn_bwd(P(q), P(k), P(v), P(o), P(lse), P(do), P(outs[0]), P(outs[1]), P(outs[2]),
+                             B, Hq, Hkv, N, d, scale, 1, ctypes.c_void_p(0), ctypes.c_size_t(0),
+                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert attn.attn_get_device_status() == 0
+    for a, b in zip(outs, ref_g):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_scale_zero_is_uniform_attention(attn, causal):
+    """scale = 0: every visible key gets the same weight (no NaN from masked scores)."""
+    B, Hq, Hkv, N, d = 1, 2, 1, 200, 64
+    x = make_inputs(B, Hq, Hkv, N, d, seed=91)
+    (q, k, v, do, o, lse), grads, _ = run_fwd_bwd(attn, x, d, causal, scale=0.0)
+    from tests.parity import check_lse, check_o
+    o_ref, lse_ref = ref.ref_fwd(to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"]), 0.0, causal)
+    check_o(f64(o), o_ref)
+    check_lse(f64(lse), lse_ref)
+    g_ref = ref.ref_bwd(to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"]), to_f64(x["do"]), 0.0, causal)
+    for g, r, name in zip(grads, g_ref, ("dQ", "dK", "dV")):
+        check_grad(f64(g), r, name)

@@ -61,7 +61,7 @@ def test_workload_forward(attn, name):
         rows = np.arange(w.N) if w.N <= 1024 else sample_rows(w.N, 100 * b + h)
         o_ref, lse_ref = ref.attend_head(qh, kh, vh, w.scale, w.causal, rows=rows)
         check_o(f64(o[b, h])[rows], o_ref, what=f"{name} O[b={b},h={h}]")
-        check_lse(f64(lse[b, h])[rows], lse_ref)
+        check_lse(f64(lse[b, h])[rows], lse_ref, what=f"{name} LSE[b={b},h={h}]")
 
 
 @pytest.mark.parametrize("name", [n for n, w in WORKLOADS.items() if "bwd" in w.passes])
