@@ -50,6 +50,15 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 DRAM_METRICS = "dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum"
+# pipe utilisation read in the same one-kernel capture
+PIPE_METRICS = ("sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active,"
+                "sm__inst_executed_pipe_xu.avg.pct_of_peak_sustained_active,"
+                "smsp__issue_active.avg.pct_of_peak_sustained_active,"
+                "sm__cycles_elapsed.avg.per_second")
+PIPE_LABELS = {"sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active": "tensor pipe active, % of active cycles",
+               "sm__inst_executed_pipe_xu.avg.pct_of_peak_sustained_active": "XU (MUFU) instructions, % of peak",
+               "smsp__issue_active.avg.pct_of_peak_sustained_active": "issue slots used, %",
+               "sm__cycles_elapsed.avg.per_second": "SM clock during the capture (cycles/s)"}
 # kernel name pattern for -k, per kernel of the path, and the pass it belongs to
 KERNELS = {"fwd": ("attn_fwd_pp", "fwd"), "bwd_prep": ("attn_bwd_prep", "bwd"),
            "bwd_kv": ("attn_bwd_kv", "bwd"), "bwd_q": ("attn_bwd_q", "bwd")}
@@ -70,8 +79,8 @@ def launches_command(workload: str) -> str:
 def dram_command(workload: str, div: int, kernel: str) -> str:
     run = f"python bench_traffic.py run --workload {workload} --div {div}"
     pat = KERNELS[kernel][0]
-    return (f"{run} > plain.log 2>&1 && \\\nncu --metrics {DRAM_METRICS} --clock-control none -k regex:{pat} "
-            f"-s 1 -c 1 --csv --log-file dram_{kernel}.csv {run}")
+    return (f"{run} > plain.log 2>&1 && \\\nncu --metrics {DRAM_METRICS},{PIPE_METRICS} --clock-control none "
+            f"-k regex:{pat} -s 1 -c 1 --csv --log-file dram_{kernel}.csv {run}")
 
 
 def reduced(w, div: int):
@@ -103,8 +112,11 @@ def parse_launches(text: str):
         per_launch.setdefault(r[idi], {"name": r[ki]})[r[mi]] = (float(r[vi].replace(",", "")), r[ui])
     agg = collections.OrderedDict()
     for launch in per_launch.values():
-        a = agg.setdefault(kernel_label(launch["name"]), {"n": 0, "ms": 0.0, "rd": None, "wr": None})
+        a = agg.setdefault(kernel_label(launch["name"]), {"n": 0, "ms": 0.0, "rd": None, "wr": None, "pipes": {}})
         a["n"] += 1
+        for m in PIPE_LABELS:
+            if m in launch:
+                a["pipes"][m] = launch[m][0]
         v, u = launch["gpu__time_duration.sum"]
         a["ms"] += v * _MS[u]
         for key, tag in (("dram__bytes_read.sum", "rd"), ("dram__bytes_write.sum", "wr")):
@@ -168,6 +180,7 @@ def dram_entry(workload: str, div: int, csv_texts, revision: str | None = None):
             if key is None:
                 continue
             kernels[key] = {"kernel": name, "captured_bytes": round((a["rd"] + a["wr"]) / a["n"]),
+                            "captured_ms": a["ms"] / a["n"], "pipes": a["pipes"],
                             "read_bytes_per_launch": round(a["rd"] / a["n"] * div),
                             "write_bytes_per_launch": round(a["wr"] / a["n"] * div),
                             "bytes_per_launch": round((a["rd"] + a["wr"]) / a["n"] * div)}
@@ -196,6 +209,19 @@ def dram_table(workload: str, entry) -> str:
     for k, e in entry["kernels"].items():
         out.append(f"| `{e['kernel']}` | {e['captured_bytes'] / 1e6:.1f} | {e['read_bytes_per_launch'] / 1e6:.1f} | "
                    f"{e['write_bytes_per_launch'] / 1e6:.1f} | {e['bytes_per_launch'] / 1e6:.1f} |")
+    pipes = [m for m in PIPE_LABELS if any(m in e["pipes"] for e in entry["kernels"].values())]
+    if pipes:
+        out += ["", "Pipe counters of the same captures (reduced case, one launch, serialised):", "",
+                "| metric | " + " | ".join(f"`{e['kernel']}`" for e in entry["kernels"].values()) + " |",
+                "|---|" + "---|" * len(entry["kernels"])]
+        out.append("| duration under ncu (ms) | " + " | ".join(f"{e['captured_ms']:.3f}"
+                                                           for e in entry["kernels"].values()) + " |")
+        for m in pipes:
+            vals = []
+            for e in entry["kernels"].values():
+                v = e["pipes"].get(m)
+                vals.append("-" if v is None else (f"{v / 1e9:.3f} GHz" if m.endswith("per_second") else f"{v:.1f}"))
+            out.append(f"| {PIPE_LABELS[m]} | " + " | ".join(vals) + " |")
     out += ["", "| pass | DRAM MB / launch | algorithmic minimum MB | ratio |", "|---|---|---|---|"]
     for pas in ("fwd", "bwd"):
         if pas in entry:

@@ -9,6 +9,9 @@
  *
  * Layout: q, o, dO, dq are [B][Hq][N][d]; k, v, dk, dv are [B][Hkv][N][d];
  * lse is [B][Hq][N]; all double, row-major.  Causal: query i sees keys j <= i.
+ * Local window (page "attn-efficient", sliding-window row of the family table):
+ * query i sees keys j with i - wl <= j <= i + wr; wl or wr < 0 means no limit on
+ * that side; intersected with the causal rule when causal != 0.
  * q-head h reads kv-head h / (Hq / Hkv).
  */
 #include <math.h>
@@ -20,24 +23,34 @@ static long double score(const double* qi, const double* kj, int d, long double 
     return scale * s;
 }
 
+static int sees(int i, int j, int causal, int wl, int wr) {
+    if (causal && j > i) return 0;
+    if (wl >= 0 && j < i - wl) return 0;
+    if (wr >= 0 && j > i + wr) return 0;
+    return 1;
+}
+
 /* Fills p[0..N) with the softmax row of query i (masked keys get 0); returns LSE. */
 static long double prob_row(const double* q, const double* k, int N, int d, int i,
-                            long double scale, int causal, long double* p) {
-    int last = causal ? i : N - 1;
+                            long double scale, int causal, int wl, int wr, long double* p) {
     long double m = -INFINITY;
-    for (int j = 0; j <= last; ++j) {
+    for (int j = 0; j < N; ++j) {
+        if (!sees(i, j, causal, wl, wr)) continue;
         p[j] = score(q + (size_t)i * d, k + (size_t)j * d, d, scale);
         if (p[j] > m) m = p[j];
     }
     long double l = 0.0L;
-    for (int j = 0; j <= last; ++j) { p[j] = expl(p[j] - m); l += p[j]; }
-    for (int j = 0; j <= last; ++j) p[j] /= l;
-    for (int j = last + 1; j < N; ++j) p[j] = 0.0L;
+    for (int j = 0; j < N; ++j) {
+        if (!sees(i, j, causal, wl, wr)) continue;
+        p[j] = expl(p[j] - m);
+        l += p[j];
+    }
+    for (int j = 0; j < N; ++j) p[j] = sees(i, j, causal, wl, wr) ? p[j] / l : 0.0L;
     return m + logl(l);
 }
 
 int brute_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
-              int B, int Hq, int Hkv, int N, int d, double scale, int causal) {
+              int B, int Hq, int Hkv, int N, int d, double scale, int causal, int wl, int wr) {
     if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1 || Hq % Hkv) return -1;
     int G = Hq / Hkv;
     long double* p = (long double*)malloc(sizeof(long double) * (size_t)N);
@@ -48,7 +61,7 @@ int brute_fwd(const double* q, const double* k, const double* v, double* o, doub
             size_t koff = ((size_t)b * Hkv + h / G) * N * d;
             for (int i = 0; i < N; ++i) {
                 lse[((size_t)b * Hq + h) * N + i] =
-                    (double)prob_row(q + qoff, k + koff, N, d, i, scale, causal, p);
+                    (double)prob_row(q + qoff, k + koff, N, d, i, scale, causal, wl, wr, p);
                 for (int c = 0; c < d; ++c) {
                     long double acc = 0.0L;
                     for (int j = 0; j < N; ++j) acc += p[j] * (long double)v[koff + (size_t)j * d + c];
@@ -62,7 +75,7 @@ int brute_fwd(const double* q, const double* k, const double* v, double* o, doub
 
 int brute_bwd(const double* q, const double* k, const double* v, const double* dO,
               double* dq, double* dk, double* dv,
-              int B, int Hq, int Hkv, int N, int d, double scale, int causal) {
+              int B, int Hq, int Hkv, int N, int d, double scale, int causal, int wl, int wr) {
     if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1 || Hq % Hkv) return -1;
     int G = Hq / Hkv;
     long double* p = (long double*)malloc(sizeof(long double) * (size_t)N);
@@ -76,7 +89,7 @@ int brute_bwd(const double* q, const double* k, const double* v, const double* d
             size_t koff = ((size_t)b * Hkv + h / G) * N * d;
             for (int i = 0; i < N; ++i) {
                 const double* doi = dO + qoff + (size_t)i * d;
-                prob_row(q + qoff, k + koff, N, d, i, scale, causal, p);
+                prob_row(q + qoff, k + koff, N, d, i, scale, causal, wl, wr, p);
                 /* D_i = sum_c dO_ic O_ic with O_i = sum_j p_j V_j */
                 long double D = 0.0L;
                 for (int c = 0; c < d; ++c) {

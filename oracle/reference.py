@@ -8,6 +8,13 @@ P_ij = exp(S_ij - m_i) / sum_j exp(S_ij - m_i).
 Readings where the pages are silent:
 * ``scale`` is an explicit argument; the intended value is 1/sqrt(d).
 * causal: query i sees keys j <= i (equal query and key lengths).
+* local (sliding-window) attention, page "attn-efficient", efficient-attention
+  family table, sliding-window row (Longformer / Mistral: each position attends
+  only to the w positions nearest it, O(n*w)): the pages give no convention for
+  "nearest", so ``window = (left, right)`` lets query i see keys j with
+  i - left <= j <= i + right (None = no limit on that side).  Mistral's causal
+  window of w positions is (w - 1, 0); a symmetric window is (w/2, w/2).  With
+  causal=True the window is intersected with j <= i.
 * GQA (page "attn-efficient", table of the three families, row ③): q-head h uses
   kv-head h // (Hq // Hkv), contiguous groups.
 * LSE_i = m_i + ln sum_j exp(S_ij - m_i), natural log over the scaled scores,
@@ -26,12 +33,27 @@ from __future__ import annotations
 import numpy as np
 
 
-def _scores(qh, kh, scale, causal, rows):
+def visible(rows, nkeys, causal, window=None):
+    """[len(rows), nkeys] booleans: may query row i see key j (the mask of the definition)."""
+    i = np.asarray(rows)[:, None]
+    j = np.arange(nkeys)[None, :]
+    vis = np.ones((i.shape[0], nkeys), dtype=bool)
+    if causal:
+        vis &= j <= i
+    if window is not None:
+        left, right = window
+        if left is not None:
+            vis &= j >= i - left
+        if right is not None:
+            vis &= j <= i + right
+    return vis
+
+
+def _scores(qh, kh, scale, causal, rows, window=None):
     """S for the query rows ``rows`` (array of indices) of one head, fp64, masked with -inf."""
     s = scale * (qh[rows] @ kh.T)
-    if causal:
-        keys = np.arange(kh.shape[0])
-        s = np.where(keys[None, :] <= rows[:, None], s, -np.inf)
+    if causal or window is not None:
+        s = np.where(visible(rows, kh.shape[0], causal, window), s, -np.inf)
     return s
 
 
@@ -43,7 +65,7 @@ def _softmax_rows(s):
     return e / l[:, None], m, m + np.log(l)
 
 
-def attend_head(qh, kh, vh, scale, causal, rows=None, block=1024):
+def attend_head(qh, kh, vh, scale, causal, rows=None, block=1024, window=None):
     """O and LSE for the given query rows of one head (all rows when ``rows`` is None).
 
     qh: [N, d]; kh, vh: [N, d]; fp64.  Returns (O[len(rows), d], LSE[len(rows)]).
@@ -54,12 +76,12 @@ def attend_head(qh, kh, vh, scale, causal, rows=None, block=1024):
     lse = np.empty(rows.shape[0])
     for a in range(0, rows.shape[0], block):
         r = rows[a:a + block]
-        p, _, lse[a:a + block] = _softmax_rows(_scores(qh, kh, scale, causal, r))
+        p, _, lse[a:a + block] = _softmax_rows(_scores(qh, kh, scale, causal, r, window))
         o[a:a + block] = p @ vh
     return o, lse
 
 
-def ref_fwd(q, k, v, scale, causal, block=1024):
+def ref_fwd(q, k, v, scale, causal, block=1024, window=None):
     """Forward oracle.  q [B,Hq,N,d], k/v [B,Hkv,N,d] fp64 -> O [B,Hq,N,d], LSE [B,Hq,N]."""
     B, Hq, N, d = q.shape
     G = Hq // k.shape[1]
@@ -68,14 +90,14 @@ def ref_fwd(q, k, v, scale, causal, block=1024):
     for b in range(B):
         for h in range(Hq):
             o[b, h], lse[b, h] = attend_head(q[b, h], k[b, h // G], v[b, h // G], scale, causal,
-                                             block=block)
+                                             block=block, window=window)
     return o, lse
 
 
-def grad_rows(qh, kh, vh, doh, scale, causal, r):
+def grad_rows(qh, kh, vh, doh, scale, causal, r, window=None):
     """The part of the one-head gradient that comes from the query rows ``r``:
     (dQ[r], that block's terms of dK, that block's terms of dV), fp64."""
-    p, _, _ = _softmax_rows(_scores(qh, kh, scale, causal, r))
+    p, _, _ = _softmax_rows(_scores(qh, kh, scale, causal, r, window))
     o = p @ vh
     dd = (doh[r] * o).sum(axis=1)              # D_i = sum_k dO_ik O_ik
     dp = doh[r] @ vh.T                          # dP = dO V^T
@@ -83,7 +105,7 @@ def grad_rows(qh, kh, vh, doh, scale, causal, r):
     return scale * (ds @ kh), scale * (ds.T @ qh[r]), p.T @ doh[r]
 
 
-def grad_head(qh, kh, vh, doh, scale, causal, block=1024):
+def grad_head(qh, kh, vh, doh, scale, causal, block=1024, window=None):
     """Gradients of sum(O * dO) for one q-head against its kv-head: (dQ, dK, dV), fp64.
     dK and dV are sums over query rows, taken one row block at a time."""
     n = qh.shape[0]
@@ -92,13 +114,13 @@ def grad_head(qh, kh, vh, doh, scale, causal, block=1024):
     dv = np.zeros_like(vh)
     for a in range(0, n, block):
         r = np.arange(a, min(n, a + block))
-        dq[r], dkr, dvr = grad_rows(qh, kh, vh, doh, scale, causal, r)
+        dq[r], dkr, dvr = grad_rows(qh, kh, vh, doh, scale, causal, r, window)
         dk += dkr
         dv += dvr
     return dq, dk, dv
 
 
-def ref_bwd(q, k, v, do, scale, causal, block=1024):
+def ref_bwd(q, k, v, do, scale, causal, block=1024, window=None):
     """Backward oracle: (dQ [B,Hq,N,d], dK [B,Hkv,N,d], dV [B,Hkv,N,d]) in fp64."""
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
@@ -110,13 +132,13 @@ def ref_bwd(q, k, v, do, scale, causal, block=1024):
         for h in range(Hq):
             g = h // G
             dq[b, h], dkh, dvh = grad_head(q[b, h], k[b, g], v[b, g], do[b, h], scale, causal,
-                                           block=block)
+                                           block=block, window=window)
             dk[b, g] += dkh
             dv[b, g] += dvh
     return dq, dk, dv
 
 
-def online_fwd_head(qh, kh, vh, scale, causal, bounds):
+def online_fwd_head(qh, kh, vh, scale, causal, bounds, window=None):
     """The pages' blockwise online softmax for one head (used only in self-tests).
 
     Page "attention 的显存线性化" §三: for each key block j, with S_ij = Q_i K_j^T,
@@ -136,9 +158,8 @@ def online_fwd_head(qh, kh, vh, scale, causal, bounds):
     acc = np.zeros((n, dv))
     for a, b in zip(bounds[:-1], bounds[1:]):
         s = scale * (qh @ kh[a:b].T)
-        if causal:
-            keys = np.arange(a, b)
-            s = np.where(keys[None, :] <= rows[:, None], s, -np.inf)
+        if causal or window is not None:
+            s = np.where(visible(rows, kh.shape[0], causal, window)[:, a:b], s, -np.inf)
         m_new = np.maximum(m, s.max(axis=1))
         live = np.isfinite(m_new)   # rows that have seen at least one unmasked key
         alpha = np.where(live, np.exp(np.where(live, m - m_new, 0.0)), 1.0)
@@ -149,18 +170,18 @@ def online_fwd_head(qh, kh, vh, scale, causal, bounds):
     return acc / l[:, None], m + np.log(l)
 
 
-def grad_q_rows(qh, kh, vh, doh, scale, causal, rows):
+def grad_q_rows(qh, kh, vh, doh, scale, causal, rows, window=None):
     """dQ for the given query rows of one head (full key range), from the same formulas as
     ``grad_head``; used to check sampled rows of full-size problems."""
     rows = np.asarray(rows, dtype=np.int64)
-    p, _, _ = _softmax_rows(_scores(qh, kh, scale, causal, rows))
+    p, _, _ = _softmax_rows(_scores(qh, kh, scale, causal, rows, window))
     o = p @ vh
     dd = (doh[rows] * o).sum(axis=1)
     ds = p * (doh[rows] @ vh.T - dd[:, None])
     return scale * (ds @ kh)
 
 
-def grad_kv_rows(qhs, kh, vh, dohs, scale, causal, keys, block=1024):
+def grad_kv_rows(qhs, kh, vh, dohs, scale, causal, keys, block=1024, window=None):
     """dK and dV for the given key rows of one kv-head, summed over the q-heads in
     ``qhs`` / ``dohs`` (the GQA group).  Needs LSE and D of every query row, so it
     costs one full forward per q-head."""
@@ -171,7 +192,7 @@ def grad_kv_rows(qhs, kh, vh, dohs, scale, causal, keys, block=1024):
     for qh, doh in zip(qhs, dohs):
         for a in range(0, n, block):
             r = np.arange(a, min(n, a + block))
-            p_full, m, lse = _softmax_rows(_scores(qh, kh, scale, causal, r))
+            p_full, m, lse = _softmax_rows(_scores(qh, kh, scale, causal, r, window))
             o = p_full @ vh
             dd = (doh[r] * o).sum(axis=1)
             p = p_full[:, keys]                          # P[r, keys]

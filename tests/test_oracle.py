@@ -126,7 +126,7 @@ def test_finite_differences_catch_a_planted_sign_error(monkeypatch):
     q, k, v, do = rand(1, 1, 4, 3), rand(1, 1, 4, 3), rand(1, 1, 4, 3), rand(1, 1, 4, 3)
     fd = _fd_grads(ref.ref_fwd, q, k, v, do, 0.6, False)
 
-    def bad_grad_head(qh, kh, vh, doh, scale, causal, block=1024):
+    def bad_grad_head(qh, kh, vh, doh, scale, causal, block=1024, window=None):
         p, _, _ = ref._softmax_rows(ref._scores(qh, kh, scale, causal, np.arange(qh.shape[0])))
         o = p @ vh
         dd = (doh * o).sum(axis=1)
@@ -319,3 +319,89 @@ def test_sampled_gradient_rows_match_full_backward(causal):
                               rows, block=16)
     np.testing.assert_allclose(gk, dk[0, 1, rows], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(gv, dv[0, 1, rows], rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------- local (sliding-window) attention
+# Page "attn-efficient", efficient-attention family table, sliding-window row: each
+# position attends only to the w positions nearest it.  window = (left, right):
+# query i sees keys j with i - left <= j <= i + right (None = no limit).
+WINDOWS = [(2, 0), (0, 3), (3, 2), (None, 1), (1, None), (5, 5)]
+
+
+@pytest.mark.parametrize("window", WINDOWS)
+@pytest.mark.parametrize("causal", [False, True])
+def test_window_fwd_bwd_match_c_brute_force(window, causal):
+    B, Hq, Hkv, N, d = 1, 4, 2, 11, 3
+    q, k, v, do = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d), rand(B, Hq, N, d)
+    o, lse = ref.ref_fwd(q, k, v, 0.8, causal, window=window)
+    ob, lseb = obuild.brute_fwd(q, k, v, 0.8, causal, window=window)
+    np.testing.assert_allclose(o, ob, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lseb, rtol=1e-12, atol=1e-13)
+    for g, e in zip(ref.ref_bwd(q, k, v, do, 0.8, causal, window=window),
+                    obuild.brute_bwd(q, k, v, do, 0.8, causal, window=window)):
+        np.testing.assert_allclose(g, e, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("window", WINDOWS)
+def test_window_matches_torch_sdpa_with_a_band_mask(window):
+    """torch's fp64 SDPA with an explicit boolean band mask (a library routine), and autograd."""
+    B, Hq, Hkv, N, d = 2, 2, 1, 13, 4
+    q, k, v, do = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d), rand(B, Hq, N, d)
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    band = torch.ones(N, N, dtype=torch.bool)
+    if window[0] is not None:
+        band &= j >= i - window[0]
+    if window[1] is not None:
+        band &= j <= i + window[1]
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk.repeat_interleave(Hq // Hkv, dim=1), tv.repeat_interleave(Hq // Hkv, dim=1), attn_mask=band, scale=0.5)
+    o, lse = ref.ref_fwd(q, k, v, 0.5, False, window=window)
+    np.testing.assert_allclose(o, to.detach().numpy(), rtol=1e-10, atol=1e-12)
+    (to * torch.tensor(do)).sum().backward()
+    for g, e in zip(ref.ref_bwd(q, k, v, do, 0.5, False, window=window), (tq.grad, tk.grad, tv.grad)):
+        np.testing.assert_allclose(g, e.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_window_special_cases():
+    B, H, N, d = 1, 2, 17, 5
+    q, k, v = rand(B, H, N, d, scale=2.0), rand(B, H, N, d, scale=2.0), rand(B, H, N, d)
+    full = ref.ref_fwd(q, k, v, 0.7, False)
+    causal = ref.ref_fwd(q, k, v, 0.7, True)
+    for a, b in zip(ref.ref_fwd(q, k, v, 0.7, False, window=(N, N)), full):        # wider than N: no mask
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(ref.ref_fwd(q, k, v, 0.7, False, window=(None, 0)), causal):   # (None, 0) is causal
+        np.testing.assert_array_equal(a, b)
+    o, lse = ref.ref_fwd(q, k, v, 0.7, False, window=(0, 0))                      # only itself: O_i = V_i
+    np.testing.assert_allclose(o, v, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(lse, 0.7 * np.einsum("bhnd,bhnd->bhn", q, k), rtol=1e-13, atol=1e-14)
+    # left window 1, causal: row i averages V_{i-1}, V_i with weights from the two scores
+    o, _ = ref.ref_fwd(q, k, v, 0.7, True, window=(1, None))
+    s1 = 0.7 * np.einsum("bhnd,bhnd->bhn", q[:, :, 1:], k[:, :, :-1])
+    s0 = 0.7 * np.einsum("bhnd,bhnd->bhn", q[:, :, 1:], k[:, :, 1:])
+    w1 = 1 / (1 + np.exp(s0 - s1))
+    want = w1[..., None] * v[:, :, :-1] + (1 - w1[..., None]) * v[:, :, 1:]
+    np.testing.assert_allclose(o[:, :, 1:], want, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(o[:, :, 0], v[:, :, 0], rtol=1e-14)
+
+
+@pytest.mark.parametrize("window", [(3, 0), (2, 4)])
+def test_window_bwd_matches_finite_differences(window):
+    q, k, v, do = rand(1, 2, 7, 2), rand(1, 1, 7, 2), rand(1, 1, 7, 2), rand(1, 2, 7, 2)
+
+    def fwd(qq, kk, vv, scale, causal):
+        return ref.ref_fwd(qq, kk, vv, scale, causal, window=window)
+    fd = _fd_grads(fwd, q, k, v, do, 0.6, False)
+    for g, e in zip(ref.ref_bwd(q, k, v, do, 0.6, False, window=window), fd):
+        np.testing.assert_allclose(g, e, rtol=1e-7, atol=1e-8)
+
+
+@pytest.mark.parametrize("window", [(4, 0), (2, 3)])
+def test_window_blockwise_online_softmax_equals_full(window):
+    n, d = 19, 4
+    qh, kh, vh = rand(n, d, scale=2.0), rand(n, d, scale=2.0), rand(n, d)
+    o_full, lse_full = ref.attend_head(qh, kh, vh, 0.4, False, window=window)
+    o_on, lse_on = ref.online_fwd_head(qh, kh, vh, 0.4, False, [0, 3, 4, 10, 12, n], window=window)
+    np.testing.assert_allclose(o_on, o_full, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse_on, lse_full, rtol=1e-13, atol=1e-14)
