@@ -65,6 +65,19 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
              void* stream);
 
+/* Local (sliding-window) forward: as attn_fwd, but query i sees only keys j with
+ *     i - window_left <= j <= i + window_right
+ * (page "attn-efficient", sliding-window row of the efficient-attention family
+ * table: each position attends to the w positions nearest it, O(n*w) work).  A
+ * negative side means no limit on that side, so (-1, 0) is causal attention,
+ * (-1, -1) full attention, (w - 1, 0) a causal window of w keys and (w, w) a
+ * symmetric one.  Key tiles outside every row's band are skipped, so the work
+ * grows with N * (window_left + window_right + 1).  Same layouts, errors and
+ * stream behaviour as attn_fwd. */
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int Hq, int Hkv, int N, int d, float scale,
+                    int window_left, int window_right, void* stream);
+
 /* Bytes of device workspace attn_bwd needs for this shape (8 bytes per query row:
  * the row's log-sum-exp in log2 units and D_i = sum_k dO_ik O_ik, both fp32; rows
  * padded to a multiple of 128).  Contents need no initialisation.  Returns 0 for
@@ -87,6 +100,16 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              const void* dO, void* dq, void* dk, void* dv,
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of attn_fwd_window: gradients of sum(O * dO) for the same band of
+ * visible keys (window_left / window_right as in attn_fwd_window; o and lse must
+ * come from attn_fwd_window with the same window).  Workspace and stream rules
+ * are those of attn_bwd; attn_bwd_workspace_size does not depend on the mask. */
+int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dO, void* dq, void* dk, void* dv,
+                    int B, int Hq, int Hkv, int N, int d, float scale,
+                    int window_left, int window_right,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* Backward without a caller-provided workspace (no counterpart on the pages; an
  * interface convenience).  Same arguments, layouts and results as attn_bwd, minus

@@ -9,9 +9,11 @@ from .binding import (  # noqa: F401
     AttnError,
     attn_bwd,
     attn_bwd_noalloc,
+    attn_bwd_window,
     NOALLOC_SCRATCH_BYTES,
     attn_bwd_workspace_size,
     attn_fwd,
+    attn_fwd_window,
     attn_get_device_status,
     attn_selftest_timeout,
     attn_status_string,

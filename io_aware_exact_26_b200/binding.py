@@ -42,6 +42,10 @@ def lib():
     L.attn_bwd_workspace_size.restype = sz
     L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     L.attn_bwd.restype = i
+    L.attn_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    L.attn_fwd_window.restype = i
+    L.attn_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
+    L.attn_bwd_window.restype = i
     L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     L.attn_bwd_noalloc.restype = i
     L.attn_get_device_status.argtypes = [vp]
@@ -99,6 +103,58 @@ def attn_fwd(q, k, v, o=None, lse=None, *, scale=None, causal=False, stream=None
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
     return o, lse
+
+
+def _window_args(window):
+    # (left, right) with None for no limit -> the ABI's convention (negative = no limit)
+    left, right = window
+    return (-1 if left is None else int(left)), (-1 if right is None else int(right))
+
+
+def attn_fwd_window(q, k, v, o=None, lse=None, *, window, scale=None, stream=None):
+    """Local attention: query i sees keys i - left .. i + right, ``window = (left, right)``
+    (None = no limit on that side); returns (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(o, "o")
+    _check(lse, "lse", torch.float32)
+    if scale is None:
+        scale = d ** -0.5
+    wl, wr = _window_args(window)
+    st = lib().attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                               float(scale), wl, wr, _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_window")
+    return o, lse
+
+
+def attn_bwd_window(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, window, scale=None, workspace=None,
+                    stream=None):
+    """Backward of attn_fwd_window for the same ``window``; returns (dq, dk, dv)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _check(t, n)
+    _check(lse, "lse", torch.float32)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _check(t, n)
+    if scale is None:
+        scale = d ** -0.5
+    wl, wr = _window_args(window)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().attn_bwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                               _ptr(dv), B, Hq, Hkv, N, d, float(scale), wl, wr, _ptr(workspace),
+                               ctypes.c_size_t(ws_bytes), _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_window")
+    return dq, dk, dv
 
 
 def attn_bwd_workspace_size(B, Hq, Hkv, N, d, causal=False) -> int:

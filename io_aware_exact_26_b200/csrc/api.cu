@@ -86,6 +86,16 @@ int check_common(int B, int Hq, int Hkv, int N, int d, float scale, int causal) 
 }
 
 
+// Band of visible keys as the kernels take it: query i sees keys i - wl .. i + wr,
+// each side at most N (= no limit).  A negative window side means no limit.
+struct Band {
+  int wl, wr;
+};
+Band band_of_causal(int N, int causal) { return {N, causal ? 0 : N}; }
+Band band_of_window(int N, int left, int right) {
+  return {(left < 0 || left > N) ? N : left, (right < 0 || right > N) ? N : right};
+}
+
 // Work-unit counter slot for the next dynamically scheduled launch (rotates over
 // attn::kSchedSlots; concurrent launches in flight take different slots).
 int next_sched_slot() {
@@ -96,7 +106,7 @@ int next_sched_slot() {
 // Forward: two query tiles per CTA (fwd_pp.cuh).
 template <int D>
 int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-               int N, float scale, int causal, cudaStream_t stream, const DeviceInfo& di) {
+               int N, float scale, Band band, cudaStream_t stream, const DeviceInfo& di) {
   using C = attn::PpCfg<D>;
   static std::once_flag attr_once[64];
   static bool attr_ok[64];
@@ -122,7 +132,9 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   p.G = Hq / Hkv;
   p.n_qtiles = (N + 127) / 128;
   p.c = attn::folded_scale(scale);
-  p.causal = causal;
+  p.wl = band.wl;
+  p.wr = band.wr;
+  p.desc = band.wr <= band.wl;
   const int units = B * Hkv * ((p.G * p.n_qtiles + 1) / 2);
   const int grid = units < di.sms ? units : di.sms;
   p.sched_slot = next_sched_slot();
@@ -138,7 +150,7 @@ namespace attn {
 template <int D>
 static int launch_bwd_d(const void* q, const void* k, const void* v, const void* o, const float* lse,
                         const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, float scale,
-                        int causal, void* workspace, cudaStream_t stream, int sms) {
+                        int wl, int wr, void* workspace, cudaStream_t stream, int sms) {
   static std::once_flag attr_once[64];
   static bool attr_ok[64];
   int dev = 0;
@@ -181,12 +193,15 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   p.N = N;
   p.G = Hq / Hkv;
   p.nt = nt;
-  p.causal = causal;
+  p.wl = wl;
+  p.wr = wr;
+  p.pair = wr == 0 && wl >= N - 1;     // causal: every key tile sees all later query tiles
+  p.desc = wr <= wl;
   p.c = folded_scale(scale);
   p.scale = scale;
-  // dK, dV: one item per (b, kv-head, key tile)
+  // dK, dV: one item per (b, kv-head, key tile); causal: units of two key tiles
   p.npair = (nt + 1) / 2;
-  p.total_items = B * Hkv * (causal ? p.npair : nt);
+  p.total_items = B * Hkv * (p.pair ? p.npair : nt);
   int grid = p.total_items < sms ? p.total_items : sms;
   attn_bwd_kv_kernel<D><<<grid, KvCfg<D>::kThreads, KvCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
   if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
@@ -198,11 +213,11 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
 }
 
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-               void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+               void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int wl, int wr,
                void* workspace, cudaStream_t stream, int sms) {
   if (d == 64)
-    return launch_bwd_d<64>(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, stream, sms);
-  return launch_bwd_d<128>(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, scale, causal, workspace, stream, sms);
+    return launch_bwd_d<64>(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, scale, wl, wr, workspace, stream, sms);
+  return launch_bwd_d<128>(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, scale, wl, wr, workspace, stream, sms);
 }
 
 }  // namespace attn
@@ -242,8 +257,8 @@ static void* noalloc_scratch_on_current_device() {
 
 extern "C" {
 
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
-             int d, float scale, int causal, void* stream) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                    int N, int d, float scale, int causal, Band band, void* stream) {
   int st = check_common(B, Hq, Hkv, N, d, scale, causal);
   if (st != ATTN_OK) return st;
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
@@ -252,8 +267,19 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   DeviceInfo* di = nullptr;
   if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_fwd_pp<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, *di);
-  return launch_fwd_pp<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, *di);
+  if (d == 64) return launch_fwd_pp<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, band, s, *di);
+  return launch_fwd_pp<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, band, s, *di);
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+             int d, float scale, int causal, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, band_of_causal(N, causal), stream);
+}
+
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                    int N, int d, float scale, int window_left, int window_right, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, 0, band_of_window(N, window_left, window_right),
+                  stream);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int causal) {
@@ -261,9 +287,9 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int causal)
   return attn::bwd_workspace_bytes(B, Hq, Hkv, N, d);
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
-             void* workspace, size_t workspace_bytes, void* stream) {
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                    void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                    Band band, void* workspace, size_t workspace_bytes, void* stream) {
   int st = check_common(B, Hq, Hkv, N, d, scale, causal);
   if (st != ATTN_OK) return st;
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
@@ -285,13 +311,28 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
       return ATTN_ERR_ALLOC;
     }
   }
-  const int st2 = attn::launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, ws, s,
-                                   di->sms);
+  const int st2 = attn::launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, band.wl, band.wr,
+                                   ws, s, di->sms);
   if (!workspace && cudaFreeAsync(ws, s) != cudaSuccess) {
     (void)cudaGetLastError();
     return st2 != ATTN_OK ? st2 : ATTN_ERR_ALLOC;
   }
   return st2;
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, band_of_causal(N, causal),
+                  workspace, workspace_bytes, stream);
+}
+
+int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                    float scale, int window_left, int window_right, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, 0,
+                  band_of_window(N, window_left, window_right), workspace, workspace_bytes, stream);
 }
 
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,

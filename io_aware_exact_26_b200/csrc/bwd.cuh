@@ -118,24 +118,28 @@ struct BwdParams {
   int nt;           // number of 128-row tiles along N
   int npair;        // (nt + 1) / 2: key-tile pairs per KV head (causal dK/dV units)
   int total_items;
-  int causal;
+  int wl, wr;       // window: query i sees keys i - wl .. i + wr (0 <= wl, wr <= N)
+  int pair;         // causal (wl = N, wr = 0): dK/dV units are pairs of key tiles
+  int desc;         // dQ items list query tiles last-first (key ranges grow with the tile)
   float c;          // scale * log2(e)
   float scale;
 };
 
 // Exps of one 16-column slice of a score tile held by this thread: p = 2^(s c - l).
-// Masked columns (only on diagonal / ragged tiles) get an exponent argument of -inf
-// after scaling, so p = 0 for any c >= 0 (2^-126.5 on the FMA-pipe path).
+// Masked columns (only on band-edge / ragged tiles) get s = -inf first; c > 0 (the
+// host floors it at 1e-30), so p = 0 (or 2^-126.5 on the FMA-pipe path); the exp
+// loop itself has no branch.
 __device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const float (&lv)[16], float c, bool masked,
                                           int col0, int lo, int hi, float* pf) {
+  if (masked) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (col0 + k < lo || col0 + k > hi) sr[k] = 0xff800000u;
+  }
 #pragma unroll
   for (int k = 0; k < 16; k += 2) {
-    float x0 = fmaf(__uint_as_float(sr[k]), c, -lv[k]);
-    float x1 = fmaf(__uint_as_float(sr[k + 1]), c, -lv[k + 1]);
-    if (masked) {
-      if (col0 + k < lo || col0 + k > hi) x0 = -INFINITY;
-      if (col0 + k + 1 < lo || col0 + k + 1 > hi) x1 = -INFINITY;
-    }
+    const float x0 = fmaf(__uint_as_float(sr[k]), c, -lv[k]);
+    const float x1 = fmaf(__uint_as_float(sr[k + 1]), c, -lv[k + 1]);
     if ((k & 6) == 6) {
       exp2_fma_pair(x0, x1, pf[k], pf[k + 1]);   // one pair in four on the FMA pipe
     } else {
@@ -179,7 +183,8 @@ struct KvShared {
 
 // Work units of the dK/dV kernel, numbered KV head by KV head, so the CTAs running at
 // the same time stream the Q/dO of the same few head groups.
-//  - Non-causal: unit t is key tile j = t mod nt, one item.
+//  - In general unit t is key tile j = t mod nt, one item, walking its query tiles
+//    from the last one down.
 //  - Causal: unit t is the pair of key tiles (pr, nt-1-pr), two items (one for the
 //    middle tile when nt is odd). Together they see nt+1 query tiles whatever pr is,
 //    so units cost the same and the CTAs that start them together stay in step.
@@ -188,12 +193,12 @@ struct KvShared {
 //    query tile nt-1-T or T-1, so each Q/dO tile reaches L2 from HBM about twice
 //    per group instead of once per key tile.
 __device__ __forceinline__ int kv_halves(const BwdParams& p, int t) {
-  if (!p.causal) return 1;
+  if (!p.pair) return 1;
   const int pr = t % p.npair;
   return 2 * pr + 1 == p.nt ? 1 : 2;
 }
 __device__ __forceinline__ void kv_item(const BwdParams& p, int t, int hf, int& bhkv, int& j, bool& up) {
-  if (!p.causal) {
+  if (!p.pair) {
     bhkv = t / p.nt;
     j = t - bhkv * p.nt;
     up = false;
@@ -204,11 +209,14 @@ __device__ __forceinline__ void kv_item(const BwdParams& p, int t, int hf, int& 
   j = hf ? p.nt - 1 - pr : pr;
   up = hf != 0;
 }
-// s-th query tile an item visits, s in [0, nt - first)
-__device__ __forceinline__ int kv_q_tile(const BwdParams& p, int first, bool up, int s) {
-  return up ? first + s : p.nt - 1 - s;
+// Query tiles [i0, i1] that see key tile j: queries i with key - wr <= i <= key + wl.
+__device__ __forceinline__ void kv_q_range(const BwdParams& p, int j, int& i0, int& i1) {
+  const int k0 = j * 128, k1 = min(p.N - 1, k0 + 127);
+  i0 = max(0, k0 - p.wr) >> 7;
+  i1 = min(p.N - 1, k1 + p.wl) >> 7;
 }
-__device__ __forceinline__ int kv_first_q(const BwdParams& p, int j) { return p.causal ? j : 0; }
+// s-th query tile an item visits, s in [0, i1 - i0]
+__device__ __forceinline__ int kv_q_tile(int i0, int i1, bool up, int s) { return up ? i0 + s : i1 - s; }
 
 template <int D>
 __global__ void __launch_bounds__(320, 1)
@@ -270,9 +278,10 @@ __global__ void __launch_bounds__(320, 1)
         nkv = it + 1;
         const int b = bhkv / p.Hkv, hk = bhkv - b * p.Hkv;
         // Query tiles in the item's order, the G heads of the group inside.
-        const int first = kv_first_q(p, j);
-        for (int s = 0; s < p.nt - first && ok; ++s) {
-          const int i = kv_q_tile(p, first, up, s);
+        int i0, i1;
+        kv_q_range(p, j, i0, i1);
+        for (int s = 0; s <= i1 - i0 && ok; ++s) {
+          const int i = kv_q_tile(i0, i1, up, s);
           for (int h = 0; h < p.G; ++h, ++gs) {
             const int bhq = b * p.Hq + hk * p.G + h;
             const int st = gs & 1;
@@ -356,7 +365,9 @@ __global__ void __launch_bounds__(320, 1)
       kv_item(p, t, hf, bhkv, j, up);
       ok = wait(&sh.kv_full, it & 1);
       if (!ok) break;
-      const int n_steps = p.G * (p.nt - kv_first_q(p, j));
+      int i0, i1;
+      kv_q_range(p, j, i0, i1);
+      const int n_steps = p.G * (i1 - i0 + 1);
       ok = issue_st(gs) && issue_dp(gs);
       for (int u = 0; u < n_steps && ok; ++u, ++gs) {
         const int st = gs & 1;
@@ -416,17 +427,19 @@ __global__ void __launch_bounds__(320, 1)
       kv_item(p, t, hf, bhkv, j, up);
       const int key = j * 128 + r;
       const bool key_live = key < p.N;
-      const int first = kv_first_q(p, j);
-      for (int s = 0; s < p.nt - first && ok; ++s) {
-        const int i = kv_q_tile(p, first, up, s);
+      int i0, i1;
+      kv_q_range(p, j, i0, i1);
+      for (int s = 0; s <= i1 - i0 && ok; ++s) {
+        const int i = kv_q_tile(i0, i1, up, s);
         for (int h = 0; h < p.G && ok; ++h, ++gs) {
           const int st = gs & 1;
           const float* sLse = sVec + st * 256 + 64 * hb;
           const float* sDd = sLse + 128;
-          // visible query columns (relative to this warpgroup's 64) for this key row
+          // visible query columns (relative to this warpgroup's 64) for this key row:
+          // queries key - wr .. key + wl
           const int qbase = i * 128 + 64 * hb;
-          const int hi = key_live ? (p.N - 1 - qbase) : -1;
-          const int lo = p.causal ? (key - qbase) : 0;
+          const int hi = key_live ? (min(p.N - 1, key + p.wl) - qbase) : -1;
+          const int lo = key - p.wr - qbase;
           const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= 63);
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.qdo_full[st], (gs >> 1) & 1));
           if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full, gs & 1));
@@ -559,17 +572,22 @@ struct QShared {
 
 // item t -> (bh_q, query tile i).  Numbered KV head by KV head (the G query heads
 // of a group interleaved), so CTAs running at the same time share K/V in L2;
-// causal: longest rows first within a group.
+// longest rows first within a group when key ranges grow with the tile (causal).
 __device__ __forceinline__ void q_item(const BwdParams& p, int t, int& bhq, int& i) {
   const int per_group = p.G * p.nt;
   const int gk = t / per_group;                  // b * Hkv + kv-head
   const int r = t - gk * per_group;
   const int rq = r / p.G;
   const int hin = r - rq * p.G;
-  i = p.causal ? (p.nt - 1 - rq) : rq;
+  i = p.desc ? (p.nt - 1 - rq) : rq;
   bhq = (gk / p.Hkv) * p.Hq + (gk % p.Hkv) * p.G + hin;
 }
-__device__ __forceinline__ int q_n_kv(const BwdParams& p, int i) { return p.causal ? (i + 1) : p.nt; }
+// Key tiles [j0, j0 + n) that query tile i sees: keys i - wl .. i + wr.
+__device__ __forceinline__ void q_kv_range(const BwdParams& p, int i, int& j0, int& n) {
+  const int r0 = i * 128, r1 = min(p.N - 1, r0 + 127);
+  j0 = max(0, r0 - p.wl) >> 7;
+  n = (min(p.N - 1, r1 + p.wr) >> 7) - j0 + 1;
+}
 
 template <int D>
 __global__ void __launch_bounds__(352, 1)
@@ -620,7 +638,8 @@ __global__ void __launch_bounds__(352, 1)
         int bhq, i;
         q_item(p, t, bhq, i);
         const int bkv = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / p.G;
-        const int n_kv = q_n_kv(p, i);
+        int j0, n_kv;
+        q_kv_range(p, i, j0, n_kv);
         if (it >= 1) ok = mbar_wait(&sh.qdo_empty, (it - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&sh.qdo_full, 2 * C::kTile);
@@ -635,7 +654,7 @@ __global__ void __launch_bounds__(352, 1)
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, j * 128, bkv);
+            tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, (j0 + j) * 128, bkv);
           nk = g + 1;
         }
         gj += n_kv;
@@ -655,14 +674,15 @@ __global__ void __launch_bounds__(352, 1)
         int bhq, i;
         q_item(p, t, bhq, i);
         const int bkv = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / p.G;
-        const int n_kv = q_n_kv(p, i);
+        int j0, n_kv;
+        q_kv_range(p, i, j0, n_kv);
         for (int j = 0; j < n_kv && ok; ++j) {
           const int g = gj + j, st = g % C::KVST;
           if (g >= C::KVST) ok = mbar_wait(&sh.v_empty[st], ((g / C::KVST) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sV + st * C::kTile + c * C::kBox, &tmv, &sh.v_full[st], c * 64, j * 128, bkv);
+            tma_load_3d(sV + st * C::kTile + c * C::kBox, &tmv, &sh.v_full[st], c * 64, (j0 + j) * 128, bkv);
           nv = g + 1;
         }
         gj += n_kv;
@@ -725,7 +745,8 @@ __global__ void __launch_bounds__(352, 1)
     for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
       int bhq, i;
       q_item(p, t, bhq, i);
-      const int n_kv = q_n_kv(p, i);
+      int j0, n_kv;
+      q_kv_range(p, i, j0, n_kv);
       ok = wait(&sh.qdo_full, it & 1);
       if (!ok) break;
       ok = issue_s(gj) && issue_dp(gj);
@@ -772,7 +793,8 @@ __global__ void __launch_bounds__(352, 1)
     for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x) {
       int bhq, i;
       q_item(p, t, bhq, i);
-      const int n_kv = q_n_kv(p, i);
+      int j0, n_kv;
+      q_kv_range(p, i, j0, n_kv);
       const int qrow = i * 128 + r;
       const size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + qrow;
       const float l2 = p.lse2[vrow], drow = p.dd[vrow];
@@ -782,10 +804,12 @@ __global__ void __launch_bounds__(352, 1)
       for (int u = 0; u < n_kv && ok; ++u) {
         const int g = gj + u, sb = g & 1;
         const uint32_t sbase = lane_base + (sb ? C::kS1 : C::kS0) + 64 * hb;
-        // visible key columns (relative to this warpgroup's 64) for this query row
-        const int kbase = u * 128 + 64 * hb;
-        const int hi = min(p.N - 1, p.causal ? qrow : p.N - 1) - kbase;
-        const bool masked = !__all_sync(0xffffffffu, hi >= 63);
+        // visible key columns (relative to this warpgroup's 64) for this query row:
+        // keys qrow - wl .. qrow + wr
+        const int kbase = (j0 + u) * 128 + 64 * hb;
+        const int hi = min(p.N - 1, qrow + p.wr) - kbase;
+        const int lo = qrow - p.wl - kbase;
+        const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= 63);
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[sb], (g >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
@@ -797,7 +821,7 @@ __global__ void __launch_bounds__(352, 1)
           tmem_ld16(sbase + q16 * 16, sr);
           tmem_wait_ld();
           reg_fence(sr);
-          bwd_exp16(sr, lv, c, masked, q16 * 16, 0, hi, pf + q16 * 16);
+          bwd_exp16(sr, lv, c, masked, q16 * 16, lo, hi, pf + q16 * 16);
         }
         // phase B: dS = P (dP - D) -> bf16 over the S buffer
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.dp_full, g & 1));
@@ -864,7 +888,7 @@ __global__ void __launch_bounds__(352, 1)
 }
 
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-               void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+               void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int wl, int wr,
                void* workspace, cudaStream_t stream, int sms);
 
 }  // namespace attn

@@ -26,20 +26,26 @@ __host__ __device__ inline float folded_scale(float scale) {
   return c > 1e-30f ? c : 1e-30f;
 }
 
+// Visibility of key j from query i: i - wl <= j <= i + wr.  wl = wr = N is full
+// attention, (N, 0) causal, (w - 1, 0) a causal sliding window of w keys (page
+// "attn-efficient", sliding-window row of the family table).
 struct FwdParams {
   void* o;
   float* lse;
   int B, Hq, Hkv, N, G;
   int n_qtiles;
   float c;          // scale * log2(e)
-  int causal;
+  int wl, wr;       // window: 0 <= wl, wr <= N
+  int desc;         // list query tiles last-first (their key ranges grow with the tile)
   int sched_slot;   // g_sched slot this launch claims work units from
 };
 
-// Key tiles a query tile sees: all of them, or (causal) those up to its diagonal.
-__device__ __forceinline__ int fwd_n_kv(const FwdParams& p, int qt) {
-  int n_kv_all = (p.N + 127) / 128;
-  return p.causal ? (qt + 1) : n_kv_all;
+// Key tiles [j0, j0 + n) that query tile qt sees (n >= 1 for a tile with a row < N).
+__device__ __forceinline__ void fwd_kv_range(const FwdParams& p, int qt, int& j0, int& n) {
+  const int r0 = qt * 128, r1 = min(p.N - 1, r0 + 127);
+  const int k0 = max(0, r0 - p.wl), k1 = min(p.N - 1, r1 + p.wr);
+  j0 = k0 >> 7;
+  n = (k1 >> 7) - j0 + 1;
 }
 
 }  // namespace attn

@@ -83,18 +83,21 @@ static_assert(sizeof(PpShared) <= 8192, "PpShared does not fit its slot");
 
 
 struct PpUnit {
-  int bh0, qt0, n0;           // tile A
-  int bh1, qt1, n1;           // tile B (n1 = 0: no tile B)
+  int bh0, qt0, a0, n0;       // tile A: key tiles [a0, a0 + n0)
+  int bh1, qt1, a1, n1;       // tile B (n1 = 0: no tile B)
+  int u0, u1;                 // union of the two key ranges, [u0, u1]
   int bkv;
   __device__ __forceinline__ int n(int x) const { return x ? n1 : n0; }
+  __device__ __forceinline__ int a(int x) const { return x ? a1 : a0; }
   __device__ __forceinline__ int qt(int x) const { return x ? qt1 : qt0; }
   __device__ __forceinline__ int bh(int x) const { return x ? bh1 : bh0; }
 };
 
 // Unit u -> two query tiles of one KV head.  The tiles of a KV head group are
-// listed query-tile-major, longest first under causal masking, the G heads
-// inside; consecutive list entries are paired, so under causal masking tile A
-// sees as many key tiles as tile B or one more.
+// listed query-tile-major (last tile first when key ranges grow with the tile,
+// as under causal masking: longest first), the G heads inside; consecutive list
+// entries are paired.  The unit streams the union of the two tiles' key ranges;
+// each team works on its own range inside it.
 __device__ __forceinline__ PpUnit pp_unit(const FwdParams& p, int u) {
   const int per_group = p.G * p.n_qtiles;
   const int upg = (per_group + 1) >> 1;
@@ -102,19 +105,21 @@ __device__ __forceinline__ PpUnit pp_unit(const FwdParams& p, int u) {
   const int m = u - gk * upg;
   PpUnit r;
   r.bkv = gk;
-  auto tile = [&](int l, int& bh, int& qt, int& n) {
+  auto tile = [&](int l, int& bh, int& qt, int& a, int& n) {
     if (l < per_group) {
       const int rq = l / p.G;
       const int h = l - rq * p.G;
-      qt = p.causal ? (p.n_qtiles - 1 - rq) : rq;
+      qt = p.desc ? (p.n_qtiles - 1 - rq) : rq;
       bh = (gk / p.Hkv) * p.Hq + (gk % p.Hkv) * p.G + h;
-      n = fwd_n_kv(p, qt);
+      fwd_kv_range(p, qt, a, n);
     } else {
-      bh = 0; qt = 0; n = 0;
+      bh = 0; qt = 0; a = 0; n = 0;
     }
   };
-  tile(2 * m, r.bh0, r.qt0, r.n0);
-  tile(2 * m + 1, r.bh1, r.qt1, r.n1);
+  tile(2 * m, r.bh0, r.qt0, r.a0, r.n0);
+  tile(2 * m + 1, r.bh1, r.qt1, r.a1, r.n1);
+  r.u0 = r.n1 > 0 ? min(r.a0, r.a1) : r.a0;
+  r.u1 = r.n1 > 0 ? max(r.a0 + r.n0, r.a1 + r.n1) - 1 : r.a0 + r.n0 - 1;
   return r;
 }
 
@@ -190,7 +195,7 @@ __global__ void __launch_bounds__(576, 1)
         };
         ok = load_q(0, uq0++);
         if (ok && w.n1 > 0) ok = load_q(1, uq1++);
-        for (int j = 0; j < w.n0 && ok; ++j, ++kc) {
+        for (int j = w.u0; j <= w.u1 && ok; ++j, ++kc) {
           const int st = kc & 1;
           if (kc >= 2) ok = mbar_wait(&sh.k_empty[st], ((kc >> 1) - 1) & 1);
           if (!ok) break;
@@ -262,14 +267,16 @@ __global__ void __launch_bounds__(576, 1)
       const int u = unit_ring_take(sh.ring, k, lane, ok);
       if (u < 0) break;
       const PpUnit w = pp_unit(p, u);
-      // first S of each team
+      // Team x works on key tiles [a_x, l_x] inside the unit's union [u0, u1]; its S for
+      // the first of them is issued as soon as that K tile is in (K(u0) here, later ones
+      // from the step before).
       {
         const int st = kc & 1;
         ok = wait(&sh.k_full[st], (kc >> 1) & 1);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           const int uux = x ? uu1 : uu0;
-          if (!ok || w.n(x) == 0) continue;
+          if (!ok || w.n(x) == 0 || w.a(x) != w.u0) continue;
           ok = wait(&sh.q_full[x][uux % C::QST], (uux / C::QST) & 1);
           if (!ok) continue;
           tc_fence_after();
@@ -280,29 +287,41 @@ __global__ void __launch_bounds__(576, 1)
         __syncwarp();
         ++kc;
       }
-      for (int j = 0; j < w.n0 && ok; ++j, ++vc) {
+      for (int j = w.u0; j <= w.u1 && ok; ++j, ++vc) {
         const int vst = vc & 1;
         ok = wait(&sh.v_full[vst], (vc >> 1) & 1);
-        const bool next_k = j + 1 < w.n0;
+        const bool next_k = j + 1 <= w.u1;
         bool k_ready = false;
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          const int gsx = x ? gs1 : gs0, uux = x ? uu1 : uu0, nx = w.n(x);
-          if (!ok || j >= nx) continue;
-          const int g = gsx + j;
-          ok = wait(&sh.p_ready[x], g & 1);
-          if (ok && j == 0 && uux >= 1) ok = wait(&sh.o_free[x], (uux - 1) & 1);
-          if (!ok) continue;
-          tc_fence_after();
-          issue_pv(x, vst, j == 0);
-          if (j + 1 < nx) {
+          const int gsx = x ? gs1 : gs0, uux = x ? uu1 : uu0, nx = w.n(x), ax = w.a(x);
+          if (!ok || nx == 0) continue;
+          const int lx = ax + nx - 1;
+          if (ax <= j && j <= lx) {
+            const int g = gsx + (j - ax);
+            ok = wait(&sh.p_ready[x], g & 1);
+            if (ok && j == ax && uux >= 1) ok = wait(&sh.o_free[x], (uux - 1) & 1);
+            if (!ok) continue;
+            tc_fence_after();
+            issue_pv(x, vst, j == ax);
+            if (j + 1 <= lx) {
+              if (!k_ready) {
+                ok = wait(&sh.k_full[kc & 1], (kc >> 1) & 1);
+                k_ready = true;
+              }
+              if (!ok) continue;
+              tc_fence_after();
+              issue_s(x, uux % C::QST, kc & 1, j + 1 == lx);   // in issue order behind PV_X(j)
+            }
+          } else if (j + 1 == ax) {          // team x starts at the next key tile
             if (!k_ready) {
               ok = wait(&sh.k_full[kc & 1], (kc >> 1) & 1);
               k_ready = true;
             }
+            if (ok) ok = wait(&sh.q_full[x][uux % C::QST], (uux / C::QST) & 1);
             if (!ok) continue;
             tc_fence_after();
-            issue_s(x, uux % C::QST, kc & 1, j + 2 == nx);   // in issue order behind PV_X(j)
+            issue_s(x, uux % C::QST, kc & 1, nx == 1);
           }
         }
         if (!ok) break;
@@ -335,16 +354,16 @@ __global__ void __launch_bounds__(576, 1)
     const uint64_t c2 = f2pack(c, c);
     int gs = 0, uu = 0;
     bool ok = true;
-    auto mask16 = [&](uint32_t (&r)[16], int col0, int lim) {
+    auto mask16 = [&](uint32_t (&r)[16], int col0, int lo, int lim) {
 #pragma unroll
       for (int k = 0; k < 16; ++k)
-        if (col0 + k > lim) r[k] = 0xff800000u;
+        if (col0 + k < lo || col0 + k > lim) r[k] = 0xff800000u;
     };
     for (int k = 0; ok; ++k) {
       const int u = unit_ring_take(sh.ring, k, lane, ok);
       if (u < 0) break;
       const PpUnit w = pp_unit(p, u);
-      const int n = w.n(x);
+      const int n = w.n(x), a = w.a(x);
       if (n == 0) continue;
       const int qrow = w.qt(x) * 128 + row;
       const int bh = w.bh(x);
@@ -355,9 +374,10 @@ __global__ void __launch_bounds__(576, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[x], g & 1));
         if (!ok) break;
         tc_fence_after();
-        const int kbase = j * 128 + grp * 64;
-        const int lim = p.causal ? min(p.N - 1, qrow) - kbase : p.N - 1 - kbase;   // last visible column
-        const bool msk = __any_sync(0xffffffffu, lim < 63);
+        const int kbase = (a + j) * 128 + grp * 64;
+        const int lo = qrow - p.wl - kbase;                          // first visible column
+        const int lim = min(p.N - 1, qrow + p.wr) - kbase;           // last visible column
+        const bool msk = __any_sync(0xffffffffu, lo > 0 || lim < 63);
         // pass 1: this group's partial row max of the 64 columns
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         {
@@ -371,7 +391,7 @@ __global__ void __launch_bounds__(576, 1)
           reg_fence(r1);
           reg_fence(r2);
           reg_fence(r3);
-          if (msk) { mask16(r0, 0, lim); mask16(r1, 16, lim); mask16(r2, 32, lim); mask16(r3, 48, lim); }
+          if (msk) { mask16(r0, 0, lo, lim); mask16(r1, 16, lo, lim); mask16(r2, 32, lo, lim); mask16(r3, 48, lo, lim); }
 #pragma unroll
           for (int k = 0; k < 16; k += 8) {
 #pragma unroll
@@ -430,7 +450,7 @@ __global__ void __launch_bounds__(576, 1)
           tmem_ld16(s_base + cc * 16, r);
           tmem_wait_ld();
           reg_fence(r);
-          if (msk) mask16(r, cc * 16, lim);
+          if (msk) mask16(r, cc * 16, lo, lim);
           uint32_t pk[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {

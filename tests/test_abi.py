@@ -27,7 +27,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
-         "attn_status_string", "attn_selftest_timeout"])
+         "attn_status_string", "attn_selftest_timeout", "attn_fwd_window", "attn_bwd_window"])
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -113,3 +113,21 @@ def test_selftest_timeout_rejects_out_of_range_limits(L):
     assert L.attn_selftest_timeout(0, None) == -1
     assert L.attn_selftest_timeout(-5, None) == -1
     assert L.attn_selftest_timeout(2_000_000_000, None) == -1
+
+
+def test_window_entry_points_validate_like_the_plain_ones(L):
+    def fwdw(q=FAKE, d=64, N=128, scale=0.125, wl=16, wr=0):
+        return L.attn_fwd_window(q, FAKE, FAKE, FAKE, FAKE, 1, 1, 1, N, d, scale, wl, wr, None)
+    assert fwdw(d=96) == -2
+    assert fwdw(N=0) == -1
+    assert fwdw(scale=-1.0) == -1
+    assert fwdw(q=ODD) == -3
+    assert fwdw(q=ctypes.c_void_p(0)) == -1
+    size = L.attn_bwd_workspace_size(1, 2, 1, 300, 128, 0)
+
+    def bwdw(wsb=size, dq=FAKE, d=128):
+        return L.attn_bwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, dq, FAKE, FAKE, 1, 2, 1, 300, d, 0.1, 31, 0,
+                                 FAKE, ctypes.c_size_t(wsb), None)
+    assert bwdw(wsb=size - 1) == -6
+    assert bwdw(dq=ODD) == -3
+    assert bwdw(d=80) == -2

@@ -50,7 +50,7 @@ def test_bwd_matches_oracle(attn, B, Hq, Hkv, N, d, causal):
     _, grads, scale = run_fwd_bwd(attn, x, d, causal)
     g_ref = ref.ref_bwd(to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"]), to_f64(x["do"]), scale, causal)
     for g, r, name in zip(grads, g_ref, ("dQ", "dK", "dV")):
-        check_grad(f64(g), r, name)
+        check_grad(f64(g), r, f"B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} {'causal' if causal else 'full'} {name}")
 
 
 def test_bwd_is_bitwise_deterministic(attn):

@@ -50,8 +50,9 @@ SMALL = [
 def test_fwd_matches_oracle(attn, B, Hq, Hkv, N, d, causal):
     x, o, lse, scale = run_fwd(attn, B, Hq, Hkv, N, d, causal, seed=N * 7 + d + causal)
     o_ref, lse_ref = ref.ref_fwd(to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"]), scale, causal)
-    check_o(f64(o), o_ref)
-    check_lse(f64(lse), lse_ref)
+    tag = f"B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} {'causal' if causal else 'full'}"
+    check_o(f64(o), o_ref, f"{tag} O")
+    check_lse(f64(lse), lse_ref, f"{tag} LSE")
 
 
 def test_fwd_large_scores_force_rescaling(attn):
