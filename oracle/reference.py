@@ -138,6 +138,23 @@ def ref_bwd(q, k, v, do, scale, causal, block=1024, window=None):
     return dq, dk, dv
 
 
+def ref_decode(q, k, v, scale, causal):
+    """Attention of Nq new query rows against Nk cached keys (split-KV decoding; page
+    "attention 的显存线性化", reading list on FlashDecoding, and the online-softmax
+    part of page "attn-efficient", whose rescale merges the per-split partials).
+
+    q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d], fp64.  The result is the plain definition over
+    all Nk keys; how the keys are split never shows.  Causal reading (the pages give
+    none for Nq != Nk): the query rows are the LAST Nq positions of the sequence, so
+    query i sits at position Nk - Nq + i and sees keys j <= Nk - Nq + i -- the window
+    (None, Nk - Nq) of ``visible``.  Returns (O [B,Hq,Nq,d], LSE [B,Hq,Nq]).
+    """
+    nq, nk = q.shape[2], k.shape[2]
+    if causal and nq > nk:
+        raise ValueError("causal decoding needs Nq <= Nk")
+    return ref_fwd(q, k, v, scale, False, window=(None, nk - nq) if causal else None)
+
+
 def online_fwd_head(qh, kh, vh, scale, causal, bounds, window=None):
     """The pages' blockwise online softmax for one head (used only in self-tests).
 

@@ -405,3 +405,51 @@ def test_window_blockwise_online_softmax_equals_full(window):
     o_on, lse_on = ref.online_fwd_head(qh, kh, vh, 0.4, False, [0, 3, 4, 10, 12, n], window=window)
     np.testing.assert_allclose(o_on, o_full, rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(lse_on, lse_full, rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------- decoding: Nq query rows against Nk keys
+@pytest.mark.parametrize("nq,nk", [(1, 1), (1, 9), (3, 9), (9, 9), (4, 17)])
+def test_causal_decode_is_the_tail_of_full_causal_attention(nq, nk):
+    """The reading puts the Nq queries at the last positions: their rows of square
+    causal attention over all Nk positions (itself pinned to the C brute force)."""
+    B, Hq, Hkv, d = 2, 4, 2, 3
+    qfull, k, v = rand(B, Hq, nk, d), rand(B, Hkv, nk, d), rand(B, Hkv, nk, d)
+    o_full, lse_full = ref.ref_fwd(qfull, k, v, 0.7, True)
+    o, lse = ref.ref_decode(qfull[:, :, nk - nq:], k, v, 0.7, True)
+    np.testing.assert_allclose(o, o_full[:, :, nk - nq:], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse, lse_full[:, :, nk - nq:], rtol=1e-13, atol=1e-14)
+    ob, lseb = obuild.brute_fwd(qfull, k, v, 0.7, True)
+    np.testing.assert_allclose(o, ob[:, :, nk - nq:], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_decode_matches_torch_sdpa_rectangular(causal):
+    B, Hq, Hkv, nq, nk, d = 2, 6, 3, 5, 23, 4
+    q, k, v = rand(B, Hq, nq, d), rand(B, Hkv, nk, d), rand(B, Hkv, nk, d)
+    mask = None
+    if causal:   # bottom-right aligned: query i sees keys j <= nk - nq + i
+        mask = torch.arange(nk)[None, :] <= torch.arange(nq)[:, None] + (nk - nq)
+    to = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q), torch.tensor(k).repeat_interleave(2, dim=1), torch.tensor(v).repeat_interleave(2, dim=1),
+        attn_mask=mask, scale=0.3)
+    o, lse = ref.ref_decode(q, k, v, 0.3, causal)
+    np.testing.assert_allclose(o, to.numpy(), rtol=1e-10, atol=1e-12)
+    s = 0.3 * np.einsum("bhqd,bhkd->bhqk", q, np.repeat(k, 2, axis=1))
+    if causal:
+        s = np.where(mask.numpy(), s, -np.inf)
+    np.testing.assert_allclose(lse, np.log(np.exp(s).sum(axis=-1)), rtol=1e-12)
+
+
+def test_decode_partials_merge_by_lse():
+    """The merge rule the split-KV path relies on: attention over disjoint key ranges,
+    combined with weights exp(LSE_s - LSE), equals attention over all keys."""
+    nq, nk, d = 3, 40, 5
+    qh, kh, vh = rand(nq, d), rand(nk, d), rand(nk, d)
+    o, lse = ref.attend_head(qh, kh, vh, 0.9, False)
+    parts = [ref.attend_head(qh, kh[a:b], vh[a:b], 0.9, False) for a, b in ((0, 7), (7, 8), (8, 40))]
+    m = np.max([p[1] for p in parts], axis=0)
+    w = [np.exp(p[1] - m) for p in parts]
+    lse_m = m + np.log(sum(w))
+    o_m = sum(wi[:, None] * p[0] for wi, p in zip(w, parts)) / sum(w)[:, None]
+    np.testing.assert_allclose(o_m, o, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse_m, lse, rtol=1e-13)
