@@ -63,6 +63,47 @@ WORKLOADS = {
         qk_std=3.0, boost_frac=0.01, boost=8.0, seed=1004),
 }
 
+# Decoding problems (split-KV path): Nq new query rows against an Nk-key cache.  Shapes
+# of a grouped-query model at long context (32 query heads, 8 KV heads, d = 128);
+# inputs N(0, 1).
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int = 3000
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+DECODE_WORKLOADS = {
+    "decode_b16_hq32_hkv8_nq1_nk32768_d128": DecodeWorkload(
+        "decode_b16_hq32_hkv8_nq1_nk32768_d128", 16, 32, 8, 1, 32768, 128, True, seed=3000),
+    "decode_b4_hq32_hkv8_nq16_nk131072_d128": DecodeWorkload(
+        "decode_b4_hq32_hkv8_nq16_nk131072_d128", 4, 32, 8, 16, 131072, 128, True, seed=3001),
+    "decode_b64_hq16_hkv16_nq1_nk4096_d64": DecodeWorkload(
+        "decode_b64_hq16_hkv16_nq1_nk4096_d64", 64, 16, 16, 1, 4096, 64, True, seed=3002),
+}
+
+
+def make_decode_inputs(w: DecodeWorkload, device="cpu"):
+    """q [B,Hq,Nq,d], k and v [B,Hkv,Nk,d]: bf16 N(0,1) draws from one seeded generator."""
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    q = _normal_bf16((w.B, w.Hq, w.Nq, w.d), 1.0, gen, dev)
+    k = _normal_bf16((w.B, w.Hkv, w.Nk, w.d), 1.0, gen, dev)
+    v = _normal_bf16((w.B, w.Hkv, w.Nk, w.d), 1.0, gen, dev)
+    return {"q": q, "k": k, "v": v}
+
+
 # Sequence-length sweep: a fixed number of tokens B*N and a fixed model width Hq*d,
 # so the work per token grows with N and the FLOP/byte of each head is ~N/4.  At
 # N = 32768 one sequence already exceeds the token budget, so B stays 1 there.

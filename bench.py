@@ -35,7 +35,8 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from attn_inputs import WORKLOADS, Workload, make_inputs, sweep_workloads  # noqa: E402
+from attn_inputs import (DECODE_WORKLOADS, WORKLOADS, Workload, make_decode_inputs, make_inputs,  # noqa: E402
+                         sweep_workloads)
 from io_aware_exact_26_b200 import accounting as acc  # noqa: E402
 
 # The largest single-GPU workload (forward + backward, causal, d = 128, N = 32768).
@@ -350,6 +351,66 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_decode(args):
+    """Split-KV decoding, timed apart: one JSON line per decode workload.  The path is bound
+    by HBM, so the roofline is algorithmic bytes (Q, K, V read once, O and LSE written)
+    over the event-timed duration, against the measured copy bandwidth."""
+    import torch
+    import io_aware_exact_26_b200 as attn
+
+    peaks, peaks_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    names = [args.decode_workload] if args.decode_workload else list(DECODE_WORKLOADS)
+    for name in names:
+        w = DECODE_WORKLOADS[name]
+        x = make_decode_inputs(w, device=dev)
+        o = torch.empty_like(x["q"])
+        lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(1, attn.attn_decode_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal)),
+                         dtype=torch.uint8, device=dev)
+        # inputs of one call are smaller than L2 for some shapes: rotate through copies
+        kv_bytes = 2 * x["k"].numel() * 2
+        copies = max(1, -(-2 * 126 * 2 ** 20 // kv_bytes))
+        bufs = [x] + [{n: t.clone() for n, t in x.items()} for _ in range(copies - 1)]
+
+        def call(i):
+            b = bufs[i % len(bufs)]
+            attn.attn_decode(b["q"], b["k"], b["v"], o, lse, scale=w.scale, causal=w.causal, workspace=ws)
+
+        for i in range(args.warmup):
+            call(i)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.sweep_reps)]
+        sampler = ClockSampler(0)
+        sampler.start()
+        for i, (a, b) in enumerate(evs):
+            a.record(stream)
+            call(i)
+            b.record(stream)
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
+        if attn.attn_get_device_status() != 0:
+            raise SystemExit(f"device-side error in decode {name}")
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        nbytes = acc.min_bytes_decode(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        splits = attn.attn_decode_splits(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal)
+        print(json.dumps({
+            "decode": name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+            "causal": w.causal, "splits": splits, "reps": args.sweep_reps, "warmup": args.warmup, "ms": round(ms, 4),
+            "tflops": round(acc.flops_decode(w.B, w.Hq, w.Nq, w.Nk, w.d, w.causal) / (ms * 1e-3) / 1e12, 2),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
+                         "peak_source": f"{peaks_kind} copy bandwidth"},
+            "l2": f"{len(bufs)} input copies rotated (K+V {kv_bytes / 1e6:.0f} MB each)",
+            "gpu_launches_per_call": 2 + (splits > 1), "clocks": clocks}), flush=True)
+        del x, bufs, o, lse, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -362,10 +423,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="time the sequence-length sweep, one line per point")
     ap.add_argument("--sweep-reps", type=int, default=50)
+    ap.add_argument("--decode", action="store_true", help="time split-KV decoding, one line per decode workload")
+    ap.add_argument("--decode-workload", default=None, choices=sorted(DECODE_WORKLOADS))
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.sweep:
         run_sweep(args)
+        return
+    if args.decode:
+        run_decode(args)
         return
 
     rank = int(os.environ.get("RANK", "0"))

@@ -111,6 +111,30 @@ int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, 
                     int window_left, int window_right,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decoding: Nq new query rows against Nk keys (a KV cache), split over the keys
+ * (page "attention 的显存线性化", reading list: FlashDecoding).  The keys of each
+ * (batch, kv-head) are cut into splits processed in parallel; each split leaves a
+ * partial output and log-sum-exp, and the partials are merged with the online-
+ * softmax rescale (page "attn-efficient", online-softmax section):
+ * O = sum_s exp(LSE_s - LSE) O_s.  The result is exact attention over all Nk keys.
+ *   q, o : bf16 [B][Hq][Nq][d]     k, v : bf16 [B][Hkv][Nk][d]     lse : fp32 [B][Hq][Nq]
+ *   causal: 1 = the queries are the last Nq positions of the sequence: query i
+ *     sees keys j <= Nk - Nq + i (requires Nq <= Nk); 0 = every query sees every key.
+ *   Hq / Hkv <= 128 (the group's query heads share one K/V stream).
+ * Workspace (the split partials): attn_decode_workspace_size(...) bytes, queried
+ * with the same device current (the split count depends on its SM count; 0 when
+ * one split suffices).  NULL: the library allocates it on `stream` with
+ * cudaMallocAsync / cudaFreeAsync.  Errors as attn_fwd, plus ATTN_ERR_WORKSPACE
+ * (too small) and ATTN_ERR_ALLOC.  Enqueues a counter-reset kernel, the split
+ * kernel and, with more than one split, the merge kernel. */
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
+int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                void* workspace, size_t workspace_bytes, void* stream);
+/* Number of key splits attn_decode uses for this shape on the current device
+ * (0 for arguments it would reject). */
+int attn_decode_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
+
 /* Backward without a caller-provided workspace (no counterpart on the pages; an
  * interface convenience).  Same arguments, layouts and results as attn_bwd, minus
  * `workspace`/`workspace_bytes`: the scratch lives in a fixed 64 MiB device array

@@ -10,6 +10,9 @@ from .binding import (  # noqa: F401
     attn_bwd,
     attn_bwd_noalloc,
     attn_bwd_window,
+    attn_decode,
+    attn_decode_splits,
+    attn_decode_workspace_size,
     NOALLOC_SCRATCH_BYTES,
     attn_bwd_workspace_size,
     attn_fwd,

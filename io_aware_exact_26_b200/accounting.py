@@ -84,3 +84,17 @@ def balance_point(flops_per_s, bytes_per_s):
 
 def tflops(flops, ms):
     return flops / (ms * 1e-3) / 1e12
+
+
+def min_bytes_decode(B, Hq, Hkv, Nq, Nk, d):
+    """Decoding reads Q, K, V once and writes O and LSE: K and V dominate, O(Nk * d)."""
+    return 2 * B * Hq * Nq * d * BF16 + 2 * B * Hkv * Nk * d * BF16 + B * Hq * Nq * FP32
+
+
+def flops_decode(B, Hq, Nq, Nk, d, causal):
+    """4*d FLOPs per visible (query, key) pair; causal queries are the last Nq positions."""
+    if causal:
+        pairs = sum(Nk - Nq + 1 + i for i in range(Nq))
+    else:
+        pairs = Nq * Nk
+    return 4.0 * B * Hq * pairs * d

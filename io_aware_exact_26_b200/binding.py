@@ -46,6 +46,12 @@ def lib():
     L.attn_fwd_window.restype = i
     L.attn_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
     L.attn_bwd_window.restype = i
+    L.attn_decode_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    L.attn_decode_workspace_size.restype = sz
+    L.attn_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
+    L.attn_decode.restype = i
+    L.attn_decode_splits.argtypes = [i, i, i, i, i, i, i]
+    L.attn_decode_splits.restype = i
     L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     L.attn_bwd_noalloc.restype = i
     L.attn_get_device_status.argtypes = [vp]
@@ -155,6 +161,39 @@ def attn_bwd_window(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, window, s
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd_window")
     return dq, dk, dv
+
+
+def attn_decode(q, k, v, o=None, lse=None, *, scale=None, causal=False, workspace=None, stream=None):
+    """Nq query rows against Nk keys, split over the keys and merged by LSE; returns (o, lse).
+
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] bf16.  causal: the queries are the last Nq
+    positions (query i sees keys j <= Nk - Nq + i).  workspace=None lets the library
+    allocate the split partials on the stream.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(o, "o")
+    _check(lse, "lse", torch.float32)
+    if scale is None:
+        scale = d ** -0.5
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                           int(bool(causal)), _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_decode")
+    return o, lse
+
+
+def attn_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal=False) -> int:
+    return int(lib().attn_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, int(bool(causal))))
+
+
+def attn_decode_splits(B, Hq, Hkv, Nq, Nk, d, causal=False) -> int:
+    return int(lib().attn_decode_splits(B, Hq, Hkv, Nq, Nk, d, int(bool(causal))))
 
 
 def attn_bwd_workspace_size(B, Hq, Hkv, N, d, causal=False) -> int:

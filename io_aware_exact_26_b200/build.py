@@ -9,7 +9,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libattn_b200.so")
 SOURCES = [os.path.join(CSRC, "api.cu")]
-HEADERS = [os.path.join(CSRC, f) for f in ("sm100.cuh", "fwd.cuh", "fwd_pp.cuh", "bwd.cuh")] + [
+HEADERS = [os.path.join(CSRC, f) for f in ("sm100.cuh", "fwd.cuh", "fwd_pp.cuh", "bwd.cuh", "decode.cuh")] + [
     os.path.join(ROOT, "include", "attn.h")]
 
 NVCC_FLAGS = [

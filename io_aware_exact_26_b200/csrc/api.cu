@@ -17,6 +17,7 @@
 #include "fwd.cuh"
 #include "fwd_pp.cuh"
 #include "bwd.cuh"
+#include "decode.cuh"
 
 namespace {
 
@@ -141,6 +142,118 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   attn::sched_reset_kernel<<<1, 32, 0, stream>>>(p.sched_slot);
   attn::attn_fwd_pp_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+// Split-KV decoding (decode.cuh): how the keys of each (b, kv-head, query block) are
+// split.  The work is bound by HBM; units are claimed dynamically, so a few per SM
+// keep the tail short while each unit still streams several key tiles.
+struct DecodePlan {
+  int G, R, nqb, nkt, S, T;
+  long long units;
+};
+
+DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int sms) {
+  DecodePlan pl;
+  pl.G = Hq / Hkv;
+  pl.R = Nq < 128 / pl.G ? Nq : 128 / pl.G;
+  pl.nqb = (Nq + pl.R - 1) / pl.R;
+  pl.nkt = (Nk + 127) / 128;
+  const long long pairs = static_cast<long long>(B) * Hkv * pl.nqb;
+  const long long target = 8LL * sms;                       // units to aim for
+  long long T = (pl.nkt * pairs + target - 1) / target;     // key tiles per split
+  if (T < 4) T = 4;
+  if (T > pl.nkt) T = pl.nkt;
+  pl.T = static_cast<int>(T);
+  pl.S = (pl.nkt + pl.T - 1) / pl.T;
+  pl.units = pairs * pl.S;
+  return pl;
+}
+
+// Workspace of the split partials: O_s fp32 [rows][S][d], then LSE_s fp32 [rows][S].
+struct DecodeWs {
+  size_t o_off, l_off, total;
+};
+DecodeWs decode_ws(long long rows, int S, int d) {
+  DecodeWs w;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  w.o_off = 0;
+  if (S <= 1) {
+    w.l_off = 0;
+    w.total = 0;
+    return w;
+  }
+  w.l_off = up(static_cast<size_t>(rows) * S * d * 4);
+  w.total = up(w.l_off + static_cast<size_t>(rows) * S * 4);
+  return w;
+}
+
+template <int D>
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                  int Nq, int Nk, float scale, int causal, const DecodePlan& pl, void* ws, cudaStream_t stream,
+                  const DeviceInfo& di) {
+  using C = attn::DecCfg<D>;
+  static std::once_flag attr_once[64];
+  static bool attr_ok[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(attr_once[dev], [&] {
+    attr_ok[dev] = cudaFuncSetAttribute(attn::attn_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmem) == cudaSuccess;
+  });
+  if (!attr_ok[dev]) return ATTN_ERR_LAUNCH;
+  CUtensorMap tk, tv;
+  if (!make_map(&tk, k, D, Nk, static_cast<long long>(B) * Hkv, 128) ||
+      !make_map(&tv, v, D, Nk, static_cast<long long>(B) * Hkv, 128))
+    return ATTN_ERR_LAUNCH;
+  const long long rows = static_cast<long long>(B) * Hq * Nq;
+  const DecodeWs W = decode_ws(rows, pl.S, D);
+  attn::DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.opart = pl.S > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + W.o_off) : nullptr;
+  p.lpart = pl.S > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + W.l_off) : nullptr;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = pl.G;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.R = pl.R;
+  p.nqb = pl.nqb;
+  p.S = pl.S;
+  p.T = pl.T;
+  p.causal = causal;
+  p.c = attn::folded_scale(scale);
+  p.n_units = static_cast<int>(pl.units);
+  p.sched_slot = next_sched_slot();
+  const int grid = pl.units < di.sms ? static_cast<int>(pl.units) : di.sms;
+  attn::sched_reset_kernel<<<1, 32, 0, stream>>>(p.sched_slot);
+  attn::attn_decode_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tk, tv, p);
+  if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (pl.S > 1) {
+    long long blocks = (rows * 32 + 255) / 256;
+    const long long cap = static_cast<long long>(di.sms) * 16;
+    if (blocks > cap) blocks = cap;
+    attn::attn_decode_merge_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        p.opart, p.lpart, static_cast<__nv_bfloat16*>(o), lse, rows, pl.S);
+    if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  }
+  return ATTN_OK;
+}
+
+int check_decode(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal) {
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || Hq / Hkv > 128) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (causal && Nq > Nk) return ATTN_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * Hq * Nq;
+  if (rows * d >= (1ll << 40) || static_cast<long long>(Nk) * d * 2 >= (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  // work units (b, kv-head, query block, key split) must stay below 2^31: blocks <= Nq, splits <= key tiles
+  if (static_cast<long long>(B) * Hkv * Nq * ((Nk + 127) / 128) >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
 }
 
 }  // namespace
@@ -333,6 +446,51 @@ int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, 
                     void* stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, 0,
                   band_of_window(N, window_left, window_right), workspace, workspace_bytes, stream);
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {
+  if (check_decode(B, Hq, Hkv, Nq, Nk, d, 1.f, causal) != ATTN_OK) return 0;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return 0;
+  const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, di->sms);
+  return decode_ws(static_cast<long long>(B) * Hq * Nq, pl.S, d).total;
+}
+
+int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                int Nk, int d, float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_decode(B, Hq, Hkv, Nq, Nk, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_ALIGNMENT;
+  if (workspace && !aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
+  const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, di->sms);
+  const size_t need = decode_ws(static_cast<long long>(B) * Hq * Nq, pl.S, d).total;
+  if (workspace && workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (!ws && need > 0) {
+    if (cudaMallocAsync(&ws, need, s) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return ATTN_ERR_ALLOC;
+    }
+  }
+  const int st2 = d == 64 ? launch_decode<64>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, pl, ws, s, *di)
+                          : launch_decode<128>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, pl, ws, s, *di);
+  if (!workspace && need > 0 && cudaFreeAsync(ws, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return st2 != ATTN_OK ? st2 : ATTN_ERR_ALLOC;
+  }
+  return st2;
+}
+
+int attn_decode_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {
+  if (check_decode(B, Hq, Hkv, Nq, Nk, d, 1.f, causal) != ATTN_OK) return 0;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return 0;
+  return decode_plan(B, Hq, Hkv, Nq, Nk, di->sms).S;
 }
 
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,

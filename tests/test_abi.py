@@ -27,7 +27,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
-         "attn_status_string", "attn_selftest_timeout", "attn_fwd_window", "attn_bwd_window"])
+         "attn_status_string", "attn_selftest_timeout", "attn_fwd_window", "attn_bwd_window", "attn_decode",
+         "attn_decode_workspace_size", "attn_decode_splits"])
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -131,3 +132,21 @@ def test_window_entry_points_validate_like_the_plain_ones(L):
     assert bwdw(wsb=size - 1) == -6
     assert bwdw(dq=ODD) == -3
     assert bwdw(d=80) == -2
+
+
+def test_decode_validates_before_any_launch(L):
+    def dec(q=FAKE, Hq=8, Hkv=2, Nq=1, Nk=1000, d=128, scale=0.088, causal=1, ws=FAKE, wsb=1 << 30):
+        return L.attn_decode(q, FAKE, FAKE, FAKE, FAKE, 2, Hq, Hkv, Nq, Nk, d, scale, causal, ws,
+                             ctypes.c_size_t(wsb), None)
+    assert dec(d=96) == -2
+    assert dec(Nq=0) == -1
+    assert dec(Nk=0) == -1
+    assert dec(Nq=5, Nk=4) == -1                # causal needs Nq <= Nk
+    assert dec(Hq=258, Hkv=1) == -1             # group larger than one 128-row tile
+    assert dec(Hq=9) == -1
+    assert dec(scale=float("nan")) == -1
+    assert dec(q=ODD) == -3
+    assert dec(ws=ODD) == -3
+    assert dec(q=ctypes.c_void_p(0)) == -1
+    assert L.attn_decode_workspace_size(2, 8, 2, 5, 4, 128, 1) == 0
+    assert L.attn_decode_splits(2, 8, 2, 5, 4, 128, 1) == 0
