@@ -135,6 +135,19 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
  * (0 for arguments it would reject). */
 int attn_decode_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
 
+/* Merge of a partial attention result into a running one, for keys that arrive in
+ * blocks -- e.g. sequence shards passed around a ring of GPUs (the online-softmax
+ * rescale of page "attn-efficient" applied to whole blocks):
+ *   m = max(lse_acc, lse_part), a = exp(lse_acc - m), b = exp(lse_part - m),
+ *   o_acc = (a o_acc + b o_part) / (a + b),  lse_acc = m + ln(a + b).
+ *   o_acc  : fp32 [rows][d], updated in place (its contents are ignored where lse_acc = -inf)
+ *   lse_acc: fp32 [rows], updated in place; initialise to -inf for an empty accumulator
+ *   o_part : bf16 [rows][d] and lse_part fp32 [rows] -- an attn_fwd / attn_decode result
+ *   out    : NULL, or bf16 [rows][d] that receives the merged O rounded to bf16
+ * d is 64 or 128.  One kernel on `stream`. */
+int attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+               long long rows, int d, void* out, void* stream);
+
 /* Backward without a caller-provided workspace (no counterpart on the pages; an
  * interface convenience).  Same arguments, layouts and results as attn_bwd, minus
  * `workspace`/`workspace_bytes`: the scratch lives in a fixed 64 MiB device array

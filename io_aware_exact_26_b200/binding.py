@@ -52,6 +52,8 @@ def lib():
     L.attn_decode.restype = i
     L.attn_decode_splits.argtypes = [i, i, i, i, i, i, i]
     L.attn_decode_splits.restype = i
+    L.attn_merge.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, i, vp, vp]
+    L.attn_merge.restype = i
     L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     L.attn_bwd_noalloc.restype = i
     L.attn_get_device_status.argtypes = [vp]
@@ -186,6 +188,26 @@ def attn_decode(q, k, v, o=None, lse=None, *, scale=None, causal=False, workspac
     if st != ATTN_OK:
         raise AttnError(st, "attn_decode")
     return o, lse
+
+
+def attn_merge(o_acc, lse_acc, o_part, lse_part, out=None, *, stream=None):
+    """Merge a partial (o_part bf16, lse_part fp32) into the running (o_acc fp32, lse_acc fp32)
+    in place; writes the merged O as bf16 into ``out`` when given."""
+    _check(o_acc, "o_acc", torch.float32)
+    _check(lse_acc, "lse_acc", torch.float32)
+    _check(o_part, "o_part")
+    _check(lse_part, "lse_part", torch.float32)
+    if out is not None:
+        _check(out, "out")
+    d = o_acc.shape[-1]
+    rows = o_acc.numel() // d
+    if o_part.numel() != o_acc.numel() or lse_acc.numel() != rows or lse_part.numel() != rows:
+        raise ValueError("attn_merge: shapes of the accumulator and the partial differ")
+    st = lib().attn_merge(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), rows, d, _ptr(out),
+                          _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_merge")
+    return o_acc, lse_acc
 
 
 def attn_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal=False) -> int:

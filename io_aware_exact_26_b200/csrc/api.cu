@@ -493,6 +493,29 @@ int attn_decode_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal
   return decode_plan(B, Hq, Hkv, Nq, Nk, di->sms).S;
 }
 
+int attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows, int d,
+               void* out, void* stream) {
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (rows < 1 || rows * d >= (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  if (!o_acc || !lse_acc || !o_part || !lse_part) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o_acc) || !aligned16(lse_acc) || !aligned16(o_part) || !aligned16(lse_part) ||
+      (out && !aligned16(out)))
+    return ATTN_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
+  long long blocks = (rows * 32 + 255) / 256;
+  const long long cap = static_cast<long long>(di->sms) * 16;
+  if (blocks > cap) blocks = cap;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto* po = static_cast<const __nv_bfloat16*>(o_part);
+  auto* pout = static_cast<__nv_bfloat16*>(out);
+  if (d == 64)
+    attn::attn_merge_kernel<64><<<static_cast<int>(blocks), 256, 0, s>>>(o_acc, lse_acc, po, lse_part, pout, rows);
+  else
+    attn::attn_merge_kernel<128><<<static_cast<int>(blocks), 256, 0, s>>>(o_acc, lse_acc, po, lse_part, pout, rows);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
                      float scale, int causal, void* stream) {

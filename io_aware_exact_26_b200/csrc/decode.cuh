@@ -513,3 +513,47 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const float* __r
 }
 
 }  // namespace attn
+
+namespace attn {
+
+// Merge of one partial result into a running one, for attention whose keys arrive in
+// blocks (the ring of sequence shards across GPUs): with m = max(lse_acc, lse_part),
+// a = exp(lse_acc - m), b = exp(lse_part - m):
+//     o_acc <- (a o_acc + b o_part) / (a + b),   lse_acc <- m + ln(a + b)
+// (page "attn-efficient", online-softmax section: the same rescale as the tiled
+// loop, applied to whole blocks).  lse_acc = -inf marks an empty accumulator.
+// o_acc is fp32 so that repeated merges round only once, when `out` (bf16) is given.
+template <int D>
+__global__ void __launch_bounds__(256) attn_merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc,
+                                                         const __nv_bfloat16* __restrict__ o_part,
+                                                         const float* __restrict__ lse_part,
+                                                         __nv_bfloat16* __restrict__ out, long long rows) {
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r = w0; r < rows; r += nw) {
+    const float la = lse_acc[r], lb = lse_part[r];
+    const float m = fmaxf(la, lb);
+    const float a = la == -INFINITY ? 0.f : ex2_approx((la - m) * 1.4426950408889634f);
+    const float b = lb == -INFINITY ? 0.f : ex2_approx((lb - m) * 1.4426950408889634f);
+    const float inv = a + b > 0.f ? 1.f / (a + b) : 0.f;
+    float* acc = o_acc + r * D + lane * PER;
+    const __nv_bfloat16* part = o_part + r * D + lane * PER;
+    float res[PER];
+#pragma unroll
+    for (int x = 0; x < PER; ++x) {
+      const float prev = a > 0.f ? acc[x] : 0.f;     // an empty accumulator may hold anything
+      res[x] = (a * prev + b * __bfloat162float(part[x])) * inv;
+      acc[x] = res[x];
+    }
+    if (out) {
+#pragma unroll
+      for (int x = 0; x < PER; x += 2)
+        *reinterpret_cast<uint32_t*>(out + r * D + lane * PER + x) = pack_bf16x2(res[x], res[x + 1]);
+    }
+    if (lane == 0) lse_acc[r] = a + b > 0.f ? m + __logf(a + b) : -INFINITY;
+  }
+}
+
+}  // namespace attn

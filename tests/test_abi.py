@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
          "attn_status_string", "attn_selftest_timeout", "attn_fwd_window", "attn_bwd_window", "attn_decode",
-         "attn_decode_workspace_size", "attn_decode_splits"])
+         "attn_decode_workspace_size", "attn_decode_splits", "attn_merge"])
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -150,3 +150,11 @@ def test_decode_validates_before_any_launch(L):
     assert dec(q=ctypes.c_void_p(0)) == -1
     assert L.attn_decode_workspace_size(2, 8, 2, 5, 4, 128, 1) == 0
     assert L.attn_decode_splits(2, 8, 2, 5, 4, 128, 1) == 0
+
+
+def test_merge_validates_before_any_launch(L):
+    assert L.attn_merge(FAKE, FAKE, FAKE, FAKE, 10, 96, None, None) == -2
+    assert L.attn_merge(FAKE, FAKE, FAKE, FAKE, 0, 128, None, None) == -1
+    assert L.attn_merge(ctypes.c_void_p(0), FAKE, FAKE, FAKE, 10, 128, None, None) == -1
+    assert L.attn_merge(FAKE, FAKE, ODD, FAKE, 10, 128, None, None) == -3
+    assert L.attn_merge(FAKE, FAKE, FAKE, FAKE, 10, 128, ODD, None) == -3

@@ -1,0 +1,84 @@
+"""Sequence-parallel ring attention: the host logic on CPU ranks (gloo), no GPU.
+
+Each rank holds one contiguous shard of Q, K, V; the K/V shards travel around the
+ring and every partial is merged by its log-sum-exp.  Here the partial attention is
+the fp64 oracle and the merge a plain fp64 restatement of the LSE rescale, so the
+test checks the ring's schedule, its point-to-point exchange and the merge order:
+the result on every rank must equal the oracle's attention over the whole sequence.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from io_aware_exact_26_b200 import ring
+from oracle import reference as ref
+
+
+def test_schedule_covers_every_shard_once_and_masks_causally():
+    for world in (1, 2, 3, 5):
+        for rank in range(world):
+            sch = ring.ring_schedule(rank, world, causal=True)
+            assert sorted(src for _, src, _ in sch) == list(range(world))
+            for _, src, kind in sch:
+                assert kind == (ring.CAUSAL if src == rank else ring.FULL if src < rank else ring.SKIP)
+            assert all(kind == ring.FULL for _, _, kind in ring.ring_schedule(rank, world, causal=False))
+
+
+def _partial(q, k, v, causal, scale):
+    o, lse = ref.ref_fwd(q.numpy(), k.numpy(), v.numpy(), scale, causal)
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def _merge(o_acc, lse_acc, o_p, lse_p):
+    m = torch.maximum(lse_acc, lse_p)
+    a = torch.where(torch.isinf(lse_acc), torch.zeros_like(m), torch.exp(lse_acc - m))
+    b = torch.where(torch.isinf(lse_p), torch.zeros_like(m), torch.exp(lse_p - m))
+    o_acc.copy_((a[..., None] * o_acc + b[..., None] * o_p) / (a + b)[..., None])
+    lse_acc.copy_(m + torch.log(a + b))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, causal, shape, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, Hq, Hkv, N, d = shape
+        g = torch.Generator().manual_seed(1234)            # the same full problem on every rank
+        q, k, v = (torch.randn(B, h, N, d, generator=g, dtype=torch.float64) for h in (Hq, Hkv, Hkv))
+        n = N // world
+        sl = slice(rank * n, (rank + 1) * n)
+        o, lse = ring.ring_attention_fwd(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
+                                         v[:, :, sl].contiguous(), causal=causal, scale=0.4,
+                                         partial=_partial, merge=_merge, acc_dtype=torch.float64)
+        np.save(os.path.join(out_dir, f"o{rank}.npy"), o.numpy())
+        np.save(os.path.join(out_dir, f"lse{rank}.npy"), lse.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_equals_attention_over_the_whole_sequence(tmp_path, world, causal):
+    shape = (2, 4, 2, 12 * world, 5)
+    mp.start_processes(_rank_main, args=(world, _free_port(), causal, shape, str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    B, Hq, Hkv, N, d = shape
+    g = torch.Generator().manual_seed(1234)
+    q, k, v = (torch.randn(B, h, N, d, generator=g, dtype=torch.float64).numpy() for h in (Hq, Hkv, Hkv))
+    o_ref, lse_ref = ref.ref_fwd(q, k, v, 0.4, causal)
+    n = N // world
+    for r in range(world):
+        np.testing.assert_allclose(np.load(tmp_path / f"o{r}.npy"), o_ref[:, :, r * n:(r + 1) * n],
+                                   rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(np.load(tmp_path / f"lse{r}.npy"), lse_ref[:, :, r * n:(r + 1) * n],
+                                   rtol=1e-12, atol=1e-13)
