@@ -81,7 +81,10 @@ def check_grad(got, ref, what):
     _record("grad", what, err, f"{bound:.3g}", rr, ref)
     worst = np.unravel_index(np.argmax(err), err.shape)
     assert err.max() <= bound, f"{what}: max |err| {err.max():.3g} > {bound:.3g} at {worst}: got {got[worst]} ref {ref[worst]}"
-    assert rr <= G_RRMS, f"{what}: relative RMS {rr:.3g}"
+    # a gradient that is exactly zero (e.g. dQ when each row sees one key) has no
+    # relative error; the absolute gate above covers it
+    if np.any(ref != 0):
+        assert rr <= G_RRMS, f"{what}: relative RMS {rr:.3g}"
 
 
 def render_report(lines):
