@@ -160,6 +160,27 @@ def make_inputs(B, Hq, Hkv, N, d, *, seed=0, qk_std=1.0, vo_std=1.0, boost_frac=
     return out
 
 
+def make_fp8_inputs(B, Hq, Hkv, N, d, *, seed=0, qk_std=1.0, vo_std=1.0, device="cpu"):
+    """e4m3 q, k, v (torch.float8_e4m3fn) and their per-tensor descales.
+
+    Values are drawn as fp32 normals (q, k, v in that order from one seeded
+    generator), each tensor's descale is its largest magnitude over 448 (the largest
+    finite e4m3), and the codes are the values divided by the descale, cast by torch
+    (round to nearest even).  Returns {"q", "k", "v", "q_descale", "k_descale", "v_descale"}.
+    """
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    out = {}
+    for name, shape, std in (("q", (B, Hq, N, d), qk_std), ("k", (B, Hkv, N, d), qk_std),
+                             ("v", (B, Hkv, N, d), vo_std)):
+        x = torch.randn(shape, generator=gen, dtype=torch.float32, device=dev) * std
+        descale = float(x.abs().max()) / 448.0
+        out[name] = (x / descale).to(torch.float8_e4m3fn)
+        out[name + "_descale"] = descale
+    return out
+
+
 def workload_inputs(w: Workload, device="cpu", with_grad=None):
     if with_grad is None:
         with_grad = "bwd" in w.passes

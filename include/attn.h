@@ -65,6 +65,20 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
              void* stream);
 
+/* FP8 forward: as attn_fwd with Q, K and V in e4m3 (OCP FP8: 1 sign, 4 exponent
+ * bits with bias 7, 3 mantissa bits; one byte each, same [B][H][N][d] layouts) and
+ * per-tensor descales: the values attended to are q * q_descale, k * k_descale and
+ * v * v_descale.  Both products run on the tensor cores with 8-bit operands
+ * (tcgen05 kind::f8f6f4): S from the e4m3 Q and K, and O from P rounded to e4m3
+ * (round to nearest even; P <= 256 by the lazy rescale) times the e4m3 V.  The row
+ * sums and the LSE use the unrounded P, as in attn_fwd.  O is bf16, lse fp32
+ * (page "attention 的显存线性化" §五 names FP8 support for the later versions; the
+ * pages give no recipe, so the per-tensor descales are this library's reading).
+ * d must be 128 (ATTN_ERR_UNSUPPORTED otherwise); descales finite and > 0. */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int N, int d, float scale,
+                 float q_descale, float k_descale, float v_descale, int causal, void* stream);
+
 /* Local (sliding-window) forward: as attn_fwd, but query i sees only keys j with
  *     i - window_left <= j <= i + window_right
  * (page "attn-efficient", sliding-window row of the efficient-attention family

@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     NOALLOC_SCRATCH_BYTES,
     attn_bwd_workspace_size,
     attn_fwd,
+    attn_fwd_fp8,
     attn_fwd_window,
     attn_get_device_status,
     attn_selftest_timeout,

@@ -52,6 +52,8 @@ def lib():
     L.attn_decode.restype = i
     L.attn_decode_splits.argtypes = [i, i, i, i, i, i, i]
     L.attn_decode_splits.restype = i
+    L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, vp]
+    L.attn_fwd_fp8.restype = i
     L.attn_merge.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, i, vp, vp]
     L.attn_merge.restype = i
     L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
@@ -110,6 +112,28 @@ def attn_fwd(q, k, v, o=None, lse=None, *, scale=None, causal=False, stream=None
                         float(scale), int(bool(causal)), _stream_ptr(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_fp8(q, k, v, o=None, lse=None, *, q_descale, k_descale, v_descale, scale=None, causal=False,
+                 stream=None):
+    """Forward with e4m3 Q, K, V (torch.float8_e4m3fn) and per-tensor descales; returns
+    (o bf16, lse fp32).  The attended values are q * q_descale etc.; d must be 128."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.float8_e4m3fn)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if o is None else o
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(o, "o")
+    _check(lse, "lse", torch.float32)
+    if scale is None:
+        scale = d ** -0.5
+    st = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, float(scale),
+                            float(q_descale), float(k_descale), float(v_descale), int(bool(causal)),
+                            _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_fp8")
     return o, lse
 
 

@@ -35,17 +35,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D view [heads][rows][d] of a bf16 tensor; box = 64 columns x box_rows rows, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, int d, int rows, long long heads, int box_rows) {
+// 3-D view [heads][rows][d] of a bf16 (elem = 2) or 8-bit (elem = 1) tensor; box =
+// 128 bytes of columns x box_rows rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int d, int rows, long long heads, int box_rows, int elem = 2) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(heads)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(d) * 2 * rows};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem, static_cast<cuuint64_t>(d) * elem * rows};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+             const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -104,24 +106,26 @@ int next_sched_slot() {
   return static_cast<int>(n.fetch_add(1, std::memory_order_relaxed) % attn::kSchedSlots);
 }
 
-// Forward: two query tiles per CTA (fwd_pp.cuh).
-template <int D>
+// Forward: two query tiles per CTA (fwd_pp.cuh); F8: e4m3 inputs with descales
+// (qk_descale multiplies the scores, o_scale the output).
+template <int D, bool F8 = false>
 int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-               int N, float scale, Band band, cudaStream_t stream, const DeviceInfo& di) {
-  using C = attn::PpCfg<D>;
+               int N, float scale, Band band, cudaStream_t stream, const DeviceInfo& di, float qk_descale = 1.f,
+               float o_scale = 1.f) {
+  using C = attn::PpCfg<D, F8>;
   static std::once_flag attr_once[64];
   static bool attr_ok[64];
   int dev = 0;
   cudaGetDevice(&dev);
   std::call_once(attr_once[dev], [&] {
-    attr_ok[dev] = cudaFuncSetAttribute(attn::attn_fwd_pp_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::kSmem) == cudaSuccess;
+    attr_ok[dev] = cudaFuncSetAttribute(attn::attn_fwd_pp_kernel<D, F8>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) == cudaSuccess;
   });
   if (!attr_ok[dev]) return ATTN_ERR_LAUNCH;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, D, N, static_cast<long long>(B) * Hq, 128) ||
-      !make_map(&tk, k, D, N, static_cast<long long>(B) * Hkv, 128) ||
-      !make_map(&tv, v, D, N, static_cast<long long>(B) * Hkv, 128))
+  if (!make_map(&tq, q, D, N, static_cast<long long>(B) * Hq, 128, C::ES) ||
+      !make_map(&tk, k, D, N, static_cast<long long>(B) * Hkv, 128, C::ES) ||
+      !make_map(&tv, v, D, N, static_cast<long long>(B) * Hkv, 128, C::ES))
     return ATTN_ERR_LAUNCH;
   attn::FwdParams p;
   p.o = o;
@@ -132,7 +136,8 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   p.N = N;
   p.G = Hq / Hkv;
   p.n_qtiles = (N + 127) / 128;
-  p.c = attn::folded_scale(scale);
+  p.c = attn::folded_scale(scale * qk_descale);
+  p.oscale = o_scale;
   p.wl = band.wl;
   p.wr = band.wr;
   p.desc = band.wr <= band.wl;
@@ -140,7 +145,7 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   const int grid = units < di.sms ? units : di.sms;
   p.sched_slot = next_sched_slot();
   attn::sched_reset_kernel<<<1, 32, 0, stream>>>(p.sched_slot);
-  attn::attn_fwd_pp_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  attn::attn_fwd_pp_kernel<D, F8><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -393,6 +398,23 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
                     int N, int d, float scale, int window_left, int window_right, void* stream) {
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, 0, band_of_window(N, window_left, window_right),
                   stream);
+}
+
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                 int d, float scale, float q_descale, float k_descale, float v_descale, int causal, void* stream) {
+  int st = check_common(B, Hq, Hkv, N, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  for (float x : {q_descale, k_descale, v_descale})
+    if (!std::isfinite(x) || !(x > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale * q_descale * k_descale)) return ATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
+  return launch_fwd_pp<128, true>(q, k, v, o, lse, B, Hq, Hkv, N, scale, band_of_causal(N, causal),
+                                  static_cast<cudaStream_t>(stream), *di, q_descale * k_descale, v_descale);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int causal) {

@@ -34,7 +34,8 @@ struct FwdParams {
   float* lse;
   int B, Hq, Hkv, N, G;
   int n_qtiles;
-  float c;          // scale * log2(e)
+  float c;          // scale * log2(e) (with the Q and K descales for e4m3 inputs)
+  float oscale;     // output multiplier: V's descale for e4m3 inputs, else 1
   int wl, wr;       // window: 0 <= wl, wr <= N
   int desc;         // list query tiles last-first (their key ranges grow with the tile)
   int sched_slot;   // g_sched slot this launch claims work units from

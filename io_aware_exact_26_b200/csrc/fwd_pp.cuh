@@ -38,10 +38,18 @@
 
 namespace attn {
 
-template <int D>
+// F8 = false: bf16 Q, K, V and P (kind::f16).  F8 = true: e4m3 Q, K, V and P
+// (kind::f8f6f4), each tile row of d bytes, with per-tensor descales folded into
+// the exponent scale (Q, K) and the output (V).
+template <int D, bool F8 = false>
 struct PpCfg {
-  static constexpr int kTile = 128 * D * 2;
-  static constexpr int kBox = 128 * 128;
+  static constexpr int ES = F8 ? 1 : 2;                 // bytes per element
+  static constexpr int kTile = 128 * D * ES;
+  static constexpr int kBox = 128 * 128;                // one TMA box: 128 rows x 128 bytes
+  static constexpr int NB = D * ES / 128;               // boxes per tile
+  static constexpr int KS = D * ES / 32;                // S = Q K^T: 32-byte K steps
+  static constexpr int PVK = F8 ? 32 : 16;              // keys per P V instruction
+  static_assert(NB >= 1, "a tile row must fill one 128-byte swizzle row");
   static constexpr int KST = 2;
   static constexpr int VST = 2;
   static constexpr int kThreads = 576;
@@ -53,7 +61,7 @@ struct PpCfg {
   // Q buffers per team: two at d = 64, so the next unit's Q loads while the current
   // unit still reads its own (short units, e.g. N = 1024, would wait for it); one
   // at d = 128, where shared memory has no room and units are longer.
-  static constexpr int QST = (D == 64) ? 2 : 1;
+  static constexpr int QST = (kTile <= 16384) ? 2 : 1;
   static constexpr int kOffQ = 0;                       // Q slots [team][QST]
   static constexpr int kOffK = 2 * QST * kTile;
   static constexpr int kOffV = kOffK + KST * kTile;
@@ -127,11 +135,11 @@ __device__ __forceinline__ int pp_units(const FwdParams& p) {
   return p.B * p.Hkv * ((p.G * p.n_qtiles + 1) >> 1);
 }
 
-template <int D>
+template <int D, bool F8 = false>
 __global__ void __launch_bounds__(576, 1)
     attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
-  using C = PpCfg<D>;
+  using C = PpCfg<D, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   PpShared& sh = *reinterpret_cast<PpShared*>(smem + C::kOffSh);
@@ -188,8 +196,8 @@ __global__ void __launch_bounds__(576, 1)
           const int qs = uq % C::QST;
           if (uq >= C::QST && !mbar_wait(&sh.q_empty[x][qs], ((uq / C::QST) - 1) & 1)) return false;
           mbar_arrive_expect_tx(&sh.q_full[x][qs], C::kTile);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ + (x * C::QST + qs) * C::kTile + c * C::kBox, &tmq, &sh.q_full[x][qs], c * 64,
+          for (int c = 0; c < C::NB; ++c)
+            tma_load_3d(sQ + (x * C::QST + qs) * C::kTile + c * C::kBox, &tmq, &sh.q_full[x][qs], c * 128 / C::ES,
                         w.qt(x) * 128, w.bh(x));
           return true;
         };
@@ -200,13 +208,13 @@ __global__ void __launch_bounds__(576, 1)
           if (kc >= 2) ok = mbar_wait(&sh.k_empty[st], ((kc >> 1) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, j * 128, w.bkv);
+          for (int c = 0; c < C::NB; ++c)
+            tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 128 / C::ES, j * 128, w.bkv);
           if (kc >= 2) ok = mbar_wait(&sh.v_empty[st], ((kc >> 1) - 1) & 1);
           if (!ok) { nk = kc + 1; break; }
           mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sV + st * C::kTile + c * C::kBox, &tmv, &sh.v_full[st], c * 64, j * 128, w.bkv);
+          for (int c = 0; c < C::NB; ++c)
+            tma_load_3d(sV + st * C::kTile + c * C::kBox, &tmv, &sh.v_full[st], c * 128 / C::ES, j * 128, w.bkv);
           nk = kc + 1;
         }
       }
@@ -222,8 +230,8 @@ __global__ void __launch_bounds__(576, 1)
     // Per step j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_X(j+1) waits for PV_X(j)
     // (the P it overwrites); meanwhile the tensor cores run the other team's work.
     const bool leader = elect_one();
-    constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-    constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
+    constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t idO = F8 ? idesc_e4m3_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
     constexpr uint32_t hi = sdesc_hi_sw128(1024);
     const uint32_t q_lo0 = sdesc_lo(smem_u32(sQ), 16);
     const uint32_t k_lo0 = sdesc_lo(smem_u32(sK), 16);
@@ -241,9 +249,12 @@ __global__ void __launch_bounds__(576, 1)
         const uint32_t q_lo = q_lo0 + (x * C::QST + qs) * (C::kTile >> 4);
         const uint32_t k_lo = k_lo0 + st * (C::kTile >> 4);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < C::KS; ++k) {
           const uint32_t off = ((k >> 2) * C::kBox + (k & 3) * 32) >> 4;
-          umma_ss_lo(tmem + (x ? C::kS1 : C::kS0), q_lo + off, k_lo + off, hi, idS, k > 0);
+          if constexpr (F8)
+            umma_ss_f8_lo(tmem + (x ? C::kS1 : C::kS0), q_lo + off, k_lo + off, hi, idS, k > 0);
+          else
+            umma_ss_lo(tmem + (x ? C::kS1 : C::kS0), q_lo + off, k_lo + off, hi, idS, k > 0);
         }
         umma_commit(&sh.s_full[x]);
         if (last) umma_commit(&sh.q_empty[x][qs]);
@@ -255,10 +266,19 @@ __global__ void __launch_bounds__(576, 1)
       if (leader) {
         const uint32_t v_lo = v_lo0 + st * (C::kTile >> 4);
         const uint32_t sbase = tmem + (x ? C::kS1 : C::kS0);
+        // P of keys [k * PVK, (k + 1) * PVK) sits in 8 TMEM columns: keys 0-63 from column
+        // 0, keys 64-127 from column 64 (bf16: 2 per column, e4m3: 4 per column)
+        if constexpr (F8) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          umma_ts_lo(tmem + (x ? C::kO1 : C::kO0), sbase + (k >> 2) * 64 + (k & 3) * 8, v_lo + ((k * 2048) >> 4), hi,
-                     idO, !(first && k == 0));
+          for (int k = 0; k < 4; ++k)
+            umma_ts_f8_lo(tmem + (x ? C::kO1 : C::kO0), sbase + (k >> 1) * 64 + (k & 1) * 8,
+                          v_lo + ((k * C::PVK * 128) >> 4), hi, idO, !(first && k == 0));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_ts_lo(tmem + (x ? C::kO1 : C::kO0), sbase + (k >> 2) * 64 + (k & 3) * 8,
+                       v_lo + ((k * C::PVK * 128) >> 4), hi, idO, !(first && k == 0));
+        }
         umma_commit(&sh.pv_done[x]);
       }
       __syncwarp();
@@ -465,9 +485,20 @@ __global__ void __launch_bounds__(576, 1)
               b = ex2_approx(x1);
             }
             lsum = fadd2(lsum, f2pack(a, b));
-            pk[k] = pack_bf16x2(a, b);
+            if constexpr (F8) {
+              // four e4m3 per column, lowest key in the low byte; p <= 2^tau = 256 < 448
+              const uint32_t two = pack_e4m3x2(a, b);
+              pk[k >> 1] = (k & 1) ? (pk[k >> 1] | (two << 16)) : two;
+            } else {
+              pk[k] = pack_bf16x2(a, b);
+            }
           }
-          tmem_st8(s_base + cc * 8, pk);
+          if constexpr (F8) {
+            const uint32_t (&p4)[4] = *reinterpret_cast<const uint32_t (*)[4]>(pk);
+            tmem_st4(s_base + cc * 4, p4);
+          } else {
+            tmem_st8(s_base + cc * 8, pk);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -488,7 +519,7 @@ __global__ void __launch_bounds__(576, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.pv_done[x], glast & 1));
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = p.oscale / l;      // oscale: V's descale (1 for bf16)
       const bool live = qrow < p.N;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D + grp * OH;
 #pragma unroll 1

@@ -155,6 +155,27 @@ def ref_decode(q, k, v, scale, causal):
     return ref_fwd(q, k, v, scale, False, window=(None, nk - nq) if causal else None)
 
 
+def decode_e4m3(codes):
+    """Values of e4m3 bytes (OCP FP8 E4M3: sign bit, 4 exponent bits with bias 7, 3
+    mantissa bits; exponent 0 is subnormal, m/8 * 2^-6; the all-ones pattern
+    S.1111.111 is NaN; there are no infinities), as float64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return sign * val
+
+
+def ref_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale, causal):
+    """Forward oracle for e4m3 inputs: the plain definition on the values they stand
+    for, q = decode(q8) * q_descale (likewise k, v), in fp64.  q8/k8/v8 are the raw
+    bytes (uint8 arrays)."""
+    return ref_fwd(decode_e4m3(q8) * q_descale, decode_e4m3(k8) * k_descale, decode_e4m3(v8) * v_descale,
+                   scale, causal)
+
+
 def online_fwd_head(qh, kh, vh, scale, causal, bounds, window=None):
     """The pages' blockwise online softmax for one head (used only in self-tests).
 

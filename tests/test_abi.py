@@ -21,14 +21,14 @@ def L():
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "attn.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
          "attn_status_string", "attn_selftest_timeout", "attn_fwd_window", "attn_bwd_window", "attn_decode",
-         "attn_decode_workspace_size", "attn_decode_splits", "attn_merge"])
+         "attn_decode_workspace_size", "attn_decode_splits", "attn_merge", "attn_fwd_fp8"])
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -158,3 +158,15 @@ def test_merge_validates_before_any_launch(L):
     assert L.attn_merge(ctypes.c_void_p(0), FAKE, FAKE, FAKE, 10, 128, None, None) == -1
     assert L.attn_merge(FAKE, FAKE, ODD, FAKE, 10, 128, None, None) == -3
     assert L.attn_merge(FAKE, FAKE, FAKE, FAKE, 10, 128, ODD, None) == -3
+
+
+def test_fp8_forward_validates_before_any_launch(L):
+    def f8(q=FAKE, d=128, dq=0.01, dk=0.01, dv=0.01, scale=0.088, N=256):
+        return L.attn_fwd_fp8(q, FAKE, FAKE, FAKE, FAKE, 1, 2, 1, N, d, scale, dq, dk, dv, 1, None)
+    assert f8(d=64) == -2                 # e4m3 tiles need 128-byte rows
+    assert f8(dq=0.0) == -1
+    assert f8(dk=-1.0) == -1
+    assert f8(dv=float("inf")) == -1
+    assert f8(N=0) == -1
+    assert f8(q=ODD) == -3
+    assert f8(q=ctypes.c_void_p(0)) == -1

@@ -453,3 +453,25 @@ def test_decode_partials_merge_by_lse():
     o_m = sum(wi[:, None] * p[0] for wi, p in zip(w, parts)) / sum(w)[:, None]
     np.testing.assert_allclose(o_m, o, rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(lse_m, lse, rtol=1e-13)
+
+
+# ---------------------------------------------------------------- e4m3 inputs
+def test_e4m3_decoding_matches_torch_on_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = ref.decode_e4m3(codes)
+    theirs = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(theirs)
+    assert nan.sum() == 2 and np.array_equal(np.isnan(ours), nan)          # 0x7f, 0xff
+    np.testing.assert_array_equal(ours[~nan], theirs[~nan])
+    assert ours[0x7e] == 448.0 and ours[0x01] == 2.0 ** -9 and ours[0x38] == 1.0 and ours[0xb8] == -1.0
+
+
+def test_fp8_oracle_is_the_definition_on_the_dequantised_values():
+    from attn_inputs import make_fp8_inputs
+    x = make_fp8_inputs(1, 2, 1, 9, 4, seed=5)
+    q8, k8, v8 = (x[n].view(torch.uint8).numpy() for n in ("q", "k", "v"))
+    o, lse = ref.ref_fwd_fp8(q8, k8, v8, x["q_descale"], x["k_descale"], x["v_descale"], 0.5, True)
+    qf, kf, vf = (x[n].to(torch.float64).numpy() * x[n + "_descale"] for n in ("q", "k", "v"))
+    ob, lseb = obuild.brute_fwd(qf, kf, vf, 0.5, True)
+    np.testing.assert_allclose(o, ob, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lseb, rtol=1e-12, atol=1e-13)
