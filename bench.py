@@ -416,6 +416,58 @@ def run_decode(args):
         torch.cuda.empty_cache()
 
 
+def run_fp8(args):
+    """FP8 forward (e4m3 inputs) next to the bf16 forward on the same shapes, timed apart.
+    The fp8 roofline peak is the measured bf16 dense peak times the nominal fp8 : bf16
+    ratio of 2 (4.5 vs 2.25 PFLOP/s dense)."""
+    import torch
+    import io_aware_exact_26_b200 as attn
+    from attn_inputs import make_fp8_inputs
+
+    peaks, peaks_kind = load_peaks()
+    peak16 = float(peaks["bf16_tflops"])
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    for name in ("causal_b8_h16_n4096_d128", "long_causal_b1_h32_n32768_d128", "gqa_causal_b4_hq32_hkv8_n8192_d128"):
+        w = WORKLOADS[name]
+        x8 = make_fp8_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, qk_std=w.qk_std, device=dev)
+        x16 = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, qk_std=w.qk_std, vo_std=w.vo_std,
+                          boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=False)
+        o = torch.empty(x16["q"].shape, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        calls = {
+            "fp8": lambda: attn.attn_fwd_fp8(x8["q"], x8["k"], x8["v"], o, lse, q_descale=x8["q_descale"],
+                                             k_descale=x8["k_descale"], v_descale=x8["v_descale"], causal=w.causal),
+            "bf16": lambda: attn.attn_fwd(x16["q"], x16["k"], x16["v"], o, lse, scale=w.scale, causal=w.causal)}
+        f_fwd = acc.flops_fwd(w.B, w.Hq, w.N, w.d, w.causal)
+        line = {"fp8_forward": name, "reps": args.sweep_reps, "warmup": args.warmup}
+        sampler = ClockSampler(0)
+        sampler.start()
+        for kind, fn in calls.items():
+            for _ in range(args.warmup):
+                fn()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.sweep_reps)]
+            for a, b in evs:
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+            tf = f_fwd / (ms * 1e-3) / 1e12
+            peak = peak16 * (2 if kind == "fp8" else 1)
+            line[kind] = {"ms": round(ms, 4), "tflops": round(tf, 1), "peak": peak, "frac": round(tf / peak, 4),
+                          "peak_source": f"{peaks_kind} bf16 dense (burst)" + (" x 2 (nominal fp8:bf16)" if kind == "fp8"
+                                                                             else "")}
+        line["clocks"] = sampler.stop()
+        if attn.attn_get_device_status() != 0:
+            raise SystemExit(f"device-side error in the fp8 run at {name}")
+        print(json.dumps(line), flush=True)
+        del x8, x16, o, lse
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -429,6 +481,7 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="time the sequence-length sweep, one line per point")
     ap.add_argument("--sweep-reps", type=int, default=50)
     ap.add_argument("--decode", action="store_true", help="time split-KV decoding, one line per decode workload")
+    ap.add_argument("--fp8", action="store_true", help="time the fp8 forward next to the bf16 forward")
     ap.add_argument("--decode-workload", default=None, choices=sorted(DECODE_WORKLOADS))
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -437,6 +490,9 @@ def main():
         return
     if args.decode:
         run_decode(args)
+        return
+    if args.fp8:
+        run_fp8(args)
         return
 
     rank = int(os.environ.get("RANK", "0"))

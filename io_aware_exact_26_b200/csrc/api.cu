@@ -323,8 +323,8 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   int grid = p.total_items < sms ? p.total_items : sms;
   attn_bwd_kv_kernel<D><<<grid, KvCfg<D>::kThreads, KvCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
   if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  // dQ: one item per (b, q-head, query tile)
-  p.total_items = B * Hq * nt;
+  // dQ: one item per (b, q-head, query tile); causal: units of two query tiles
+  p.total_items = B * Hq * (p.pair ? p.npair : nt);
   grid = p.total_items < sms ? p.total_items : sms;
   attn_bwd_q_kernel<D><<<grid, QCfg<D>::kThreads, QCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;

@@ -570,16 +570,28 @@ struct QShared {
   uint32_t tmem_base;
 };
 
-// item t -> (bh_q, query tile i).  Numbered KV head by KV head (the G query heads
-// of a group interleaved), so CTAs running at the same time share K/V in L2;
-// longest rows first within a group when key ranges grow with the tile (causal).
-__device__ __forceinline__ void q_item(const BwdParams& p, int t, int& bhq, int& i) {
-  const int per_group = p.G * p.nt;
-  const int gk = t / per_group;                  // b * Hkv + kv-head
-  const int r = t - gk * per_group;
+// Work units of the dQ kernel, numbered KV head by KV head (the G query heads of a
+// group interleaved), so CTAs running at the same time share K/V in L2.
+//  - In general unit t is one query tile (longest rows first within a group when
+//    key ranges grow with the tile).
+//  - Causal: unit t is the pair of query tiles (nt-1-pr, pr), two items (one for
+//    the middle tile when nt is odd), which together see nt+1 key tiles whatever pr
+//    is, so units cost the same and a static round-robin over them stays balanced.
+__device__ __forceinline__ int q_halves(const BwdParams& p, int t) {
+  if (!p.pair) return 1;
+  const int pr = (t / p.G) % p.npair;
+  return 2 * pr + 1 == p.nt ? 1 : 2;
+}
+__device__ __forceinline__ void q_item(const BwdParams& p, int t, int hf, int& bhq, int& i) {
+  const int units = p.G * (p.pair ? p.npair : p.nt);   // per (b, kv-head)
+  const int gk = t / units;                             // b * Hkv + kv-head
+  const int r = t - gk * units;
   const int rq = r / p.G;
   const int hin = r - rq * p.G;
-  i = p.desc ? (p.nt - 1 - rq) : rq;
+  if (p.pair)
+    i = hf ? rq : p.nt - 1 - rq;
+  else
+    i = p.desc ? (p.nt - 1 - rq) : rq;
   bhq = (gk / p.Hkv) * p.Hq + (gk % p.Hkv) * p.G + hin;
 }
 // Key tiles [j0, j0 + n) that query tile i sees: keys i - wl .. i + wr.
@@ -634,9 +646,10 @@ __global__ void __launch_bounds__(352, 1)
       tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmdo);
       int gj = 0, it = 0, nk = 0, nqd = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
+      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
+      for (int hf = 0; hf < q_halves(p, t) && ok; ++hf, ++it) {
         int bhq, i;
-        q_item(p, t, bhq, i);
+        q_item(p, t, hf, bhq, i);
         const int bkv = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / p.G;
         int j0, n_kv;
         q_kv_range(p, i, j0, n_kv);
@@ -670,9 +683,10 @@ __global__ void __launch_bounds__(352, 1)
       tma_prefetch_desc(&tmv);
       int gj = 0, nv = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x) {
+      for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
+      for (int hf = 0; hf < q_halves(p, t) && ok; ++hf) {
         int bhq, i;
-        q_item(p, t, bhq, i);
+        q_item(p, t, hf, bhq, i);
         const int bkv = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / p.G;
         int j0, n_kv;
         q_kv_range(p, i, j0, n_kv);
@@ -742,9 +756,10 @@ __global__ void __launch_bounds__(352, 1)
       __syncwarp();
       return true;
     };
-    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x, ++it) {
+    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
+    for (int hf = 0; hf < q_halves(p, t) && ok; ++hf, ++it) {
       int bhq, i;
-      q_item(p, t, bhq, i);
+      q_item(p, t, hf, bhq, i);
       int j0, n_kv;
       q_kv_range(p, i, j0, n_kv);
       ok = wait(&sh.qdo_full, it & 1);
@@ -790,9 +805,10 @@ __global__ void __launch_bounds__(352, 1)
     const float c = p.c;
     int gj = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x) {
+    for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
+    for (int hf = 0; hf < q_halves(p, t) && ok; ++hf) {
       int bhq, i;
-      q_item(p, t, bhq, i);
+      q_item(p, t, hf, bhq, i);
       int j0, n_kv;
       q_kv_range(p, i, j0, n_kv);
       const int qrow = i * 128 + r;
