@@ -52,7 +52,8 @@ typedef enum {
   ATTN_ERR_LAUNCH = -4,        /* the CUDA runtime refused a launch or an attribute */
   ATTN_ERR_DEVICE_TIMEOUT = -5,/* a bounded device wait expired (see attn_get_device_status) */
   ATTN_ERR_WORKSPACE = -6,     /* backward workspace too small (or beyond the no-alloc scratch) */
-  ATTN_ERR_ALLOC = -7          /* the library's own stream-ordered allocation failed */
+  ATTN_ERR_ALLOC = -7,         /* the library's own stream-ordered allocation failed */
+  ATTN_ERR_DEVICE_BOUNDS = -8  /* checking build only: a kernel computed an index outside its tensor */
 } attn_status_t;
 
 /* Forward: O and LSE for every (b, h, i).
@@ -186,12 +187,28 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                      void* stream);
 
 /* Synchronises `stream`, then returns ATTN_OK if no kernel of this library
- * recorded a device-side error since the last call, else ATTN_ERR_DEVICE_TIMEOUT;
- * the error word is cleared.  While the word is set, later launches exit early. */
+ * recorded a device-side error since the last call, else ATTN_ERR_DEVICE_TIMEOUT
+ * (a bounded wait expired) or ATTN_ERR_DEVICE_BOUNDS (checking build: an index
+ * check failed); the error word is cleared.  While the word is set, later launches
+ * exit early. */
 int attn_get_device_status(void* stream);
 
 /* Static, human-readable text for a status code. */
 const char* attn_status_string(int status);
+
+/* Checking build (no counterpart on the pages).  The library also comes as
+ * libattn_b200_checks.so, compiled with ATTN_CHECKS: its kernels test every tile
+ * coordinate, head index and global row they compute against the tensor it
+ * addresses; an index out of range records ATTN_ERR_DEVICE_BOUNDS in the error word
+ * and the access is skipped or kept inside the tensor -- no trap, no assert.  It
+ * stands in for a memory checker where none can run.
+ * attn_checks_enabled returns 1 in that build, 0 in the normal one.
+ * attn_selftest_bounds launches one CTA that hands the check an index outside its
+ * range (nothing is accessed with it): in the checking build the following
+ * attn_get_device_status() returns ATTN_ERR_DEVICE_BOUNDS, in the normal build
+ * ATTN_OK.  Returns ATTN_ERR_LAUNCH if the launch is refused, else ATTN_OK. */
+int attn_checks_enabled(void);
+int attn_selftest_bounds(void* stream);
 
 /* Diagnostic (no counterpart on the pages): exercises the device-side failure
  * path that every kernel of this library uses.  Launches one CTA on `stream`

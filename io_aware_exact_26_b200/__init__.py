@@ -20,7 +20,11 @@ from .binding import (  # noqa: F401
     attn_fwd_fp8,
     attn_fwd_window,
     attn_get_device_status,
+    attn_checks_enabled,
+    attn_selftest_bounds,
     attn_selftest_timeout,
+    checks_library_path,
+    use_library,
     attn_status_string,
     lib,
     library_path,

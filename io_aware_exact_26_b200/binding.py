@@ -27,14 +27,42 @@ class AttnError(RuntimeError):
         super().__init__(f"{what}: {attn_status_string(status)} ({status})")
 
 
+checks_library_path = os.path.join(_HERE, "libattn_b200_checks.so")
+
+
 def lib():
     """Load libattn_b200.so (built by ``__graft_entry__.build()``); raise if it is missing."""
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(library_path):
-        raise ImportError(f"{library_path} is not built; run __graft_entry__.build()")
-    L = ctypes.CDLL(library_path)
+    _lib = load(library_path)
+    return _lib
+
+
+class use_library:
+    """Context manager: route every call of this module through another build of the
+    library (e.g. ``checks_library_path``), then restore the previous one."""
+
+    def __init__(self, path):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.prev = _lib
+        _lib = load(self.path)
+        return _lib
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.prev
+        return False
+
+
+def load(path):
+    """ctypes handle on a build of the library with every entry point's signature set."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run __graft_entry__.build()")
+    L = ctypes.CDLL(path)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     L.attn_fwd.restype = i
@@ -64,7 +92,10 @@ def lib():
     L.attn_status_string.restype = ctypes.c_char_p
     L.attn_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
     L.attn_selftest_timeout.restype = i
-    _lib = L
+    L.attn_checks_enabled.argtypes = []
+    L.attn_checks_enabled.restype = i
+    L.attn_selftest_bounds.argtypes = [vp]
+    L.attn_selftest_bounds.restype = i
     return L
 
 
@@ -309,3 +340,14 @@ def attn_selftest_timeout(limit_ns: int, stream=None) -> None:
 def attn_get_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device-side error word."""
     return int(lib().attn_get_device_status(_stream_ptr(stream)))
+
+
+def attn_selftest_bounds(stream=None) -> None:
+    """Launch the index-check self-test (records a bounds failure in the checking build only)."""
+    st = int(lib().attn_selftest_bounds(_stream_ptr(stream)))
+    if st != 0:
+        raise AttnError(st, "attn_selftest_bounds")
+
+
+def attn_checks_enabled() -> bool:
+    return bool(lib().attn_checks_enabled())

@@ -27,16 +27,29 @@ def nvcc():
     return "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    newest = max(os.path.getmtime(f) for f in SOURCES + HEADERS)
-    if not force and os.path.exists(OUT) and os.path.getmtime(OUT) >= newest:
-        return OUT
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-I", CSRC, *SOURCES, "-o", OUT + ".tmp"]
+# The checking build: the same sources with ATTN_CHECKS, whose kernels test every index
+# they compute and record failures in the error word (see include/attn.h).
+OUT_CHECKS = os.path.join(HERE, "libattn_b200_checks.so")
+
+
+def _build_one(out, extra, force, verbose):
+    newest = max(os.path.getmtime(f) for f in SOURCES + HEADERS + [__file__])
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= newest:
+        return out
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-I", CSRC, *SOURCES, "-o", out + ".tmp"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
-    os.replace(OUT + ".tmp", OUT)
-    return OUT
+    os.replace(out + ".tmp", out)
+    return out
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    return _build_one(OUT, [], force, verbose)
+
+
+def build_checks(force: bool = False) -> str:
+    return _build_one(OUT_CHECKS, ["-DATTN_CHECKS"], force, False)
 
 
 if __name__ == "__main__":

@@ -567,6 +567,10 @@ __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) (void)attn::mbar_wait_for(&bar, 0, limit_ns);
 }
+// Hands the index check a value outside its range; nothing is accessed with it.
+__global__ void selftest_bounds_kernel() {
+  if (threadIdx.x == 0) (void)attn::in_range(5, 3);
+}
 }  // namespace
 
 extern "C" {
@@ -583,7 +587,14 @@ int attn_get_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&v, attn::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
   if (v != 0 && cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
-  return v == 0 ? ATTN_OK : ATTN_ERR_DEVICE_TIMEOUT;
+  return v == 0 ? ATTN_OK : v == 2 ? ATTN_ERR_DEVICE_BOUNDS : ATTN_ERR_DEVICE_TIMEOUT;
+}
+
+int attn_checks_enabled(void) { return attn::kChecks ? 1 : 0; }
+
+int attn_selftest_bounds(void* stream) {
+  selftest_bounds_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
 const char* attn_status_string(int status) {
@@ -595,7 +606,8 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_LAUNCH: return "CUDA launch or attribute error";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
     case ATTN_ERR_WORKSPACE: return "backward workspace too small";
-    case ATTN_ERR_ALLOC: return "stream-ordered allocation of the backward workspace failed";
+    case ATTN_ERR_ALLOC: return "stream-ordered allocation of the library's workspace failed";
+    case ATTN_ERR_DEVICE_BOUNDS: return "a device-side index check failed (checking build)";
     default: return "unknown status";
   }
 }

@@ -271,6 +271,8 @@ __global__ void __launch_bounds__(320, 1)
         if (it >= 1) ok = mbar_wait(&sh.kv_empty, (it - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&sh.kv_full, 2 * C::kTile);
+        in_range(j, p.nt);
+        in_range(bhkv, static_cast<long long>(p.B) * p.Hkv);
         for (int c = 0; c < D / 64; ++c) {                  // K_j, V_j: read by this item only
           tma_load_3d_hint(sK + c * C::kBox, &tmk, &sh.kv_full, c * 64, j * 128, bhkv, pol_once);
           tma_load_3d_hint(sV + c * C::kBox, &tmv, &sh.kv_full, c * 64, j * 128, bhkv, pol_once);
@@ -294,7 +296,9 @@ __global__ void __launch_bounds__(320, 1)
               tma_load_3d_hint(sDO + st * C::kTile + c * C::kBox, &tmdo, &sh.qdo_full[st], c * 64, i * 128, bhq,
                                pol_reuse);
             }
-            const size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + i * 128;
+            size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + i * 128;
+            in_range(i, p.nt);
+            if (!in_range(bhq, static_cast<long long>(p.B) * p.Hq)) vrow = 0;   // keep the bulk copy inside
             bulk_load(sVec + st * 256, p.lse2 + vrow, 512, &sh.qdo_full[st]);
             bulk_load(sVec + st * 256 + 128, p.dd + vrow, 512, &sh.qdo_full[st]);
             nq = gs + 1;
@@ -503,7 +507,7 @@ __global__ void __launch_bounds__(320, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.k_done, (gs - 1) & 1));
       if (!ok) break;
       tc_fence_after();
-      const bool live = key < p.N;
+      const bool live = key < p.N && in_range(bhkv, static_cast<long long>(p.B) * p.Hkv);
       const float mul = hb == 0 ? 1.f : p.scale;
       __nv_bfloat16* dst = (hb == 0 ? p.dv : p.dk) + (static_cast<size_t>(bhkv) * p.N + key) * D;
       const uint32_t col = hb == 0 ? C::kDV : C::kDK;
@@ -656,6 +660,8 @@ __global__ void __launch_bounds__(352, 1)
         if (it >= 1) ok = mbar_wait(&sh.qdo_empty, (it - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&sh.qdo_full, 2 * C::kTile);
+        in_range(i, p.nt);
+        in_range(bhq, static_cast<long long>(p.B) * p.Hq);
         for (int c = 0; c < D / 64; ++c) {
           tma_load_3d(sQ + c * C::kBox, &tmq, &sh.qdo_full, c * 64, i * 128, bhq);
           tma_load_3d(sDO + c * C::kBox, &tmdo, &sh.qdo_full, c * 64, i * 128, bhq);
@@ -666,6 +672,8 @@ __global__ void __launch_bounds__(352, 1)
           if (g >= C::KVST) ok = mbar_wait(&sh.k_empty[st], ((g / C::KVST) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
+          in_range(j0 + j, p.nt);
+          in_range(bkv, static_cast<long long>(p.B) * p.Hkv);
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, (j0 + j) * 128, bkv);
           nk = g + 1;
@@ -812,7 +820,8 @@ __global__ void __launch_bounds__(352, 1)
       int j0, n_kv;
       q_kv_range(p, i, j0, n_kv);
       const int qrow = i * 128 + r;
-      const size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + qrow;
+      size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + qrow;
+      if (!in_range(static_cast<long long>(vrow), static_cast<long long>(p.B) * p.Hq * p.nt * 128)) vrow = 0;
       const float l2 = p.lse2[vrow], drow = p.dd[vrow];
       float lv[16];
 #pragma unroll
@@ -870,7 +879,7 @@ __global__ void __launch_bounds__(352, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.q_done[glast & 1], (glast >> 1) & 1));
       if (!ok) break;
       tc_fence_after();
-      const bool live = qrow < p.N;
+      const bool live = qrow < p.N && in_range(bhq, static_cast<long long>(p.B) * p.Hq);
       __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bhq) * p.N + qrow) * D;
 #pragma unroll 1
       for (int q4 = hb; q4 < D / 32; q4 += 2) {

@@ -166,9 +166,9 @@ __global__ void __launch_bounds__(320, 1)
           const int h = t / p.R, i = t - h * p.R;
           const int qi = w.qb * p.R + i;
           uint4 val = make_uint4(0u, 0u, 0u, 0u);
-          if (h < p.G && qi < p.Nq)
-            val = *reinterpret_cast<const uint4*>(
-                p.q + ((static_cast<size_t>(b) * p.Hq + g * p.G + h) * p.Nq + qi) * D + c8 * 8);
+          const size_t qoff = ((static_cast<size_t>(b) * p.Hq + g * p.G + h) * p.Nq + qi) * D + c8 * 8;
+          if (h < p.G && qi < p.Nq && in_range(static_cast<long long>(qoff), static_cast<long long>(p.B) * p.Hq * p.Nq * D))
+            val = *reinterpret_cast<const uint4*>(p.q + qoff);
           // 128B swizzle: 16-byte chunk cc of row t lands at chunk cc ^ (t & 7) of the row
           const int box = c8 >> 3, cc = c8 & 7;
           *reinterpret_cast<uint4*>(dst0 + box * C::kBox + t * 128 + ((cc ^ (t & 7)) << 4)) = val;
@@ -184,6 +184,8 @@ __global__ void __launch_bounds__(320, 1)
           if (kc >= 2) ok = mbar_wait(&sh.k_empty[st], ((kc >> 1) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
+          in_range(w.j0 + j, (p.Nk + 127) / 128);
+          in_range(w.bg, static_cast<long long>(p.B) * p.Hkv);
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 64, (w.j0 + j) * 128, w.bg);
           if (kc >= 2) ok = mbar_wait(&sh.v_empty[st], ((kc >> 1) - 1) & 1);
@@ -305,7 +307,8 @@ __global__ void __launch_bounds__(320, 1)
       if (u < 0) break;
       const DecUnit w = dec_unit(p, u);
       const int qi = w.qb * p.R + i;
-      const bool valid = h < p.G && qi < p.Nq;
+      const bool valid = h < p.G && qi < p.Nq && in_range(w.bg, static_cast<long long>(p.B) * p.Hkv) &&
+                         in_range(w.s, p.S);
       const int b = w.bg / p.Hkv, g = w.bg - b * p.Hkv;
       const size_t qrow = (static_cast<size_t>(b) * p.Hq + g * p.G + h) * p.Nq + qi;   // global query row
       if (w.n == 0) {                  // no visible key in this split: an empty partial

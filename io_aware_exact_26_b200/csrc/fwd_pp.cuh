@@ -196,6 +196,8 @@ __global__ void __launch_bounds__(576, 1)
           const int qs = uq % C::QST;
           if (uq >= C::QST && !mbar_wait(&sh.q_empty[x][qs], ((uq / C::QST) - 1) & 1)) return false;
           mbar_arrive_expect_tx(&sh.q_full[x][qs], C::kTile);
+          in_range(w.qt(x), p.n_qtiles);
+          in_range(w.bh(x), static_cast<long long>(p.B) * p.Hq);
           for (int c = 0; c < C::NB; ++c)
             tma_load_3d(sQ + (x * C::QST + qs) * C::kTile + c * C::kBox, &tmq, &sh.q_full[x][qs], c * 128 / C::ES,
                         w.qt(x) * 128, w.bh(x));
@@ -208,6 +210,8 @@ __global__ void __launch_bounds__(576, 1)
           if (kc >= 2) ok = mbar_wait(&sh.k_empty[st], ((kc >> 1) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
+          in_range(j, p.n_qtiles);
+          in_range(w.bkv, static_cast<long long>(p.B) * p.Hkv);
           for (int c = 0; c < C::NB; ++c)
             tma_load_3d(sK + st * C::kTile + c * C::kBox, &tmk, &sh.k_full[st], c * 128 / C::ES, j * 128, w.bkv);
           if (kc >= 2) ok = mbar_wait(&sh.v_empty[st], ((kc >> 1) - 1) & 1);
@@ -520,7 +524,7 @@ __global__ void __launch_bounds__(576, 1)
       if (!ok) break;
       tc_fence_after();
       const float inv_l = p.oscale / l;      // oscale: V's descale (1 for bf16)
-      const bool live = qrow < p.N;
+      const bool live = qrow < p.N && in_range(bh, static_cast<long long>(p.B) * p.Hq);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D + grp * OH;
 #pragma unroll 1
       for (int q4 = 0; q4 < OH / 16; ++q4) {

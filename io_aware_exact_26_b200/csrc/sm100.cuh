@@ -32,6 +32,26 @@ __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Checking build (compiled with -DATTN_CHECKS): every tile coordinate, head index and
+// global row the kernels compute is tested against the tensor it addresses before the
+// access; a value out of range records error 2 in the status word and the access is
+// skipped (stores) or kept harmless (TMA tile loads, which zero-fill outside the
+// tensor).  No trap, no assert.  In the normal build the tests compile away.
+#ifdef ATTN_CHECKS
+constexpr bool kChecks = true;
+#else
+constexpr bool kChecks = false;
+#endif
+__device__ __forceinline__ bool in_range(long long idx, long long n) {
+  if constexpr (kChecks) {
+    if (idx < 0 || idx >= n) {
+      record_error(&g_attn_status, 2);
+      return false;
+    }
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

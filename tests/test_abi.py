@@ -28,7 +28,8 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
          "attn_status_string", "attn_selftest_timeout", "attn_fwd_window", "attn_bwd_window", "attn_decode",
-         "attn_decode_workspace_size", "attn_decode_splits", "attn_merge", "attn_fwd_fp8"])
+         "attn_decode_workspace_size", "attn_decode_splits", "attn_merge", "attn_fwd_fp8", "attn_checks_enabled",
+         "attn_selftest_bounds"])
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -37,7 +38,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    texts = {code: binding.attn_status_string(code) for code in range(-7, 1)}
+    texts = {code: binding.attn_status_string(code) for code in range(-8, 1)}
     assert all(t and t != "unknown status" for t in texts.values())
     assert len(set(texts.values())) == len(texts)
     assert binding.attn_status_string(-99) == "unknown status"
@@ -170,3 +171,11 @@ def test_fp8_forward_validates_before_any_launch(L):
     assert f8(N=0) == -1
     assert f8(q=ODD) == -3
     assert f8(q=ctypes.c_void_p(0)) == -1
+
+
+def test_checking_build_exports_the_same_boundary(L):
+    import __graft_entry__  # noqa: F401  (build() made both libraries)
+    C = binding.load(binding.checks_library_path)
+    for name in declared_functions():
+        assert hasattr(C, name), name
+    assert C.attn_checks_enabled() == 1 and L.attn_checks_enabled() == 0
