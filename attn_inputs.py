@@ -93,6 +93,18 @@ DECODE_WORKLOADS = {
 }
 
 
+# Local (sliding-window) attention problems: a causal window of 4096 keys at 32K
+# context (Mistral-style), a 1024-key causal window at 8K, and a symmetric band.
+WINDOW_WORKLOADS = {
+    "window_causal_w4096_b1_h32_n32768_d128": (Workload("window_causal_w4096_b1_h32_n32768_d128", 1, 32, 32, 32768,
+                                                        128, False, "fwd+bwd", seed=4000), (4095, 0)),
+    "window_causal_w1024_b4_hq32_hkv8_n8192_d128": (Workload("window_causal_w1024_b4_hq32_hkv8_n8192_d128", 4, 32, 8,
+                                                             8192, 128, False, "fwd+bwd", seed=4001), (1023, 0)),
+    "window_sym_w512_b2_h16_n16384_d64": (Workload("window_sym_w512_b2_h16_n16384_d64", 2, 16, 16, 16384, 64, False,
+                                                   "fwd+bwd", seed=4002), (256, 256)),
+}
+
+
 def make_decode_inputs(w: DecodeWorkload, device="cpu"):
     """q [B,Hq,Nq,d], k and v [B,Hkv,Nk,d]: bf16 N(0,1) draws from one seeded generator."""
     dev = torch.device(device)

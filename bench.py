@@ -35,8 +35,8 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from attn_inputs import (DECODE_WORKLOADS, WORKLOADS, Workload, make_decode_inputs, make_inputs,  # noqa: E402
-                         sweep_workloads)
+from attn_inputs import (DECODE_WORKLOADS, WINDOW_WORKLOADS, WORKLOADS, Workload, make_decode_inputs,  # noqa: E402
+                         make_inputs, sweep_workloads)
 from io_aware_exact_26_b200 import accounting as acc  # noqa: E402
 
 # The largest single-GPU workload (forward + backward, causal, d = 128, N = 32768).
@@ -468,6 +468,55 @@ def run_fp8(args):
         torch.cuda.empty_cache()
 
 
+def run_window(args):
+    """Local (sliding-window) attention: forward and backward timed apart, TFLOPS over the
+    visible (query, key) pairs only, one JSON line per window workload."""
+    import torch
+    import io_aware_exact_26_b200 as attn
+
+    peaks, peaks_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    for name, (w, window) in WINDOW_WORKLOADS.items():
+        x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, device=dev, with_grad=True)
+        q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(attn.attn_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.N, w.d, False), dtype=torch.uint8,
+                         device=dev)
+        fns = {"fwd": lambda: attn.attn_fwd_window(q, k, v, o, lse, window=window, scale=w.scale),
+               "bwd": lambda: attn.attn_bwd_window(q, k, v, o, lse, do, dq, dk, dv, window=window, scale=w.scale,
+                                                   workspace=ws)}
+        line = {"window": name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "left": window[0],
+                "right": window[1], "reps": args.sweep_reps, "warmup": args.warmup,
+                "peak": peak, "peak_source": f"{peaks_kind} bf16 dense (burst)"}
+        sampler = ClockSampler(0)
+        sampler.start()
+        for kind, fn in fns.items():
+            for _ in range(args.warmup):      # the forward runs first, so o and lse are set for the backward
+                fn()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.sweep_reps)]
+            for a, b in evs:
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+            fl = acc.flops_window(w.B, w.Hq, w.N, w.d, window[0], window[1], bwd=(kind == "bwd"))
+            tf = fl / (ms * 1e-3) / 1e12
+            line[kind] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_peak": round(tf / peak, 4)}
+        line["clocks"] = sampler.stop()
+        if attn.attn_get_device_status() != 0:
+            raise SystemExit(f"device-side error in the window run at {name}")
+        print(json.dumps(line), flush=True)
+        del x, q, k, v, do, o, lse, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,6 +531,7 @@ def main():
     ap.add_argument("--sweep-reps", type=int, default=50)
     ap.add_argument("--decode", action="store_true", help="time split-KV decoding, one line per decode workload")
     ap.add_argument("--fp8", action="store_true", help="time the fp8 forward next to the bf16 forward")
+    ap.add_argument("--window", action="store_true", help="time local (sliding-window) attention, fwd and bwd")
     ap.add_argument("--decode-workload", default=None, choices=sorted(DECODE_WORKLOADS))
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -493,6 +543,9 @@ def main():
         return
     if args.fp8:
         run_fp8(args)
+        return
+    if args.window:
+        run_window(args)
         return
 
     rank = int(os.environ.get("RANK", "0"))

@@ -98,3 +98,20 @@ def flops_decode(B, Hq, Nq, Nk, d, causal):
     else:
         pairs = Nq * Nk
     return 4.0 * B * Hq * pairs * d
+
+
+def visible_pairs(N, left, right):
+    """Number of (query, key) pairs with i - left <= j <= i + right (None = no limit),
+    0 <= i, j < N."""
+    wl = N if left is None else min(left, N)
+    wr = N if right is None else min(right, N)
+    total = 0
+    for i in range(N):
+        total += min(N - 1, i + wr) - max(0, i - wl) + 1
+    return total
+
+
+def flops_window(B, Hq, N, d, left, right, bwd=False):
+    """4*d FLOPs per visible pair forward, 10*d backward (the dense counts restricted to
+    the band; causal, (None, 0), gives exactly the halved-plus-diagonal count)."""
+    return (10.0 if bwd else 4.0) * B * Hq * visible_pairs(N, left, right) * d

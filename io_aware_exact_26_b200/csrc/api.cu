@@ -168,8 +168,8 @@ DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int sms) {
   long long T = (pl.nkt * pairs + target - 1) / target;     // key tiles per split
   if (T < 4) T = 4;
   if (T > pl.nkt) T = pl.nkt;
-  pl.T = static_cast<int>(T);
-  pl.S = (pl.nkt + pl.T - 1) / pl.T;
+  pl.S = static_cast<int>((pl.nkt + T - 1) / T);
+  pl.T = (pl.nkt + pl.S - 1) / pl.S;                        // equal splits (the last may be shorter)
   pl.units = pairs * pl.S;
   return pl;
 }

@@ -54,8 +54,11 @@ struct PpCfg {
   static constexpr int VST = 2;
   static constexpr int kThreads = 576;
   // Of every 8 score pairs, how many are exponentiated on the FMA pipe instead of
-  // MUFU (16 ex2 per SM per clock).
-  static constexpr int kFmaPairs = 0;
+  // MUFU (16 ex2 per SM per clock).  At d = 64 a tile's two products take 768
+  // tensor-core cycles against 1024 MUFU cycles for its exponentials, so MUFU alone
+  // bounds the step and moving 2 pairs in 8 to the FMA pipe measured +8% to +21%
+  // (N = 1024 to 4096); at d = 128 the two are even and the share measured no gain.
+  static constexpr int kFmaPairs = (D == 64 && !F8) ? 2 : 0;
   static constexpr int kTmemCols = 512;
   static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
   // Q buffers per team: two at d = 64, so the next unit's Q loads while the current
@@ -402,32 +405,60 @@ __global__ void __launch_bounds__(576, 1)
         const int lo = qrow - p.wl - kbase;                          // first visible column
         const int lim = min(p.N - 1, qrow + p.wr) - kbase;           // last visible column
         const bool msk = __any_sync(0xffffffffu, lo > 0 || lim < 63);
-        // pass 1: this group's partial row max of the 64 columns
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        {
-          uint32_t r0[16], r1[16], r2[16], r3[16];
-          tmem_ld16(s_base, r0);
-          tmem_ld16(s_base + 16, r1);
-          tmem_ld16(s_base + 32, r2);
-          tmem_ld16(s_base + 48, r3);
-          tmem_wait_ld();
-          reg_fence(r0);
-          reg_fence(r1);
-          reg_fence(r2);
-          reg_fence(r3);
-          if (msk) { mask16(r0, 0, lo, lim); mask16(r1, 16, lo, lim); mask16(r2, 32, lo, lim); mask16(r3, 48, lo, lim); }
+        // One pass with the row's current exponent base m_used: p = 2^(s c - m_used) for the
+        // group's 64 columns, packed in registers, the group's tile max on the side.  The
+        // maxima are exchanged afterwards; only where the row max grew by more than tau
+        // (always on a unit's first step) is the pass redone from S with the new base.
+        // S is still intact then: P is written over it only at the end of the step.
+        // Masked columns hold -inf, and c > 0 (the host floors it at 1e-30), so their
+        // exponent argument is -inf and p = 0.
+        constexpr int PW = F8 ? 4 : 8;                   // packed words of P per 16 columns
+        uint32_t pk[4 * PW];
+        float mx2[2] = {-INFINITY, -INFINITY};
+        uint64_t lt = f2pack(0.f, 0.f);                  // this tile's row sum
+        auto exp_pass = [&](bool track_max) {
+          const float mb = m_used == -INFINITY ? 0.f : m_used;
+          const uint64_t nm2 = f2pack(-mb, -mb);
+          lt = f2pack(0.f, 0.f);
 #pragma unroll
-          for (int k = 0; k < 16; k += 8) {
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t r[16];
+            tmem_ld16(s_base + cc * 16, r);
+            tmem_wait_ld();
+            reg_fence(r);
+            if (msk) mask16(r, cc * 16, lo, lim);
+            if (track_max) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              mx4[e] = max3f(mx4[e], __uint_as_float(r0[k + e]), __uint_as_float(r0[k + e + 4]));
-              mx4[e] = max3f(mx4[e], __uint_as_float(r1[k + e]), __uint_as_float(r1[k + e + 4]));
-              mx4[e] = max3f(mx4[e], __uint_as_float(r2[k + e]), __uint_as_float(r2[k + e + 4]));
-              mx4[e] = max3f(mx4[e], __uint_as_float(r3[k + e]), __uint_as_float(r3[k + e + 4]));
+              for (int e = 0; e < 16; e += 4) {
+                mx2[0] = max3f(mx2[0], __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+                mx2[1] = max3f(mx2[1], __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint64_t xx = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
+              float x0, x1;
+              f2unpack(xx, x0, x1);
+              float a, b;
+              if (k >= 8 - C::kFmaPairs) {
+                exp2_fma_pair(x0, x1, a, b);
+              } else {
+                a = ex2_approx(x0);
+                b = ex2_approx(x1);
+              }
+              lt = fadd2(lt, f2pack(a, b));
+              if constexpr (F8) {
+                // four e4m3 per column, lowest key in the low byte; p <= 2^tau = 256 < 448
+                const uint32_t two = pack_e4m3x2(a, b);
+                pk[cc * PW + (k >> 1)] = (k & 1) ? (pk[cc * PW + (k >> 1)] | (two << 16)) : two;
+              } else {
+                pk[cc * PW + k] = pack_bf16x2(a, b);
+              }
             }
           }
-        }
-        sh.xmax[x][xp][grp][row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        };
+        exp_pass(true);
+        sh.xmax[x][xp][grp][row] = fmaxf(mx2[0], mx2[1]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.xbar[x][xp]);
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.xbar[x][xp], (g >> 1) & 1));
@@ -445,6 +476,21 @@ __global__ void __launch_bounds__(576, 1)
           lsum = f2pack(l0 * alpha, l1 * alpha);
           m_used = m_new;
         }
+        // rows whose base moved: the same pass again with the new base (the other rows of
+        // the warp get the same values again)
+        if (__any_sync(0xffffffffu, need)) exp_pass(false);
+        lsum = fadd2(lsum, lt);
+        // P over the columns of S (all read by now)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          if constexpr (F8) {
+            const uint32_t (&p4)[4] = *reinterpret_cast<const uint32_t (*)[4]>(pk + cc * PW);
+            tmem_st4(s_base + cc * 4, p4);
+          } else {
+            const uint32_t (&p8)[8] = *reinterpret_cast<const uint32_t (*)[8]>(pk + cc * PW);
+            tmem_st8(s_base + cc * 8, p8);
+          }
+        }
         // Rescale this group's O columns if the max moved.  The commit that signalled
         // S_X(j) also covers PV_X(j-1), so O already holds every step before j; the
         // wait below is then immediate.
@@ -461,47 +507,6 @@ __global__ void __launch_bounds__(576, 1)
 #pragma unroll
             for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
             tmem_st16(o_base + q4 * 16, o);
-          }
-        }
-        // pass 2: exponentiate, P (bf16) over the columns already read.  Masked columns
-        // hold -inf, and c > 0 (the host floors it at 1e-30), so their exponent argument
-        // is -inf and p = 0; the base is 0 while the row has seen no visible key.
-        const float mb = m_used == -INFINITY ? 0.f : m_used;
-        const uint64_t nm2 = f2pack(-mb, -mb);
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t r[16];
-          tmem_ld16(s_base + cc * 16, r);
-          tmem_wait_ld();
-          reg_fence(r);
-          if (msk) mask16(r, cc * 16, lo, lim);
-          uint32_t pk[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint64_t xx = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
-            float x0, x1;
-            f2unpack(xx, x0, x1);
-            float a, b;
-            if (k >= 8 - C::kFmaPairs) {
-              exp2_fma_pair(x0, x1, a, b);
-            } else {
-              a = ex2_approx(x0);
-              b = ex2_approx(x1);
-            }
-            lsum = fadd2(lsum, f2pack(a, b));
-            if constexpr (F8) {
-              // four e4m3 per column, lowest key in the low byte; p <= 2^tau = 256 < 448
-              const uint32_t two = pack_e4m3x2(a, b);
-              pk[k >> 1] = (k & 1) ? (pk[k >> 1] | (two << 16)) : two;
-            } else {
-              pk[k] = pack_bf16x2(a, b);
-            }
-          }
-          if constexpr (F8) {
-            const uint32_t (&p4)[4] = *reinterpret_cast<const uint32_t (*)[4]>(pk);
-            tmem_st4(s_base + cc * 4, p4);
-          } else {
-            tmem_st8(s_base + cc * 8, pk);
           }
         }
         tmem_wait_st();

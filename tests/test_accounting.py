@@ -80,3 +80,20 @@ def test_attention_flops_and_min_bytes():
     assert acc.min_bytes_fwd(4, 32, 8, 8192, 128) == pytest.approx(675e6, rel=2e-3)
     assert acc.min_bytes_bwd(64, 16, 16, 1024, 64) == 8 * 64 * 16 * 1024 * 64 * 2 + 64 * 16 * 1024 * 4
     assert acc.tflops(1e12, 1000.0) == pytest.approx(1.0)
+
+
+def test_visible_pair_counts_of_bands():
+    N = 777
+    assert acc.visible_pairs(N, None, None) == N * N
+    assert acc.visible_pairs(N, None, 0) == N * (N + 1) // 2              # causal
+    assert acc.visible_pairs(N, 0, 0) == N                                 # each row sees itself
+    assert acc.visible_pairs(N, 10, 0) == sum(min(i, 10) + 1 for i in range(N))
+    assert acc.visible_pairs(N, 3, 5) == sum(min(N - 1, i + 5) - max(0, i - 3) + 1 for i in range(N))
+    assert acc.flops_window(1, 1, N, 64, None, 0) == 4 * 64 * N * (N + 1) / 2
+
+
+def test_decode_bytes_and_flops():
+    assert acc.min_bytes_decode(2, 8, 2, 1, 1000, 128) == 2 * 2 * 8 * 128 * 2 + 2 * 2 * 2 * 1000 * 128 * 2 + 2 * 8 * 4
+    assert acc.flops_decode(1, 1, 1, 10, 4, True) == 4 * 10 * 4          # the last query sees all keys
+    assert acc.flops_decode(1, 1, 3, 10, 4, True) == 4 * 4 * (8 + 9 + 10)
+    assert acc.flops_decode(1, 1, 3, 10, 4, False) == 4 * 4 * 30
