@@ -244,15 +244,39 @@ def step_flops(w: Workload):
     return f, fb
 
 
-def config_dict(w: Workload, n_gpus):
+def config_dict(w: Workload, n_gpus, shard=False):
+    par = (f"one job, contiguous (b, kv-head) slices over {n_gpus} ranks" if shard
+           else f"independent replicas x{n_gpus}")
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
-            "passes": w.passes, "scale": "1/sqrt(d)", "parallelism": f"independent replicas x{n_gpus}",
+            "passes": w.passes, "scale": "1/sqrt(d)", "parallelism": par,
             "l2": "inputs larger than L2 (126 MB); no flush"}
 
 
 def rank_seed(w: Workload, rank: int) -> int:
     """Each rank times its own replica of the workload on its own synthetic inputs."""
     return w.seed + 101 * rank
+
+
+def shard_units(total, rank, world):
+    """Contiguous, balanced slice [u0, u1) of ``total`` independent (b, kv-head) units for
+    one rank (the first ``total % world`` ranks take one more)."""
+    base, extra = divmod(total, world)
+    u0 = rank * base + min(rank, extra)
+    return u0, u0 + base + (1 if rank < extra else 0)
+
+
+def shard_views(x, w, rank, world):
+    """This rank's slice of one batch: [B][H][N][d] is [B*H][N][d] in memory, so the
+    units [u0, u1) of the flattened (b, kv-head) order are the kv-heads u0..u1-1 and the
+    q-heads G*u0..G*u1-1 of a batch of one.  Returns (views, units)."""
+    G = w.Hq // w.Hkv
+    u0, u1 = shard_units(w.B * w.Hkv, rank, world)
+    out = {}
+    for n, t in x.items():
+        flat = t.view(1, t.shape[0] * t.shape[1], t.shape[2], t.shape[3])
+        g = G if n in ("q", "do") else 1
+        out[n] = flat[:, u0 * g:u1 * g]
+    return out, u1 - u0
 
 
 def max_over_ranks(values, dist, device):
@@ -532,6 +556,9 @@ def main():
     ap.add_argument("--decode", action="store_true", help="time split-KV decoding, one line per decode workload")
     ap.add_argument("--fp8", action="store_true", help="time the fp8 forward next to the bf16 forward")
     ap.add_argument("--window", action="store_true", help="time local (sliding-window) attention, fwd and bwd")
+    ap.add_argument("--shard", action="store_true",
+                    help="N > 1: split one job's (b, kv-head) units across the ranks (strong scaling) "
+                         "instead of running N replicas")
     ap.add_argument("--decode-workload", default=None, choices=sorted(DECODE_WORKLOADS))
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -570,8 +597,19 @@ def main():
     w = WORKLOADS[args.workload]
     has_bwd = "bwd" in w.passes
     dev = torch.device("cuda", local)
-    x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=rank_seed(w, rank), qk_std=w.qk_std, vo_std=w.vo_std,
-                    boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=has_bwd)
+    if args.shard:
+        # one job split across the ranks: the same inputs everywhere, each rank takes a
+        # contiguous slice of the (b, kv-head) units
+        full = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, qk_std=w.qk_std, vo_std=w.vo_std,
+                           boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=has_bwd)
+        views, units = shard_views(full, w, rank, world)
+        x = {n: t.contiguous() for n, t in views.items()}
+        del full
+        w = Workload(w.name, 1, units * (w.Hq // w.Hkv), units, w.N, w.d, w.causal, w.passes, w.qk_std, w.vo_std,
+                     w.boost_frac, w.boost, w.seed)
+    else:
+        x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=rank_seed(w, rank), qk_std=w.qk_std, vo_std=w.vo_std,
+                        boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=has_bwd)
     q, k, v = x["q"], x["k"], x["v"]
     do = x.get("do")
     o = torch.empty_like(q)
@@ -625,7 +663,9 @@ def main():
         [total_ms, statistics.mean(fwd_ms), statistics.mean(bwd_ms) if bwd_ms else 0.0], dist, dev)
     ms_per_step = total_ms / args.steps
     f_fwd, f_bwd = step_flops(w)
-    value = weak_scaling_tflops(f_fwd + f_bwd, world, ms_per_step)
+    # whole-job FLOPs per step: every replica's, or (shard) the one job's
+    job_flops = sum(step_flops(WORKLOADS[args.workload])) if args.shard else (f_fwd + f_bwd) * world
+    value = job_flops / (ms_per_step * 1e-3) / 1e12
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     host = {n: x[n].cpu().pin_memory() for n in x}
@@ -653,7 +693,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0] / args.e2e_steps
-    e2e_value = weak_scaling_tflops(f_fwd + f_bwd, world, e2e_ms)
+    e2e_value = job_flops / (e2e_ms * 1e-3) / 1e12
 
     # ---- roofline of the dominant kernel (backward when present)
     peaks, peaks_kind = load_peaks()
@@ -673,8 +713,8 @@ def main():
     line = {"metric": "attention fwd+bwd TFLOPS" if has_bwd else "attention fwd TFLOPS",
             "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_dict(w, world),
+            "scaling": "strong" if args.shard else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(WORKLOADS[args.workload], world, shard=args.shard),
             "fwd": {"ms": round(fwd_avg, 4), "tflops": round(f_fwd / (fwd_avg * 1e-3) / 1e12, 1),
                     "frac_of_peak": round(f_fwd / (fwd_avg * 1e-3) / 1e12 / peak, 4)},
             "roofline": roofline,

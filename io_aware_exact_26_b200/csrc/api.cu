@@ -141,8 +141,12 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   p.wl = band.wl;
   p.wr = band.wr;
   p.desc = band.wr <= band.wl;
-  const int units = B * Hkv * ((p.G * p.n_qtiles + 1) / 2);
+  const int upg = (p.G * p.n_qtiles + 1) / 2;
+  const int units = B * Hkv * upg;
   const int grid = units < di.sms ? units : di.sms;
+  // interleave the last groups that hold about two units per CTA
+  int tail = (2 * grid + upg - 1) / upg;
+  p.tail_groups = tail < 1 ? 1 : (tail > B * Hkv ? B * Hkv : tail);
   p.sched_slot = next_sched_slot();
   attn::sched_reset_kernel<<<1, 32, 0, stream>>>(p.sched_slot);
   attn::attn_fwd_pp_kernel<D, F8><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);

@@ -38,6 +38,7 @@ struct FwdParams {
   float oscale;     // output multiplier: V's descale for e4m3 inputs, else 1
   int wl, wr;       // window: 0 <= wl, wr <= N
   int desc;         // list query tiles last-first (their key ranges grow with the tile)
+  int tail_groups;  // number of last KV groups whose units are interleaved (1 <= . <= B * Hkv)
   int sched_slot;   // g_sched slot this launch claims work units from
 };
 

@@ -109,11 +109,25 @@ struct PpUnit {
 // as under causal masking: longest first), the G heads inside; consecutive list
 // entries are paired.  The unit streams the union of the two tiles' key ranges;
 // each team works on its own range inside it.
+// Units are claimed group after group, so the CTAs running at one time share the
+// K/V of a few heads in L2.  The last `tail_groups` groups are interleaved instead
+// (their units longest first across all of them): otherwise a CTA that claims a
+// long unit of the last group near the end finishes long after the others
+// (measured 7-13% idle at the end with 16-32 heads).
 __device__ __forceinline__ PpUnit pp_unit(const FwdParams& p, int u) {
   const int per_group = p.G * p.n_qtiles;
   const int upg = (per_group + 1) >> 1;
-  const int gk = u / upg;
-  const int m = u - gk * upg;
+  const int ngroups = p.B * p.Hkv;
+  const int head = (ngroups - p.tail_groups) * upg;     // units before the interleaved tail
+  int gk, m;
+  if (u < head) {
+    gk = u / upg;
+    m = u - gk * upg;
+  } else {
+    const int v = u - head;
+    m = v / p.tail_groups;
+    gk = ngroups - p.tail_groups + (v - m * p.tail_groups);
+  }
   PpUnit r;
   r.bkv = gk;
   auto tile = [&](int l, int& bh, int& qt, int& a, int& n) {
@@ -381,10 +395,18 @@ __global__ void __launch_bounds__(576, 1)
     const uint64_t c2 = f2pack(c, c);
     int gs = 0, uu = 0;
     bool ok = true;
-    auto mask16 = [&](uint32_t (&r)[16], int col0, int lo, int lim) {
+    // -inf outside the visible columns [lo, lim]; lo_on = false when no lane of the warp
+    // has a lower bound inside the tile (causal), which halves the work per element
+    auto mask16 = [&](uint32_t (&r)[16], int col0, int lo, int lim, bool lo_on) {
+      if (lo_on) {
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        if (col0 + k < lo || col0 + k > lim) r[k] = 0xff800000u;
+        for (int k = 0; k < 16; ++k)
+          if (col0 + k < lo || col0 + k > lim) r[k] = 0xff800000u;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          if (col0 + k > lim) r[k] = 0xff800000u;
+      }
     };
     for (int k = 0; ok; ++k) {
       const int u = unit_ring_take(sh.ring, k, lane, ok);
@@ -404,61 +426,39 @@ __global__ void __launch_bounds__(576, 1)
         const int kbase = (a + j) * 128 + grp * 64;
         const int lo = qrow - p.wl - kbase;                          // first visible column
         const int lim = min(p.N - 1, qrow + p.wr) - kbase;           // last visible column
-        const bool msk = __any_sync(0xffffffffu, lo > 0 || lim < 63);
-        // One pass with the row's current exponent base m_used: p = 2^(s c - m_used) for the
-        // group's 64 columns, packed in registers, the group's tile max on the side.  The
-        // maxima are exchanged afterwards; only where the row max grew by more than tau
-        // (always on a unit's first step) is the pass redone from S with the new base.
-        // S is still intact then: P is written over it only at the end of the step.
-        // Masked columns hold -inf, and c > 0 (the host floors it at 1e-30), so their
-        // exponent argument is -inf and p = 0.
-        constexpr int PW = F8 ? 4 : 8;                   // packed words of P per 16 columns
-        uint32_t pk[4 * PW];
-        float mx2[2] = {-INFINITY, -INFINITY};
-        uint64_t lt = f2pack(0.f, 0.f);                  // this tile's row sum
-        auto exp_pass = [&](bool track_max) {
-          const float mb = m_used == -INFINITY ? 0.f : m_used;
-          const uint64_t nm2 = f2pack(-mb, -mb);
-          lt = f2pack(0.f, 0.f);
+        const bool lo_on = __any_sync(0xffffffffu, lo > 0);
+        const bool msk = lo_on || __any_sync(0xffffffffu, lim < 63);
+        // pass 1: this group's partial row max of the 64 columns
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        {
+          uint32_t r0[16], r1[16], r2[16], r3[16];
+          tmem_ld16(s_base, r0);
+          tmem_ld16(s_base + 16, r1);
+          tmem_ld16(s_base + 32, r2);
+          tmem_ld16(s_base + 48, r3);
+          tmem_wait_ld();
+          reg_fence(r0);
+          reg_fence(r1);
+          reg_fence(r2);
+          reg_fence(r3);
+          if (msk) {
+            mask16(r0, 0, lo, lim, lo_on);
+            mask16(r1, 16, lo, lim, lo_on);
+            mask16(r2, 32, lo, lim, lo_on);
+            mask16(r3, 48, lo, lim, lo_on);
+          }
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t r[16];
-            tmem_ld16(s_base + cc * 16, r);
-            tmem_wait_ld();
-            reg_fence(r);
-            if (msk) mask16(r, cc * 16, lo, lim);
-            if (track_max) {
+          for (int k = 0; k < 16; k += 8) {
 #pragma unroll
-              for (int e = 0; e < 16; e += 4) {
-                mx2[0] = max3f(mx2[0], __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-                mx2[1] = max3f(mx2[1], __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint64_t xx = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
-              float x0, x1;
-              f2unpack(xx, x0, x1);
-              float a, b;
-              if (k >= 8 - C::kFmaPairs) {
-                exp2_fma_pair(x0, x1, a, b);
-              } else {
-                a = ex2_approx(x0);
-                b = ex2_approx(x1);
-              }
-              lt = fadd2(lt, f2pack(a, b));
-              if constexpr (F8) {
-                // four e4m3 per column, lowest key in the low byte; p <= 2^tau = 256 < 448
-                const uint32_t two = pack_e4m3x2(a, b);
-                pk[cc * PW + (k >> 1)] = (k & 1) ? (pk[cc * PW + (k >> 1)] | (two << 16)) : two;
-              } else {
-                pk[cc * PW + k] = pack_bf16x2(a, b);
-              }
+            for (int e = 0; e < 4; ++e) {
+              mx4[e] = max3f(mx4[e], __uint_as_float(r0[k + e]), __uint_as_float(r0[k + e + 4]));
+              mx4[e] = max3f(mx4[e], __uint_as_float(r1[k + e]), __uint_as_float(r1[k + e + 4]));
+              mx4[e] = max3f(mx4[e], __uint_as_float(r2[k + e]), __uint_as_float(r2[k + e + 4]));
+              mx4[e] = max3f(mx4[e], __uint_as_float(r3[k + e]), __uint_as_float(r3[k + e + 4]));
             }
           }
-        };
-        exp_pass(true);
-        sh.xmax[x][xp][grp][row] = fmaxf(mx2[0], mx2[1]);
+        }
+        sh.xmax[x][xp][grp][row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.xbar[x][xp]);
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.xbar[x][xp], (g >> 1) & 1));
@@ -476,21 +476,6 @@ __global__ void __launch_bounds__(576, 1)
           lsum = f2pack(l0 * alpha, l1 * alpha);
           m_used = m_new;
         }
-        // rows whose base moved: the same pass again with the new base (the other rows of
-        // the warp get the same values again)
-        if (__any_sync(0xffffffffu, need)) exp_pass(false);
-        lsum = fadd2(lsum, lt);
-        // P over the columns of S (all read by now)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          if constexpr (F8) {
-            const uint32_t (&p4)[4] = *reinterpret_cast<const uint32_t (*)[4]>(pk + cc * PW);
-            tmem_st4(s_base + cc * 4, p4);
-          } else {
-            const uint32_t (&p8)[8] = *reinterpret_cast<const uint32_t (*)[8]>(pk + cc * PW);
-            tmem_st8(s_base + cc * 8, p8);
-          }
-        }
         // Rescale this group's O columns if the max moved.  The commit that signalled
         // S_X(j) also covers PV_X(j-1), so O already holds every step before j; the
         // wait below is then immediate.
@@ -507,6 +492,47 @@ __global__ void __launch_bounds__(576, 1)
 #pragma unroll
             for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
             tmem_st16(o_base + q4 * 16, o);
+          }
+        }
+        // pass 2: exponentiate, P (bf16) over the columns already read.  Masked columns
+        // hold -inf, and c > 0 (the host floors it at 1e-30), so their exponent argument
+        // is -inf and p = 0; the base is 0 while the row has seen no visible key.
+        const float mb = m_used == -INFINITY ? 0.f : m_used;
+        const uint64_t nm2 = f2pack(-mb, -mb);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t r[16];
+          tmem_ld16(s_base + cc * 16, r);
+          tmem_wait_ld();
+          reg_fence(r);
+          if (msk) mask16(r, cc * 16, lo, lim, lo_on);
+          uint32_t pk[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t xx = ffma2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
+            float x0, x1;
+            f2unpack(xx, x0, x1);
+            float a, b;
+            if (k >= 8 - C::kFmaPairs) {
+              exp2_fma_pair(x0, x1, a, b);
+            } else {
+              a = ex2_approx(x0);
+              b = ex2_approx(x1);
+            }
+            lsum = fadd2(lsum, f2pack(a, b));
+            if constexpr (F8) {
+              // four e4m3 per column, lowest key in the low byte; p <= 2^tau = 256 < 448
+              const uint32_t two = pack_e4m3x2(a, b);
+              pk[k >> 1] = (k & 1) ? (pk[k >> 1] | (two << 16)) : two;
+            } else {
+              pk[k] = pack_bf16x2(a, b);
+            }
+          }
+          if constexpr (F8) {
+            const uint32_t (&p4)[4] = *reinterpret_cast<const uint32_t (*)[4]>(pk);
+            tmem_st4(s_base + cc * 4, p4);
+          } else {
+            tmem_st8(s_base + cc * 8, pk);
           }
         }
         tmem_wait_st();

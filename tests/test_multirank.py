@@ -1,4 +1,5 @@
-"""The multi-GPU path of bench.py (independent replicas, weak scaling) on CPU ranks.
+"""The multi-GPU path of bench.py (independent replicas, weak scaling; or one job
+sharded into contiguous (b, kv-head) slices, strong scaling) on CPU ranks.
 
 Two gloo ranks on 127.0.0.1 run bench.py's per-rank pieces: each rank seeds its own
 replica, the timings are reduced to the max over ranks (the slowest rank sets the
@@ -82,3 +83,51 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     f, fb = bench.step_flops(bench.WORKLOADS[Args.workload])
     assert abs(line["ms_per_step"] - (f + fb) / (line["value"] * 1e12) * 1e3) <= 1e-9 * line["ms_per_step"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_shard_units_partition_the_job_contiguously():
+    sys.path.insert(0, ROOT)
+    import bench
+    for total in (1, 7, 32, 128, 1000):
+        for world in (1, 2, 3, 4, 8):
+            spans = [bench.shard_units(total, r, world) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == total
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            sizes = [b - a for a, b in spans]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def _shard_rank(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    import bench
+    import numpy as np
+    import torch.distributed as dist
+    from attn_inputs import Workload, make_inputs, to_f64
+    from oracle import reference as ref
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = Workload("tiny", 3, 4, 2, 9, 4, True, "fwd", seed=77)
+        full = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, with_grad=False)
+        views, units = bench.shard_views(full, w, rank, world)
+        o, lse = ref.ref_fwd(*(to_f64(views[n]) for n in ("q", "k", "v")), 0.5, w.causal)
+        np.save(os.path.join(out_dir, f"o{rank}.npy"), o)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_shard_views_map_each_rank_to_its_heads(tmp_path, world):
+    """Each rank's contiguous slice of the (b, kv-head) units, attended on its own, gives
+    exactly its heads' rows of the whole job (GQA groups stay together)."""
+    import numpy as np
+    import torch.multiprocessing as mp
+    from attn_inputs import make_inputs, to_f64
+    from oracle import reference as ref
+    mp.start_processes(_shard_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    full = make_inputs(3, 4, 2, 9, 4, seed=77, with_grad=False)
+    o_ref, _ = ref.ref_fwd(*(to_f64(full[n]) for n in ("q", "k", "v")), 0.5, True)
+    flat = o_ref.reshape(1, 12, 9, 4)
+    got = np.concatenate([np.load(tmp_path / f"o{r}.npy") for r in range(world)], axis=1)
+    np.testing.assert_array_equal(got, flat)
