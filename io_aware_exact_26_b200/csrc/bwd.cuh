@@ -129,22 +129,12 @@ struct BwdParams {
 // Masked columns (only on band-edge / ragged tiles) get s = -inf first; c > 0 (the
 // host floors it at 1e-30), so p = 0 (or 2^-126.5 on the FMA-pipe path); the exp
 // loop itself has no branch.
-// lo_on / hi_on (warp-uniform): whether any lane has that bound inside the tile, so
-// the causal diagonal tiles test one side per element only.
-__device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const float (&lv)[16], float c, bool lo_on,
-                                          bool hi_on, int col0, int lo, int hi, float* pf) {
-  if (lo_on && hi_on) {
+__device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const float (&lv)[16], float c, bool masked,
+                                          int col0, int lo, int hi, float* pf) {
+  if (masked) {
 #pragma unroll
     for (int k = 0; k < 16; ++k)
       if (col0 + k < lo || col0 + k > hi) sr[k] = 0xff800000u;
-  } else if (lo_on) {
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-      if (col0 + k < lo) sr[k] = 0xff800000u;
-  } else if (hi_on) {
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-      if (col0 + k > hi) sr[k] = 0xff800000u;
   }
 #pragma unroll
   for (int k = 0; k < 16; k += 2) {
@@ -454,7 +444,7 @@ __global__ void __launch_bounds__(320, 1)
           const int qbase = i * 128 + 64 * hb;
           const int hi = key_live ? (min(p.N - 1, key + p.wl) - qbase) : -1;
           const int lo = key - p.wr - qbase;
-          const bool lo_on = __any_sync(0xffffffffu, lo > 0), hi_on = __any_sync(0xffffffffu, hi < 63);
+          const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= 63);
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.qdo_full[st], (gs >> 1) & 1));
           if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full, gs & 1));
           if (!ok) break;
@@ -473,7 +463,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             tmem_wait_ld();
             reg_fence(sr);
-            bwd_exp16(sr, lv, c, lo_on, hi_on, q16 * 16, lo, hi, pf + q16 * 16);
+            bwd_exp16(sr, lv, c, masked, q16 * 16, lo, hi, pf + q16 * 16);
             uint32_t pk[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k], pf[q16 * 16 + 2 * k + 1]);
@@ -844,7 +834,7 @@ __global__ void __launch_bounds__(352, 1)
         const int kbase = (j0 + u) * 128 + 64 * hb;
         const int hi = min(p.N - 1, qrow + p.wr) - kbase;
         const int lo = qrow - p.wl - kbase;
-        const bool lo_on = __any_sync(0xffffffffu, lo > 0), hi_on = __any_sync(0xffffffffu, hi < 63);
+        const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= 63);
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[sb], (g >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
@@ -856,7 +846,7 @@ __global__ void __launch_bounds__(352, 1)
           tmem_ld16(sbase + q16 * 16, sr);
           tmem_wait_ld();
           reg_fence(sr);
-          bwd_exp16(sr, lv, c, lo_on, hi_on, q16 * 16, lo, hi, pf + q16 * 16);
+          bwd_exp16(sr, lv, c, masked, q16 * 16, lo, hi, pf + q16 * 16);
         }
         // phase B: dS = P (dP - D) -> bf16 over the S buffer
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.dp_full, g & 1));

@@ -395,18 +395,13 @@ __global__ void __launch_bounds__(576, 1)
     const uint64_t c2 = f2pack(c, c);
     int gs = 0, uu = 0;
     bool ok = true;
-    // -inf outside the visible columns [lo, lim]; lo_on = false when no lane of the warp
-    // has a lower bound inside the tile (causal), which halves the work per element
-    auto mask16 = [&](uint32_t (&r)[16], int col0, int lo, int lim, bool lo_on) {
-      if (lo_on) {
+    // -inf outside the visible columns [lo, lim].  (A causal-only variant testing one
+    // bound per element measured slower: the second code path in the hot loop cost
+    // more than the compares it saved.)
+    auto mask16 = [&](uint32_t (&r)[16], int col0, int lo, int lim) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-          if (col0 + k < lo || col0 + k > lim) r[k] = 0xff800000u;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          if (col0 + k > lim) r[k] = 0xff800000u;
-      }
+      for (int k = 0; k < 16; ++k)
+        if (col0 + k < lo || col0 + k > lim) r[k] = 0xff800000u;
     };
     for (int k = 0; ok; ++k) {
       const int u = unit_ring_take(sh.ring, k, lane, ok);
@@ -426,8 +421,7 @@ __global__ void __launch_bounds__(576, 1)
         const int kbase = (a + j) * 128 + grp * 64;
         const int lo = qrow - p.wl - kbase;                          // first visible column
         const int lim = min(p.N - 1, qrow + p.wr) - kbase;           // last visible column
-        const bool lo_on = __any_sync(0xffffffffu, lo > 0);
-        const bool msk = lo_on || __any_sync(0xffffffffu, lim < 63);
+        const bool msk = __any_sync(0xffffffffu, lo > 0 || lim < 63);
         // pass 1: this group's partial row max of the 64 columns
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         {
@@ -441,12 +435,7 @@ __global__ void __launch_bounds__(576, 1)
           reg_fence(r1);
           reg_fence(r2);
           reg_fence(r3);
-          if (msk) {
-            mask16(r0, 0, lo, lim, lo_on);
-            mask16(r1, 16, lo, lim, lo_on);
-            mask16(r2, 32, lo, lim, lo_on);
-            mask16(r3, 48, lo, lim, lo_on);
-          }
+          if (msk) { mask16(r0, 0, lo, lim); mask16(r1, 16, lo, lim); mask16(r2, 32, lo, lim); mask16(r3, 48, lo, lim); }
 #pragma unroll
           for (int k = 0; k < 16; k += 8) {
 #pragma unroll
@@ -505,7 +494,7 @@ __global__ void __launch_bounds__(576, 1)
           tmem_ld16(s_base + cc * 16, r);
           tmem_wait_ld();
           reg_fence(r);
-          if (msk) mask16(r, cc * 16, lo, lim, lo_on);
+          if (msk) mask16(r, cc * 16, lo, lim);
           uint32_t pk[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
