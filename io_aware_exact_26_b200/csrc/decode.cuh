@@ -404,7 +404,15 @@ __global__ void __launch_bounds__(320, 1)
                 ffma2(f2pack(__uint_as_float(r[2 * kk]), __uint_as_float(r[2 * kk + 1])), c2, nm2);
             float x0, x1;
             f2unpack(xx, x0, x1);
-            const float a0 = ex2_approx(x0), a1 = ex2_approx(x1);
+            // at d = 64 a 32 KB K/V tile takes about as long to stream as its 16384
+            // exponentials take on MUFU: 2 pairs in 8 go to the FMA pipe, as in the forward
+            float a0, a1;
+            if (D == 64 && kk >= 6) {
+              exp2_fma_pair(x0, x1, a0, a1);
+            } else {
+              a0 = ex2_approx(x0);
+              a1 = ex2_approx(x1);
+            }
             lsum = fadd2(lsum, f2pack(a0, a1));
             pk[kk] = pack_bf16x2(a0, a1);
           }
