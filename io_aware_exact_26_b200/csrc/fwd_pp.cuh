@@ -435,7 +435,19 @@ __global__ void __launch_bounds__(576, 1)
           reg_fence(r1);
           reg_fence(r2);
           reg_fence(r3);
-          if (msk) { mask16(r0, 0, lo, lim); mask16(r1, 16, lo, lim); mask16(r2, 32, lo, lim); mask16(r3, 48, lo, lim); }
+          if (msk) {
+            // Masked columns become -inf here and go back to TMEM, so the exponent pass
+            // below reads them already masked and needs no test of its own.
+            mask16(r0, 0, lo, lim);
+            mask16(r1, 16, lo, lim);
+            mask16(r2, 32, lo, lim);
+            mask16(r3, 48, lo, lim);
+            tmem_st16(s_base, r0);
+            tmem_st16(s_base + 16, r1);
+            tmem_st16(s_base + 32, r2);
+            tmem_st16(s_base + 48, r3);
+            tmem_wait_st();
+          }
 #pragma unroll
           for (int k = 0; k < 16; k += 8) {
 #pragma unroll
@@ -484,8 +496,9 @@ __global__ void __launch_bounds__(576, 1)
           }
         }
         // pass 2: exponentiate, P (bf16) over the columns already read.  Masked columns
-        // hold -inf, and c > 0 (the host floors it at 1e-30), so their exponent argument
-        // is -inf and p = 0; the base is 0 while the row has seen no visible key.
+        // hold -inf (written back by pass 1), and c > 0 (the host floors it at 1e-30), so
+        // their exponent argument is -inf and p = 0; the base is 0 while the row has seen
+        // no visible key.
         const float mb = m_used == -INFINITY ? 0.f : m_used;
         const uint64_t nm2 = f2pack(-mb, -mb);
 #pragma unroll
@@ -494,7 +507,6 @@ __global__ void __launch_bounds__(576, 1)
           tmem_ld16(s_base + cc * 16, r);
           tmem_wait_ld();
           reg_fence(r);
-          if (msk) mask16(r, cc * 16, lo, lim);
           uint32_t pk[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
