@@ -90,3 +90,15 @@ def test_window_of_one_key_returns_v(attn):
     assert torch.equal(o, v)
     want = d ** -0.5 * np.einsum("bhnd,bhnd->bhn", f64(q), f64(k))
     assert np.abs(f64(lse) - want).max() < 1e-3
+
+
+def test_window_backward_is_bitwise_deterministic(attn):
+    B, Hq, Hkv, N, d = 1, 4, 2, 1500, 128
+    x = make_inputs(B, Hq, Hkv, N, d, seed=17)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = attn.attn_fwd_window(q, k, v, window=(300, 40))
+    g1 = attn.attn_bwd_window(q, k, v, o, lse, do, window=(300, 40))
+    g2 = attn.attn_bwd_window(q, k, v, o, lse, do, window=(300, 40))
+    torch.cuda.synchronize()
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
