@@ -62,17 +62,17 @@ def code_text(src: str) -> str:
     return " ".join(src.split())
 
 
-# The sources the forward and backward kernels (the ones the bench line times) are
-# compiled from.  Other kernels of the library (decoding, merge) live in other files
-# and do not change these.
-KERNEL_SOURCES = ("sm100.cuh", "fwd.cuh", "fwd_pp.cuh", "bwd.cuh")
+# The sources each pass's kernels (the ones the bench line times) are compiled from.
+# Other kernels of the library (decoding, merges) live in other files and change
+# neither.
+KERNEL_SOURCES = {"fwd": ("sm100.cuh", "fwd.cuh", "fwd_pp.cuh"), "bwd": ("sm100.cuh", "bwd.cuh")}
 
 
-def kernel_source_hash():
-    """Fingerprint of the forward/backward kernel sources; comment or layout edits leave it unchanged."""
+def kernel_source_hash(pas="fwd", csrc=None):
+    """Fingerprint of one pass's kernel sources; comment or layout edits leave it unchanged."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "io_aware_exact_26_b200", "csrc")
-    for name in KERNEL_SOURCES:
+    csrc = csrc or os.path.join(ROOT, "io_aware_exact_26_b200", "csrc")
+    for name in KERNEL_SOURCES[pas]:
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode() + code_text(f.read()).encode())
     return h.hexdigest()[:16]
@@ -86,7 +86,7 @@ def measured_traffic(workload, kernel):
     except (OSError, ValueError):
         return None
     e = t.get(workload, {}).get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 

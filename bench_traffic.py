@@ -156,8 +156,9 @@ def write_launches(workload: str, csv_text: str, profiles_dir: str, revision: st
     agg = parse_launches(csv_text)
     w = bench.WORKLOADS[workload]
     passes = "one attn_fwd and one attn_bwd (prep + dK/dV + dQ kernels)" if "bwd" in w.passes else "one attn_fwd"
-    note = (f"Kernel sources: git revision {revision or git_revision()} (kernel source hash "
-            f"{bench.kernel_source_hash()}). The bench step is {passes}; the run makes 6 of each (3 warm-up, "
+    note = (f"Kernel sources: git revision {revision or git_revision()} (source fingerprints: forward "
+            f"{bench.kernel_source_hash('fwd')}, backward {bench.kernel_source_hash('bwd')}). The bench step is "
+            f"{passes}; the run makes 6 of each (3 warm-up, "
             "2 timed, 1 end-to-end); the at:: kernels are torch's input generation and host-copy casts, "
             "outside the timed region.")
     os.makedirs(profiles_dir, exist_ok=True)
@@ -167,10 +168,12 @@ def write_launches(workload: str, csv_text: str, profiles_dir: str, revision: st
     return path
 
 
-def dram_entry(workload: str, div: int, csv_texts, revision: str | None = None):
-    """Per kernel: DRAM bytes of one full-size launch (captured bytes x div) and the
-    source hash; per pass: the sum over its kernels."""
-    shash = bench.kernel_source_hash()
+def dram_entry(workload: str, div: int, csv_texts, revision: str | None = None, csrc: str | None = None):
+    """Per kernel: DRAM bytes of one full-size launch (captured bytes x div); per pass: the
+    sum over its kernels, stamped with the fingerprint of that pass's sources (of the
+    tree in ``csrc``, default the working tree: pass the captured revision's sources
+    when the tree has moved on)."""
+    shash = {pas: bench.kernel_source_hash(pas, csrc) for pas in ("fwd", "bwd")}
     kernels = {}
     for text in csv_texts:
         for name, a in parse_launches(text).items():
@@ -184,11 +187,12 @@ def dram_entry(workload: str, div: int, csv_texts, revision: str | None = None):
                             "read_bytes_per_launch": round(a["rd"] / a["n"] * div),
                             "write_bytes_per_launch": round(a["wr"] / a["n"] * div),
                             "bytes_per_launch": round((a["rd"] + a["wr"]) / a["n"] * div)}
-    entry = {"div": div, "source_hash": shash, "revision": revision or git_revision(), "kernels": kernels}
+    entry = {"div": div, "revision": revision or git_revision(), "kernels": kernels}
     for pas in ("fwd", "bwd"):
         ks = [k for k, (_, p) in KERNELS.items() if p == pas]
         if all(k in kernels for k in ks):
-            entry[pas] = {"bytes_per_launch": sum(kernels[k]["bytes_per_launch"] for k in ks), "source_hash": shash}
+            entry[pas] = {"bytes_per_launch": sum(kernels[k]["bytes_per_launch"] for k in ks),
+                          "source_hash": shash[pas]}
     return entry
 
 
@@ -201,7 +205,8 @@ def dram_table(workload: str, entry) -> str:
            f"Captured per kernel on the reduced case B={rw.B}, Hq={rw.Hq}, Hkv={rw.Hkv}, N={rw.N}, d={rw.d} "
            f"(the workload's (b, kv-head) units divided by {entry['div']}), one launch each, and scaled by "
            f"{entry['div']} to a full-size launch.  Kernel sources: git revision {entry['revision']} "
-           f"(kernel source hash {entry['source_hash']}).", "", "Commands, one per kernel:", ""]
+           f"(source fingerprints: forward {entry.get('fwd', {}).get('source_hash')}, backward "
+           f"{entry.get('bwd', {}).get('source_hash')}).", "", "Commands, one per kernel:", ""]
     for k in entry["kernels"]:
         out += ["```", dram_command(workload, entry["div"], k), "```"]
     out += ["", "| kernel | captured MB | read MB / full launch | write MB / full launch | total MB / full launch |",
@@ -230,8 +235,9 @@ def dram_table(workload: str, entry) -> str:
     return "\n".join(out) + "\n"
 
 
-def write_dram(workload: str, div: int, csv_texts, profiles_dir: str, revision: str | None = None):
-    entry = dram_entry(workload, div, csv_texts, revision)
+def write_dram(workload: str, div: int, csv_texts, profiles_dir: str, revision: str | None = None,
+               csrc: str | None = None):
+    entry = dram_entry(workload, div, csv_texts, revision, csrc)
     path = os.path.join(profiles_dir, "dram_traffic.json")
     try:
         with open(path) as f:
@@ -280,6 +286,7 @@ def main():
     b.add_argument("--workload", required=True, choices=sorted(bench.WORKLOADS))
     b.add_argument("--div", type=int, required=True)
     b.add_argument("--revision", default=None)
+    b.add_argument("--csrc", default=None, help="kernel sources of the captured revision (default: this tree)")
     b.add_argument("--profiles", default=os.path.join(ROOT, "profiles"))
     b.add_argument("csv", nargs="+")
     c = sub.add_parser("run", help="run one reduced case of the workload (the program ncu captures)")
@@ -295,7 +302,8 @@ def main():
         for p in args.csv:
             with open(p) as f:
                 texts.append(f.read())
-        print(json.dumps({args.workload: write_dram(args.workload, args.div, texts, args.profiles, args.revision)}))
+        print(json.dumps({args.workload: write_dram(args.workload, args.div, texts, args.profiles, args.revision,
+                                                    args.csrc)}))
     else:
         run_case(args.workload, args.div, args.reps)
 

@@ -92,7 +92,8 @@ def test_dram_entries_scale_to_full_launches_and_are_stamped(tmp_path, monkeypat
     assert k["fwd"]["bytes_per_launch"] == round((400e6 + 600e6 + 200e6) / 2 * 4)
     assert k["bwd_kv"]["bytes_per_launch"] == round(770e6 * 4)
     assert entry["bwd"]["bytes_per_launch"] == sum(k[x]["bytes_per_launch"] for x in ("bwd_prep", "bwd_kv", "bwd_q"))
-    assert entry["fwd"]["source_hash"] == bench.kernel_source_hash()
+    assert entry["fwd"]["source_hash"] == bench.kernel_source_hash("fwd")
+    assert entry["bwd"]["source_hash"] == bench.kernel_source_hash("bwd")
     md = (tmp_path / "dram_long_causal_b1_h32_n32768_d128.md").read_text()
     assert "abc1234" in md and "-k regex:attn_bwd_kv" in md
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "dram_traffic.json"))
@@ -106,6 +107,17 @@ def test_dram_entries_scale_to_full_launches_and_are_stamped(tmp_path, monkeypat
 def test_time_only_captures_are_refused_as_dram_evidence():
     with pytest.raises(ValueError):
         bench_traffic.dram_entry("long_causal_b1_h32_n32768_d128", 4, [time_only_csv()])
+
+
+def test_pass_fingerprints_cover_only_their_own_sources(tmp_path):
+    import shutil
+    src = os.path.join(ROOT, "io_aware_exact_26_b200", "csrc")
+    for name in os.listdir(src):
+        shutil.copy(os.path.join(src, name), tmp_path / name)
+    f0, b0 = bench.kernel_source_hash("fwd", str(tmp_path)), bench.kernel_source_hash("bwd", str(tmp_path))
+    (tmp_path / "fwd_pp.cuh").write_text((tmp_path / "fwd_pp.cuh").read_text() + "\nint changed;\n")
+    assert bench.kernel_source_hash("fwd", str(tmp_path)) != f0          # the forward's stamp moves
+    assert bench.kernel_source_hash("bwd", str(tmp_path)) == b0          # the backward's does not
 
 
 def test_source_fingerprint_ignores_comments_and_layout_but_not_code():
