@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(576, 1)
       // ahead leaves units reserved by busy CTAs at the tail (measured slower).
       int u = 0;
       for (int k = 0; ok; ++k) {
-        u = unit_ring_claim(sh.ring, k, p.sched_slot, n_units);
+        u = unit_ring_claim(sh.ring, k, p.sched_slot, p.sched_gen, n_units);
         if (u < 0) break;
         const PpUnit w = pp_unit(p, u);
         auto load_q = [&](int x, int uq) -> bool {     // Q of team x, its uq-th unit
@@ -558,16 +558,19 @@ __global__ void __launch_bounds__(576, 1)
       const float inv_l = p.oscale / l;      // oscale: V's descale (1 for bf16)
       const bool live = qrow < p.N && in_range(bh, static_cast<long long>(p.B) * p.Hq);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D + grp * OH;
-#pragma unroll 1
+      // all of this group's O columns in one round of TMEM loads (no softmax registers are
+      // live here), then convert and store
+      uint32_t o[OH / 16][16];
+#pragma unroll
+      for (int q4 = 0; q4 < OH / 16; ++q4) tmem_ld16(o_base + q4 * 16, o[q4]);
+      tmem_wait_ld();
+#pragma unroll
       for (int q4 = 0; q4 < OH / 16; ++q4) {
-        uint32_t o[16];
-        tmem_ld16(o_base + q4 * 16, o);
-        tmem_wait_ld();
-        reg_fence(o);
+        reg_fence(o[q4]);
         uint32_t pk[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          pk[k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
+          pk[k] = pack_bf16x2(__uint_as_float(o[q4][2 * k]) * inv_l, __uint_as_float(o[q4][2 * k + 1]) * inv_l);
         if (live) {
           uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 16);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
