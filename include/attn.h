@@ -53,15 +53,20 @@ typedef enum {
   ATTN_ERR_DEVICE_TIMEOUT = -5,/* a bounded device wait expired (see attn_get_device_status) */
   ATTN_ERR_WORKSPACE = -6,     /* backward workspace too small (or beyond the no-alloc scratch) */
   ATTN_ERR_ALLOC = -7,         /* the library's own stream-ordered allocation failed */
-  ATTN_ERR_DEVICE_BOUNDS = -8  /* checking build only: a kernel computed an index outside its tensor */
+  ATTN_ERR_DEVICE_BOUNDS = -8, /* checking build only: a kernel computed an index outside its tensor */
+  ATTN_ERR_SCHED_CONFLICT = -9 /* more than 128 forward/decode launches in flight: one stopped early */
 } attn_status_t;
 
 /* Forward: O and LSE for every (b, h, i).
  * Reads q, k, v; writes o and lse.  Returns ATTN_OK or a negative status.
  * Enqueues two kernels on `stream`: a one-thread kernel that zeroes this call's
  * work counter, then the forward, whose persistent CTAs claim work units from
- * that counter.  Each call takes the next of 128 counters (rotating), so up to
- * 128 forward calls may be in flight at once, on any streams. */
+ * that counter.  Each call takes the next of 128 counters (rotating, shared with
+ * attn_fwd_window, attn_fwd_fp8 and attn_decode), so up to 128 such calls may be in
+ * flight at once, on any streams.  Beyond that, a call whose counter is taken over
+ * by a later one stops claiming work, leaves its outputs incomplete and reports
+ * ATTN_ERR_SCHED_CONFLICT through attn_get_device_status(); the later call is
+ * unaffected. */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
              void* stream);
@@ -188,8 +193,8 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
 
 /* Synchronises `stream`, then returns ATTN_OK if no kernel of this library
  * recorded a device-side error since the last call, else ATTN_ERR_DEVICE_TIMEOUT
- * (a bounded wait expired) or ATTN_ERR_DEVICE_BOUNDS (checking build: an index
- * check failed); the error word is cleared.  While the word is set, later launches
+ * (a bounded wait expired), ATTN_ERR_DEVICE_BOUNDS (checking build: an index
+ * check failed) or ATTN_ERR_SCHED_CONFLICT (see attn_fwd); the error word is cleared.  While the word is set, later launches
  * exit early. */
 int attn_get_device_status(void* stream);
 
@@ -219,6 +224,19 @@ int attn_selftest_bounds(void* stream);
  * ATTN_ERR_DEVICE_TIMEOUT and clears the word.  Returns ATTN_ERR_INVALID_ARG for
  * a limit out of range, ATTN_ERR_LAUNCH if the launch is refused, else ATTN_OK. */
 int attn_selftest_timeout(long long limit_ns, void* stream);
+
+/* Diagnostic (no counterpart on the pages): exercises the work-counter takeover
+ * check that attn_fwd, attn_fwd_window, attn_fwd_fp8 and attn_decode rely on, on a
+ * counter reserved for it (no call of the library shares it).  Enqueues on `stream`:
+ * a reset of that counter to launch generation 7; one CTA of generation 7 claiming
+ * four times from 3 work units; a reset to generation 8; one CTA of generation 7
+ * claiming once; one CTA of generation 8 claiming once.  `out` is a device array of
+ * at least 6 ints; the claims land there in that order and read 0 1 2 -1 -1 0 (-1 =
+ * no unit), and the following attn_get_device_status() returns
+ * ATTN_ERR_SCHED_CONFLICT (generation 7 found the counter taken over).  Returns
+ * ATTN_ERR_INVALID_ARG for NULL, ATTN_ERR_ALIGNMENT for a misaligned `out`,
+ * ATTN_ERR_LAUNCH if a launch is refused, else ATTN_OK. */
+int attn_selftest_sched(int* out, void* stream);
 
 #ifdef __cplusplus
 }

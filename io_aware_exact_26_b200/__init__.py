@@ -22,6 +22,7 @@ from .binding import (  # noqa: F401
     attn_get_device_status,
     attn_checks_enabled,
     attn_selftest_bounds,
+    attn_selftest_sched,
     attn_selftest_timeout,
     checks_library_path,
     use_library,

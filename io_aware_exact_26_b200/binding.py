@@ -96,6 +96,8 @@ def load(path):
     L.attn_checks_enabled.restype = i
     L.attn_selftest_bounds.argtypes = [vp]
     L.attn_selftest_bounds.restype = i
+    L.attn_selftest_sched.argtypes = [vp, vp]
+    L.attn_selftest_sched.restype = i
     return L
 
 
@@ -347,6 +349,15 @@ def attn_selftest_bounds(stream=None) -> None:
     st = int(lib().attn_selftest_bounds(_stream_ptr(stream)))
     if st != 0:
         raise AttnError(st, "attn_selftest_bounds")
+
+
+def attn_selftest_sched(stream=None) -> list:
+    """Run the work-counter takeover self-test; returns its six claims (0 1 2 -1 -1 0 expected)."""
+    out = torch.full((8,), -7, dtype=torch.int32, device="cuda")
+    st = int(lib().attn_selftest_sched(_ptr(out), _stream_ptr(stream)))
+    if st != 0:
+        raise AttnError(st, "attn_selftest_sched")
+    return out[:6].tolist()
 
 
 def attn_checks_enabled() -> bool:

@@ -99,11 +99,17 @@ Band band_of_window(int N, int left, int right) {
   return {(left < 0 || left > N) ? N : left, (right < 0 || right > N) ? N : right};
 }
 
-// Work-unit counter slot for the next dynamically scheduled launch (rotates over
-// attn::kSchedSlots; concurrent launches in flight take different slots).
-int next_sched_slot() {
+// Work-unit counter slot and generation for the next dynamically scheduled launch:
+// slots rotate over attn::kSchedSlots, the generation counts launches (never 0), so
+// a launch can tell when a later one has taken its slot over.
+struct SchedTicket {
+  int slot;
+  unsigned int gen;
+};
+SchedTicket next_sched_ticket() {
   static std::atomic<unsigned> n{0};
-  return static_cast<int>(n.fetch_add(1, std::memory_order_relaxed) % attn::kSchedSlots);
+  const unsigned v = n.fetch_add(1, std::memory_order_relaxed);
+  return {static_cast<int>(v % attn::kSchedSlots), v + 1u == 0u ? 1u : v + 1u};
 }
 
 // Forward: two query tiles per CTA (fwd_pp.cuh); F8: e4m3 inputs with descales
@@ -147,8 +153,10 @@ int launch_fwd_pp(const void* q, const void* k, const void* v, void* o, float* l
   // interleave the last groups that hold about two units per CTA
   int tail = (2 * grid + upg - 1) / upg;
   p.tail_groups = tail < 1 ? 1 : (tail > B * Hkv ? B * Hkv : tail);
-  p.sched_slot = next_sched_slot();
-  attn::sched_reset_kernel<<<1, 32, 0, stream>>>(p.sched_slot);
+  const SchedTicket ticket = next_sched_ticket();
+  p.sched_slot = ticket.slot;
+  p.sched_gen = ticket.gen;
+  attn::sched_reset_kernel<<<1, 32, 0, stream>>>(ticket.slot, ticket.gen);
   attn::attn_fwd_pp_kernel<D, F8><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
@@ -235,9 +243,11 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.causal = causal;
   p.c = attn::folded_scale(scale);
   p.n_units = static_cast<int>(pl.units);
-  p.sched_slot = next_sched_slot();
+  const SchedTicket ticket = next_sched_ticket();
+  p.sched_slot = ticket.slot;
+  p.sched_gen = ticket.gen;
   const int grid = pl.units < di.sms ? static_cast<int>(pl.units) : di.sms;
-  attn::sched_reset_kernel<<<1, 32, 0, stream>>>(p.sched_slot);
+  attn::sched_reset_kernel<<<1, 32, 0, stream>>>(ticket.slot, ticket.gen);
   attn::attn_decode_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tk, tv, p);
   if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   if (pl.S > 1) {
@@ -575,9 +585,43 @@ __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
 __global__ void selftest_bounds_kernel() {
   if (threadIdx.x == 0) (void)attn::in_range(5, 3);
 }
+// Runs the work-unit claim on the self-test slot as launch generation `gen`: one
+// producer posts `count` claims (of n = 3 units) into a ring, the warp takes them
+// and writes them to out[0 .. count).
+__global__ void selftest_sched_kernel(int* out, unsigned int gen, int count) {
+  __shared__ attn::UnitRing ring;
+  const int lane = threadIdx.x;
+  if (lane == 0) {
+    attn::unit_ring_init(ring, 1);
+    attn::fence_barrier_init();
+  }
+  __syncwarp();
+  if (lane == 0)
+    for (int k = 0; k < count; ++k) (void)attn::unit_ring_claim(ring, k, attn::kSchedSelftestSlot, gen, 3);
+  __syncwarp();
+  for (int k = 0; k < count; ++k) {
+    bool ok = true;
+    const int u = attn::unit_ring_take(ring, k, lane, ok);
+    if (lane == 0) out[k] = ok ? u : -2;
+  }
+}
 }  // namespace
 
 extern "C" {
+
+int attn_selftest_sched(int* out, void* stream) {
+  if (out == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(out) % alignof(int) != 0) return ATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // generation 7 claims units 0, 1, 2 and then none; after generation 8 takes the
+  // slot over, generation 7 gets nothing (and records the conflict) while 8 starts at 0
+  attn::sched_reset_kernel<<<1, 32, 0, s>>>(attn::kSchedSelftestSlot, 7u);
+  selftest_sched_kernel<<<1, 32, 0, s>>>(out, 7u, 4);
+  attn::sched_reset_kernel<<<1, 32, 0, s>>>(attn::kSchedSelftestSlot, 8u);
+  selftest_sched_kernel<<<1, 32, 0, s>>>(out + 4, 7u, 1);
+  selftest_sched_kernel<<<1, 32, 0, s>>>(out + 5, 8u, 1);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
 
 int attn_selftest_timeout(long long limit_ns, void* stream) {
   if (limit_ns <= 0 || limit_ns > 1000000000LL) return ATTN_ERR_INVALID_ARG;
@@ -591,7 +635,8 @@ int attn_get_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&v, attn::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
   if (v != 0 && cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int)) != cudaSuccess)
     return ATTN_ERR_LAUNCH;
-  return v == 0 ? ATTN_OK : v == 2 ? ATTN_ERR_DEVICE_BOUNDS : ATTN_ERR_DEVICE_TIMEOUT;
+  return v == 0 ? ATTN_OK : v == 2 ? ATTN_ERR_DEVICE_BOUNDS : v == 3 ? ATTN_ERR_SCHED_CONFLICT
+                                                                       : ATTN_ERR_DEVICE_TIMEOUT;
 }
 
 int attn_checks_enabled(void) { return attn::kChecks ? 1 : 0; }
@@ -612,6 +657,8 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_WORKSPACE: return "backward workspace too small";
     case ATTN_ERR_ALLOC: return "stream-ordered allocation of the library's workspace failed";
     case ATTN_ERR_DEVICE_BOUNDS: return "a device-side index check failed (checking build)";
+    case ATTN_ERR_SCHED_CONFLICT:
+      return "a launch's work counter was taken over by a later launch (too many in flight); it stopped early";
     default: return "unknown status";
   }
 }

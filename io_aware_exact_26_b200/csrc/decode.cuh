@@ -45,6 +45,7 @@ struct DecParams {
   float c;      // scale * log2(e), floored (folded_scale)
   int n_units;
   int sched_slot;
+  unsigned int sched_gen;
 };
 
 struct DecUnit {
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     int u = 0;
     for (int k = 0; ok; ++k) {
-      if (lane == 0) u = unit_ring_claim(sh.ring, k, p.sched_slot, p.n_units);
+      if (lane == 0) u = unit_ring_claim(sh.ring, k, p.sched_slot, p.sched_gen, p.n_units);
       u = __shfl_sync(0xffffffffu, u, 0);
       if (u < 0) break;
       const DecUnit w = dec_unit(p, u);

@@ -40,6 +40,7 @@ struct FwdParams {
   int desc;         // list query tiles last-first (their key ranges grow with the tile)
   int tail_groups;  // number of last KV groups whose units are interleaved (1 <= . <= B * Hkv)
   int sched_slot;   // g_sched slot this launch claims work units from
+  unsigned int sched_gen;   // the launch's generation in that slot
 };
 
 // Key tiles [j0, j0 + n) that query tile qt sees (n >= 1 for a tile with a row < N).

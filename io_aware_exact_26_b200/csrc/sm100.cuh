@@ -18,14 +18,18 @@ namespace attn {
 __device__ int g_attn_status = 0;
 
 // Work-unit counters for dynamically scheduled kernels: each launch takes one
-// slot (rotated by the host), zeroed by sched_reset_kernel on the same stream
-// just before the launch, so launches in flight on different streams never share
-// a counter and a launch that ended early cannot leave a stale count behind.
+// slot (rotated by the host) and a generation number; sched_reset_kernel, on the
+// same stream just before the launch, sets the slot to (generation << 32) | 0.  A
+// claim increments the low half only while the high half still holds the launch's
+// own generation, so a launch whose slot was taken over by a later one (more than
+// kSchedSlots launches in flight at once) stops claiming, records error 3 and
+// leaves the later launch's counter untouched.
 constexpr int kSchedSlots = 128;
-__device__ unsigned int g_sched[kSchedSlots];
+constexpr int kSchedSelftestSlot = kSchedSlots;   // one more, used only by the scheduler self-test
+__device__ unsigned long long g_sched[kSchedSlots + 1];
 
-__global__ void sched_reset_kernel(int slot) {
-  if (threadIdx.x == 0) g_sched[slot] = 0u;
+__global__ void sched_reset_kernel(int slot, unsigned int gen) {
+  if (threadIdx.x == 0) g_sched[slot] = static_cast<unsigned long long>(gen) << 32;
 }
 
 __device__ __forceinline__ void record_error(int* status, int code) {
@@ -171,12 +175,28 @@ __device__ __forceinline__ void unit_ring_init(UnitRing& r, uint32_t consumers) 
   }
 }
 
-// Producer (one thread): claim the k-th unit of this CTA from counter `slot`,
-// post it (or -1 once u >= n), return it; -2 if a wait failed.
-__device__ __forceinline__ int unit_ring_claim(UnitRing& r, int k, int slot, int n) {
+// Producer (one thread): claim the k-th unit of this CTA from counter `slot` of
+// generation `gen`, post it (or -1 once u >= n, or once the slot belongs to a later
+// launch), return it; -2 if a wait failed.
+__device__ __forceinline__ int unit_ring_claim(UnitRing& r, int k, int slot, unsigned int gen, int n) {
   const int i = k & 3;
   if (k >= 4 && !mbar_wait(&r.empty[i], ((k >> 2) - 1) & 1)) return -2;
-  int u = static_cast<int>(atomicAdd(&g_sched[slot], 1u));
+  int u = -1;
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(&g_sched[slot]);
+  // every failed compare-and-swap means another CTA's succeeded, so this ends after at
+  // most one try per CTA of the launch; the cap only keeps the loop visibly bounded
+  for (int tries = 0; tries < 100000; ++tries) {
+    if (static_cast<unsigned int>(cur >> 32) != gen) {
+      record_error(&g_attn_status, 3);
+      break;
+    }
+    const unsigned long long prev = atomicCAS(&g_sched[slot], cur, cur + 1);
+    if (prev == cur) {
+      u = static_cast<int>(cur & 0xffffffffull);
+      break;
+    }
+    cur = prev;
+  }
   if (u >= n) u = -1;
   r.idx[i] = u;
   mbar_arrive(&r.full[i]);              // release: the index is visible before the arrival

@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
         ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
          "attn_status_string", "attn_selftest_timeout", "attn_fwd_window", "attn_bwd_window", "attn_decode",
          "attn_decode_workspace_size", "attn_decode_splits", "attn_merge", "attn_fwd_fp8", "attn_checks_enabled",
-         "attn_selftest_bounds"])
+         "attn_selftest_bounds", "attn_selftest_sched"])
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    texts = {code: binding.attn_status_string(code) for code in range(-8, 1)}
+    texts = {code: binding.attn_status_string(code) for code in range(-9, 1)}
     assert all(t and t != "unknown status" for t in texts.values())
     assert len(set(texts.values())) == len(texts)
     assert binding.attn_status_string(-99) == "unknown status"
@@ -109,6 +109,11 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "library_path", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         binding.lib()
+
+
+def test_selftest_sched_rejects_null_and_misaligned_output(L):
+    assert L.attn_selftest_sched(None, None) == -1
+    assert L.attn_selftest_sched(ctypes.c_void_p(0x1002), None) == -3
 
 
 def test_selftest_timeout_rejects_out_of_range_limits(L):
