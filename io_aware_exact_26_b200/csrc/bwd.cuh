@@ -154,9 +154,13 @@ template <int D>
 struct KvCfg {
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kBox = 128 * 128;
-  static constexpr int kThreads = 320;
-  // TMEM columns: S^T (lane = key, column = query), P^T as bf16 over it (queries
-  // 0-63 in columns 0-31, queries 64-127 in columns 64-95: each dS warpgroup
+  static constexpr int kGroups = 2;                      // dS warpgroups: kCols queries of every step each
+  static constexpr int kCols = 128 / kGroups;
+  static constexpr int kDsWarps = 4 * kGroups;
+  static constexpr int kWarpLoad = kDsWarps, kWarpMma = kDsWarps + 1;
+  static constexpr int kThreads = 32 * (kDsWarps + 2);   // dS warps, TMA, MMA
+  // TMEM columns: S^T (lane = key, column = query), P^T as bf16 over it (warpgroup g
+  // packs its kCols queries into the first kCols / 2 of the columns it read, so it
   // overwrites only columns it has read); dP^T with dS^T as bf16 over it (same
   // placement); dV and dK accumulators (D columns each).
   static constexpr int kS = 0, kDP = 128, kDV = 256, kDK = 256 + D;
@@ -168,6 +172,7 @@ struct KvCfg {
   static constexpr int kOffBar = kOffVec + 2048;
   static constexpr int kLayout = kOffBar + 256;
   static constexpr int kSmem = kLayout + 1024;
+  static_assert(kSmem <= 232448, "shared memory layout exceeds 227 KB");
 };
 
 struct KvShared {
@@ -180,6 +185,7 @@ struct KvShared {
   uint64_t drain;
   uint32_t tmem_base;
 };
+static_assert(sizeof(KvShared) <= 256, "KvShared does not fit its slot");
 
 // Work units of the dK/dV kernel, numbered KV head by KV head, so the CTAs running at
 // the same time stream the Q/dO of the same few head groups.
@@ -218,8 +224,14 @@ __device__ __forceinline__ void kv_q_range(const BwdParams& p, int j, int& i0, i
 // s-th query tile an item visits, s in [0, i1 - i0]
 __device__ __forceinline__ int kv_q_tile(int i0, int i1, bool up, int s) { return up ? i0 + s : i1 - s; }
 
+// TMEM column of the k-th 16-element slice of a packed bf16 operand written by
+// warpgroups of `cols` fp32 columns each (see the TMEM plans of the configs).
+__device__ __forceinline__ constexpr uint32_t packed_col(int k, int cols) {
+  return static_cast<uint32_t>(cols * (k / (cols / 16)) + (k % (cols / 16)) * 8);
+}
+
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
     attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
                        const BwdParams p) {
@@ -243,10 +255,10 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(&sh.s_full, 1);
     mbar_init(&sh.dp_full, 1);
-    mbar_init(&sh.p_ready, 8);
-    mbar_init(&sh.ds_ready, 8);
+    mbar_init(&sh.p_ready, C::kDsWarps);
+    mbar_init(&sh.ds_ready, C::kDsWarps);
     mbar_init(&sh.k_done, 1);
-    mbar_init(&sh.acc_free, 8);
+    mbar_init(&sh.acc_free, C::kDsWarps);
     mbar_init(&sh.drain, 1);
     fence_barrier_init();
   }
@@ -256,7 +268,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 8) {
+  if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv); tma_prefetch_desc(&tmdo);
@@ -310,7 +322,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int g = max(0, nq - 2); g < nq; ++g) mbar_drain_wait(&sh.qdo_full[g & 1], (g >> 1) & 1);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == C::kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     // Order per step g:  dV(g) S^T(g+1) dK(g) dP^T(g+1).  The exps of step g+1
     // (phase A) run under dK(g) and dP^T(g+1); dS of step g (phase B) under dV(g)
@@ -384,7 +396,7 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t do_mn = do_mn0 + st * (C::kTile >> 4);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts_lo(tmem + C::kDV, tmem + C::kS + (k >> 2) * 64 + (k & 3) * 8, do_mn + ((k * 2048) >> 4), hi,
+            umma_ts_lo(tmem + C::kDV, tmem + C::kS + packed_col(k, C::kCols), do_mn + ((k * 2048) >> 4), hi,
                        idKV, !(u == 0 && k == 0));
         }
         __syncwarp();
@@ -397,7 +409,7 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t q_mn = q_mn0 + st * (C::kTile >> 4);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts_lo(tmem + C::kDK, tmem + C::kDP + (k >> 2) * 64 + (k & 3) * 8, q_mn + ((k * 2048) >> 4), hi,
+            umma_ts_lo(tmem + C::kDK, tmem + C::kDP + packed_col(k, C::kCols), q_mn + ((k * 2048) >> 4), hi,
                        idKV, !(u == 0 && k == 0));
           umma_commit(&sh.k_done);
           umma_commit(&sh.qdo_empty[st]);
@@ -416,8 +428,10 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ dS warpgroups (rows = keys)
-    // warps 0-3: queries 0-63 of every step and the dV epilogue; warps 4-7: queries
-    // 64-127 and the dK epilogue.
+    // warpgroup hb (warps 4hb .. 4hb+3): queries kCols*hb .. kCols*hb + kCols-1 of
+    // every step; in the item's epilogue the first half of the warpgroups writes dV,
+    // the second half dK.
+    constexpr int CW = C::kCols;
     const int hb = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -437,24 +451,24 @@ __global__ void __launch_bounds__(320, 1)
         const int i = kv_q_tile(i0, i1, up, s);
         for (int h = 0; h < p.G && ok; ++h, ++gs) {
           const int st = gs & 1;
-          const float* sLse = sVec + st * 256 + 64 * hb;
+          const float* sLse = sVec + st * 256 + CW * hb;
           const float* sDd = sLse + 128;
-          // visible query columns (relative to this warpgroup's 64) for this key row:
+          // visible query columns (relative to this warpgroup's CW) for this key row:
           // queries key - wr .. key + wl
-          const int qbase = i * 128 + 64 * hb;
+          const int qbase = i * 128 + CW * hb;
           const int hi = key_live ? (min(p.N - 1, key + p.wl) - qbase) : -1;
           const int lo = key - p.wr - qbase;
-          const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= 63);
+          const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= CW - 1);
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.qdo_full[st], (gs >> 1) & 1));
           if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full, gs & 1));
           if (!ok) break;
           tc_fence_after();
           // ---- phase A: P^T = exp2(S^T c - lse2); bf16 into TMEM, fp32 kept for phase B
-          float pf[64];
+          float pf[CW];
 #pragma unroll
-          for (int q16 = 0; q16 < 4; ++q16) {
+          for (int q16 = 0; q16 < CW / 16; ++q16) {
             uint32_t sr[16];
-            tmem_ld16(lane_base + C::kS + 64 * hb + q16 * 16, sr);
+            tmem_ld16(lane_base + C::kS + CW * hb + q16 * 16, sr);
             float lv[16];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -467,7 +481,7 @@ __global__ void __launch_bounds__(320, 1)
             uint32_t pk[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k], pf[q16 * 16 + 2 * k + 1]);
-            tmem_st8(lane_base + C::kS + 64 * hb + q16 * 8, pk);
+            tmem_st8(lane_base + C::kS + CW * hb + q16 * 8, pk);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -478,9 +492,9 @@ __global__ void __launch_bounds__(320, 1)
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int q16 = 0; q16 < 4; ++q16) {
+          for (int q16 = 0; q16 < CW / 16; ++q16) {
             uint32_t dr[16];
-            tmem_ld16(lane_base + C::kDP + 64 * hb + q16 * 16, dr);
+            tmem_ld16(lane_base + C::kDP + CW * hb + q16 * 16, dr);
             float dv[16];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -494,7 +508,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int k = 0; k < 8; ++k)
               dk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k] * (__uint_as_float(dr[2 * k]) - dv[2 * k]),
                                   pf[q16 * 16 + 2 * k + 1] * (__uint_as_float(dr[2 * k + 1]) - dv[2 * k + 1]));
-            tmem_st8(lane_base + C::kDP + 64 * hb + q16 * 8, dk);
+            tmem_st8(lane_base + C::kDP + CW * hb + q16 * 8, dk);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -503,16 +517,19 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (!ok) break;
-      // epilogue of the item (TMEM lane = key): warps 0-3 write dV, warps 4-7 scale * dK
+      // epilogue of the item (TMEM lane = key): the first half of the warpgroups writes
+      // dV, the second half scale * dK, each warpgroup every (kGroups / 2)-th 32 columns
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.k_done, (gs - 1) & 1));
       if (!ok) break;
       tc_fence_after();
+      constexpr int kHalf = C::kGroups / 2;
+      const bool is_dv = hb < kHalf;
       const bool live = key < p.N && in_range(bhkv, static_cast<long long>(p.B) * p.Hkv);
-      const float mul = hb == 0 ? 1.f : p.scale;
-      __nv_bfloat16* dst = (hb == 0 ? p.dv : p.dk) + (static_cast<size_t>(bhkv) * p.N + key) * D;
-      const uint32_t col = hb == 0 ? C::kDV : C::kDK;
+      const float mul = is_dv ? 1.f : p.scale;
+      __nv_bfloat16* dst = (is_dv ? p.dv : p.dk) + (static_cast<size_t>(bhkv) * p.N + key) * D;
+      const uint32_t col = is_dv ? C::kDV : C::kDK;
 #pragma unroll 1
-      for (int q4 = 0; q4 < D / 32; ++q4) {
+      for (int q4 = hb % kHalf; q4 < D / 32; q4 += kHalf) {
         uint32_t x[32];
         tmem_ld32(lane_base + col + q4 * 32, x);
         tmem_wait_ld();
@@ -546,24 +563,31 @@ template <int D>
 struct QCfg {
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kBox = 128 * 128;
-  static constexpr int kThreads = 352;                   // 8 dS warps, K/Q/dO TMA, MMA, V TMA
-  static constexpr int KVST = 2;                         // K/V ring stages
+  static constexpr int kGroups = 2;                      // dS warpgroups: kCols keys of every step each
+  static constexpr int kCols = 128 / kGroups;
+  static constexpr int kDsWarps = 4 * kGroups;
+  static constexpr int kWarpLoad = kDsWarps, kWarpMma = kDsWarps + 1, kWarpV = kDsWarps + 2;
+  static constexpr int kThreads = 32 * (kDsWarps + 3);   // dS warps, K/Q/dO TMA, MMA, V TMA
+  static constexpr int KST = 3;                          // K ring stages (a K tile is held until dQ(j) is done)
+  static constexpr int VST = 2;                          // V ring stages
   // TMEM columns: two S buffers (lane = query, column = key) with dS as bf16 over
-  // them (keys 0-63 in columns 0-31, keys 64-127 in columns 64-95 of the buffer),
-  // dP, and the dQ accumulator.
+  // them (warpgroup g packs its kCols keys into the first kCols / 2 of the columns
+  // it read), dP, and the dQ accumulator.
   static constexpr int kS0 = 0, kS1 = 128, kDP = 256, kDQ = 384;
   static constexpr int kTmemCols = 512;
   static constexpr int kOffQ = 0, kOffDO = kTile;
-  static constexpr int kOffK = 2 * kTile;                // KVST stages
-  static constexpr int kOffV = kOffK + KVST * kTile;     // KVST stages
-  static constexpr int kOffBar = kOffV + KVST * kTile;
+  static constexpr int kOffK = 2 * kTile;                // KST stages
+  static constexpr int kOffV = kOffK + KST * kTile;      // VST stages
+  static constexpr int kOffBar = kOffV + VST * kTile;
   static constexpr int kLayout = kOffBar + 256;
   static constexpr int kSmem = kLayout + 1024;
+  static_assert(KST <= 4 && VST <= 4, "ring barriers hold 4 stages");
+  static_assert(kSmem <= 232448, "shared memory layout exceeds 227 KB");
 };
 
 struct QShared {
   uint64_t qdo_full, qdo_empty;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2];           // S(j) in buffer j % 2
   uint64_t dp_full;             // dP(j)
   uint64_t dp_free;             // dP(j) read by both warpgroups
@@ -573,6 +597,7 @@ struct QShared {
   uint64_t drain;
   uint32_t tmem_base;
 };
+static_assert(sizeof(QShared) <= 256, "QShared does not fit its slot");
 
 // Work units of the dQ kernel, numbered KV head by KV head (the G query heads of a
 // group interleaved), so CTAs running at the same time share K/V in L2.
@@ -606,7 +631,7 @@ __device__ __forceinline__ void q_kv_range(const BwdParams& p, int i, int& j0, i
 }
 
 template <int D>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(QCfg<D>::kThreads, 1)
     attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
                       const BwdParams p) {
@@ -623,18 +648,20 @@ __global__ void __launch_bounds__(352, 1)
   if (threadIdx.x == 0) {
     mbar_init(&sh.qdo_full, 1);
     mbar_init(&sh.qdo_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&sh.k_full[i], 1);
       mbar_init(&sh.k_empty[i], 1);
       mbar_init(&sh.v_full[i], 1);
       mbar_init(&sh.v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.s_full[i], 1);
       mbar_init(&sh.q_done[i], 1);
     }
     mbar_init(&sh.dp_full, 1);
-    mbar_init(&sh.dp_free, 8);
-    mbar_init(&sh.ds_ready, 8);
-    mbar_init(&sh.acc_free, 8);
+    mbar_init(&sh.dp_free, C::kDsWarps);
+    mbar_init(&sh.ds_ready, C::kDsWarps);
+    mbar_init(&sh.acc_free, C::kDsWarps);
     mbar_init(&sh.drain, 1);
     fence_barrier_init();
   }
@@ -644,7 +671,7 @@ __global__ void __launch_bounds__(352, 1)
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  if (warp == 8) {
+  if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------ TMA producer: Q, dO and K
     if (lane == 0) {
       tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmdo);
@@ -668,8 +695,8 @@ __global__ void __launch_bounds__(352, 1)
         }
         nqd = it + 1;
         for (int j = 0; j < n_kv && ok; ++j) {
-          const int g = gj + j, st = g % C::KVST;
-          if (g >= C::KVST) ok = mbar_wait(&sh.k_empty[st], ((g / C::KVST) - 1) & 1);
+          const int g = gj + j, st = g % C::KST;
+          if (g >= C::KST) ok = mbar_wait(&sh.k_empty[st], ((g / C::KST) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.k_full[st], C::kTile);
           in_range(j0 + j, p.nt);
@@ -682,10 +709,10 @@ __global__ void __launch_bounds__(352, 1)
       }
       if (!ok) {
         if (nqd >= 1) mbar_drain_wait(&sh.qdo_full, (nqd - 1) & 1);
-        for (int g = max(0, nk - C::KVST); g < nk; ++g) mbar_drain_wait(&sh.k_full[g % C::KVST], (g / C::KVST) & 1);
+        for (int g = max(0, nk - C::KST); g < nk; ++g) mbar_drain_wait(&sh.k_full[g % C::KST], (g / C::KST) & 1);
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == C::kWarpV) {
     // ------------------------------------------------------------ TMA producer: V
     if (lane == 0) {
       tma_prefetch_desc(&tmv);
@@ -699,8 +726,8 @@ __global__ void __launch_bounds__(352, 1)
         int j0, n_kv;
         q_kv_range(p, i, j0, n_kv);
         for (int j = 0; j < n_kv && ok; ++j) {
-          const int g = gj + j, st = g % C::KVST;
-          if (g >= C::KVST) ok = mbar_wait(&sh.v_empty[st], ((g / C::KVST) - 1) & 1);
+          const int g = gj + j, st = g % C::VST;
+          if (g >= C::VST) ok = mbar_wait(&sh.v_empty[st], ((g / C::VST) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.v_full[st], C::kTile);
           for (int c = 0; c < D / 64; ++c)
@@ -710,9 +737,9 @@ __global__ void __launch_bounds__(352, 1)
         gj += n_kv;
       }
       if (!ok)
-        for (int g = max(0, nv - C::KVST); g < nv; ++g) mbar_drain_wait(&sh.v_full[g % C::KVST], (g / C::KVST) & 1);
+        for (int g = max(0, nv - C::VST); g < nv; ++g) mbar_drain_wait(&sh.v_full[g % C::VST], (g / C::VST) & 1);
     }
-  } else if (warp == 9) {
+  } else if (warp == C::kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     // Order per step j:  S(j+1)  [dS(j)] dQ(j)  dP(j+1).  The warpgroups' exps of step
     // j+1 run under dQ(j) and dP(j+1); dS of step j needs dP(j).  The whole warp
@@ -730,8 +757,8 @@ __global__ void __launch_bounds__(352, 1)
     int gj = 0, it = 0;
     bool ok = true;
     auto issue_s = [&](int g) -> bool {     // S(g) = Q K(g)^T into buffer g % 2
-      const int st = g % C::KVST, sb = g & 1;
-      if (!wait(&sh.k_full[st], (g / C::KVST) & 1)) return false;
+      const int st = g % C::KST, sb = g & 1;
+      if (!wait(&sh.k_full[st], (g / C::KST) & 1)) return false;
       // S(g) overwrites dS(g-2): issued behind dQ(g-2), performed after it.
       tc_fence_after();
       if (leader) {
@@ -747,8 +774,8 @@ __global__ void __launch_bounds__(352, 1)
       return true;
     };
     auto issue_dp = [&](int g) -> bool {    // dP(g) = dO V(g)^T
-      const int st = g % C::KVST;
-      if (!wait(&sh.v_full[st], (g / C::KVST) & 1)) return false;
+      const int st = g % C::VST;
+      if (!wait(&sh.v_full[st], (g / C::VST) & 1)) return false;
       if (g >= 1 && !wait(&sh.dp_free, (g - 1) & 1)) return false;       // dP(g-1) read
       tc_fence_after();
       if (leader) {
@@ -774,7 +801,7 @@ __global__ void __launch_bounds__(352, 1)
       if (!ok) break;
       ok = issue_s(gj) && issue_dp(gj);
       for (int u = 0; u < n_kv && ok; ++u) {
-        const int g = gj + u, st = g % C::KVST, sb = g & 1;
+        const int g = gj + u, st = g % C::KST, sb = g & 1;
         if (u + 1 < n_kv && !issue_s(g + 1)) { ok = false; break; }
         // dQ += dS K  (A = dS in TMEM, M = queries, K = keys; B = K MN-major)
         ok = wait(&sh.ds_ready, g & 1);
@@ -786,7 +813,7 @@ __global__ void __launch_bounds__(352, 1)
           const uint32_t sbase = tmem + (sb ? C::kS1 : C::kS0);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts_lo(tmem + C::kDQ, sbase + (k >> 2) * 64 + (k & 3) * 8, k_mn + ((k * 2048) >> 4), hi, idQ,
+            umma_ts_lo(tmem + C::kDQ, sbase + packed_col(k, C::kCols), k_mn + ((k * 2048) >> 4), hi, idQ,
                        !(u == 0 && k == 0));
           umma_commit(&sh.q_done[sb]);
           umma_commit(&sh.k_empty[st]);
@@ -805,8 +832,9 @@ __global__ void __launch_bounds__(352, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ dS warpgroups (rows = queries)
-    // warps 0-3: keys 0-63 of every step, warps 4-7: keys 64-127.  The row's LSE and D
-    // are this thread's own, held in registers for the whole item.
+    // warpgroup hb (warps 4hb .. 4hb+3): keys kCols*hb .. kCols*hb + kCols-1 of every
+    // step.  The row's LSE and D are this thread's own, held in registers for the item.
+    constexpr int CW = C::kCols;
     const int hb = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -828,20 +856,20 @@ __global__ void __launch_bounds__(352, 1)
       for (int k = 0; k < 16; ++k) lv[k] = l2;
       for (int u = 0; u < n_kv && ok; ++u) {
         const int g = gj + u, sb = g & 1;
-        const uint32_t sbase = lane_base + (sb ? C::kS1 : C::kS0) + 64 * hb;
-        // visible key columns (relative to this warpgroup's 64) for this query row:
+        const uint32_t sbase = lane_base + (sb ? C::kS1 : C::kS0) + CW * hb;
+        // visible key columns (relative to this warpgroup's CW) for this query row:
         // keys qrow - wl .. qrow + wr
-        const int kbase = (j0 + u) * 128 + 64 * hb;
+        const int kbase = (j0 + u) * 128 + CW * hb;
         const int hi = min(p.N - 1, qrow + p.wr) - kbase;
         const int lo = qrow - p.wl - kbase;
-        const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= 63);
+        const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= CW - 1);
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[sb], (g >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        // phase A: P = exp2(S c - lse2) for this warpgroup's 64 keys
-        float pf[64];
+        // phase A: P = exp2(S c - lse2) for this warpgroup's CW keys
+        float pf[CW];
 #pragma unroll
-        for (int q16 = 0; q16 < 4; ++q16) {
+        for (int q16 = 0; q16 < CW / 16; ++q16) {
           uint32_t sr[16];
           tmem_ld16(sbase + q16 * 16, sr);
           tmem_wait_ld();
@@ -853,9 +881,9 @@ __global__ void __launch_bounds__(352, 1)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int q16 = 0; q16 < 4; ++q16) {
+        for (int q16 = 0; q16 < CW / 16; ++q16) {
           uint32_t dr[16];
-          tmem_ld16(lane_base + C::kDP + 64 * hb + q16 * 16, dr);
+          tmem_ld16(lane_base + C::kDP + CW * hb + q16 * 16, dr);
           tmem_wait_ld();
           reg_fence(dr);
           uint32_t dk[8];
@@ -874,7 +902,7 @@ __global__ void __launch_bounds__(352, 1)
         if (lane == 0) mbar_arrive(&sh.ds_ready);
       }
       if (!ok) break;
-      // epilogue: dQ (TMEM lane = query row), scaled, bf16; the two warpgroups split the columns
+      // epilogue: dQ (TMEM lane = query row), scaled, bf16; the warpgroups split the columns
       const int glast = gj + n_kv - 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.q_done[glast & 1], (glast >> 1) & 1));
       if (!ok) break;
@@ -882,7 +910,7 @@ __global__ void __launch_bounds__(352, 1)
       const bool live = qrow < p.N && in_range(bhq, static_cast<long long>(p.B) * p.Hq);
       __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bhq) * p.N + qrow) * D;
 #pragma unroll 1
-      for (int q4 = hb; q4 < D / 32; q4 += 2) {
+      for (int q4 = hb; q4 < D / 32; q4 += C::kGroups) {
         uint32_t x[32];
         tmem_ld32(lane_base + C::kDQ + q4 * 32, x);
         tmem_wait_ld();
