@@ -64,9 +64,9 @@ typedef enum {
  * that counter.  Each call takes the next of 128 counters (rotating, shared with
  * attn_fwd_window, attn_fwd_fp8 and attn_decode), so up to 128 such calls may be in
  * flight at once, on any streams.  Beyond that, a call whose counter is taken over
- * by a later one stops claiming work, leaves its outputs incomplete and reports
- * ATTN_ERR_SCHED_CONFLICT through attn_get_device_status(); the later call is
- * unaffected. */
+ * by a later one stops claiming work and ATTN_ERR_SCHED_CONFLICT is reported through
+ * attn_get_device_status(); the outputs of both calls are then incomplete (a stale
+ * claim may also use up one of the later call's work units). */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
              void* stream);
@@ -231,9 +231,10 @@ int attn_selftest_timeout(long long limit_ns, void* stream);
  * a reset of that counter to launch generation 7; one CTA of generation 7 claiming
  * four times from 3 work units; a reset to generation 8; one CTA of generation 7
  * claiming once; one CTA of generation 8 claiming once.  `out` is a device array of
- * at least 6 ints; the claims land there in that order and read 0 1 2 -1 -1 0 (-1 =
- * no unit), and the following attn_get_device_status() returns
- * ATTN_ERR_SCHED_CONFLICT (generation 7 found the counter taken over).  Returns
+ * at least 6 ints; the claims land there in that order and read 0 1 2 -1 -1 1 (-1 =
+ * no unit; generation 8 starts at 1 because the stale claim used up its unit 0), and
+ * the following attn_get_device_status() returns ATTN_ERR_SCHED_CONFLICT (generation
+ * 7 found the counter taken over).  Returns
  * ATTN_ERR_INVALID_ARG for NULL, ATTN_ERR_ALIGNMENT for a misaligned `out`,
  * ATTN_ERR_LAUNCH if a launch is refused, else ATTN_OK. */
 int attn_selftest_sched(int* out, void* stream);

@@ -352,7 +352,7 @@ def attn_selftest_bounds(stream=None) -> None:
 
 
 def attn_selftest_sched(stream=None) -> list:
-    """Run the work-counter takeover self-test; returns its six claims (0 1 2 -1 -1 0 expected)."""
+    """Run the work-counter takeover self-test; returns its six claims (0 1 2 -1 -1 1 expected)."""
     out = torch.full((8,), -7, dtype=torch.int32, device="cuda")
     st = int(lib().attn_selftest_sched(_ptr(out), _stream_ptr(stream)))
     if st != 0:

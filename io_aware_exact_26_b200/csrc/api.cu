@@ -614,7 +614,8 @@ int attn_selftest_sched(int* out, void* stream) {
   if (reinterpret_cast<uintptr_t>(out) % alignof(int) != 0) return ATTN_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // generation 7 claims units 0, 1, 2 and then none; after generation 8 takes the
-  // slot over, generation 7 gets nothing (and records the conflict) while 8 starts at 0
+  // slot over, generation 7 gets nothing (and records the conflict) and its stray
+  // increment makes generation 8 start at 1
   attn::sched_reset_kernel<<<1, 32, 0, s>>>(attn::kSchedSelftestSlot, 7u);
   selftest_sched_kernel<<<1, 32, 0, s>>>(out, 7u, 4);
   attn::sched_reset_kernel<<<1, 32, 0, s>>>(attn::kSchedSelftestSlot, 8u);
@@ -658,7 +659,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_ALLOC: return "stream-ordered allocation of the library's workspace failed";
     case ATTN_ERR_DEVICE_BOUNDS: return "a device-side index check failed (checking build)";
     case ATTN_ERR_SCHED_CONFLICT:
-      return "a launch's work counter was taken over by a later launch (too many in flight); it stopped early";
+      return "a launch's work counter was taken over by a later launch (over 128 in flight); both outputs are incomplete";
     default: return "unknown status";
   }
 }

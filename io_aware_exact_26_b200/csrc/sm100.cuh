@@ -19,11 +19,14 @@ __device__ int g_attn_status = 0;
 
 // Work-unit counters for dynamically scheduled kernels: each launch takes one
 // slot (rotated by the host) and a generation number; sched_reset_kernel, on the
-// same stream just before the launch, sets the slot to (generation << 32) | 0.  A
-// claim increments the low half only while the high half still holds the launch's
-// own generation, so a launch whose slot was taken over by a later one (more than
-// kSchedSlots launches in flight at once) stops claiming, records error 3 and
-// leaves the later launch's counter untouched.
+// same stream just before the launch, sets the slot to (generation << 32) | 0, and a
+// claim is one 64-bit atomicAdd whose old value carries the generation it counted
+// in.  A claim that finds another generation (more than kSchedSlots launches in
+// flight at once, so a later launch has reset the slot) stops its launch and records
+// error 3; its stray increment may cost the later launch a unit, which is why the
+// error stands for both launches.  A compare-and-swap claim would keep the later
+// launch intact, but it serialises under contention (up to 60% slower measured on
+// workloads of many short units).
 constexpr int kSchedSlots = 128;
 constexpr int kSchedSelftestSlot = kSchedSlots;   // one more, used only by the scheduler self-test
 __device__ unsigned long long g_sched[kSchedSlots + 1];
@@ -176,26 +179,16 @@ __device__ __forceinline__ void unit_ring_init(UnitRing& r, uint32_t consumers) 
 }
 
 // Producer (one thread): claim the k-th unit of this CTA from counter `slot` of
-// generation `gen`, post it (or -1 once u >= n, or once the slot belongs to a later
+// generation `gen`, post it (or -1 once u >= n, or once the slot belongs to another
 // launch), return it; -2 if a wait failed.
 __device__ __forceinline__ int unit_ring_claim(UnitRing& r, int k, int slot, unsigned int gen, int n) {
   const int i = k & 3;
   if (k >= 4 && !mbar_wait(&r.empty[i], ((k >> 2) - 1) & 1)) return -2;
-  int u = -1;
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(&g_sched[slot]);
-  // every failed compare-and-swap means another CTA's succeeded, so this ends after at
-  // most one try per CTA of the launch; the cap only keeps the loop visibly bounded
-  for (int tries = 0; tries < 100000; ++tries) {
-    if (static_cast<unsigned int>(cur >> 32) != gen) {
-      record_error(&g_attn_status, 3);
-      break;
-    }
-    const unsigned long long prev = atomicCAS(&g_sched[slot], cur, cur + 1);
-    if (prev == cur) {
-      u = static_cast<int>(cur & 0xffffffffull);
-      break;
-    }
-    cur = prev;
+  const unsigned long long old = atomicAdd(&g_sched[slot], 1ull);
+  int u = static_cast<int>(old & 0xffffffffull);
+  if (static_cast<unsigned int>(old >> 32) != gen) {
+    record_error(&g_attn_status, 3);
+    u = -1;
   }
   if (u >= n) u = -1;
   r.idx[i] = u;

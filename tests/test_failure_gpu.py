@@ -8,8 +8,8 @@ with a 20 ms limit, so the timeout path runs for real.
 
 The persistent kernels (forward, window, FP8 and decode) claim work units from one of
 128 rotating counters, each tagged with its launch's generation; a launch that finds
-its counter taken over by a later one stops claiming and reports
-ATTN_ERR_SCHED_CONFLICT.  attn_selftest_sched drives that check on a reserved
+its counter taken over by a later one stops claiming and ATTN_ERR_SCHED_CONFLICT is
+reported (both launches' outputs then count as incomplete).  attn_selftest_sched drives that check on a reserved
 counter; the concurrency test keeps many launches in flight on several streams and
 checks that each matches a lone launch of the same call.
 """
@@ -56,10 +56,10 @@ def test_context_is_usable_after_a_timeout(attn):
         assert np.isfinite(f64(lse[0, h])).all()
 
 
-def test_taken_over_counter_stops_the_older_launch_only(attn):
+def test_taken_over_counter_stops_the_older_launch_and_is_reported(attn):
     assert attn.attn_get_device_status() == 0
     claims = attn.attn_selftest_sched()
-    assert claims == [0, 1, 2, -1, -1, 0]
+    assert claims == [0, 1, 2, -1, -1, 1]      # the stale claim used up generation 8's unit 0
     assert attn.attn_get_device_status() == ATTN_ERR_SCHED_CONFLICT
     assert attn.attn_get_device_status() == 0
 
