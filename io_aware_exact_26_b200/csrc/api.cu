@@ -297,8 +297,8 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   const long long BHq = static_cast<long long>(B) * Hq;
   const BwdLayout L = bwd_layout(BHq, N);
   char* ws = static_cast<char*>(workspace);
-  float* lse2 = reinterpret_cast<float*>(ws + L.lse2_off);
-  float* dd = reinterpret_cast<float*>(ws + L.dd_off);
+  float* nlse2 = reinterpret_cast<float*>(ws + L.nlse2_off);
+  float* ndd = reinterpret_cast<float*>(ws + L.ndd_off);
   const int nt = (N + 127) / 128;
   {
     const long long rows = BHq * nt * 128;
@@ -306,7 +306,7 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
     const long long cap = static_cast<long long>(sms) * 16;
     if (blocks > cap) blocks = cap;
     attn_bwd_prep_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dd, BHq, N);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, nlse2, ndd, BHq, N);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   CUtensorMap tq, tk, tv, tdo;
@@ -317,8 +317,8 @@ static int launch_bwd_d(const void* q, const void* k, const void* v, const void*
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.lse2 = lse2;
-  p.dd = dd;
+  p.nlse2 = nlse2;
+  p.ndd = ndd;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;

@@ -38,17 +38,17 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
 }
 
 struct BwdLayout {
-  // workspace carve-up (byte offsets, each 256-byte aligned): lse2 and D per row
-  size_t lse2_off, dd_off, total;
+  // workspace carve-up (byte offsets, each 256-byte aligned): -lse2 and -D per row
+  size_t nlse2_off, ndd_off, total;
 };
 
 __host__ __device__ inline BwdLayout bwd_layout(long long BHq, int N) {
   const long long npad = (N + 127) / 128 * 128;
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   BwdLayout L;
-  L.lse2_off = 0;
-  L.dd_off = up(L.lse2_off + BHq * npad * 4);
-  L.total = up(L.dd_off + BHq * npad * 4);
+  L.nlse2_off = 0;
+  L.ndd_off = up(L.nlse2_off + BHq * npad * 4);
+  L.total = up(L.ndd_off + BHq * npad * 4);
   return L;
 }
 
@@ -59,13 +59,15 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
 }
 
 // ------------------------------------------------------------------ preprocess
-// D_i = sum_k dO_ik O_ik (fp32) and lse2_i = LSE_i * log2(e); padded rows get 0.
+// D_i = sum_k dO_ik O_ik (fp32) and lse2_i = LSE_i * log2(e), both stored negated (the
+// dS warps add them with packed f32x2 FMAs and adds, which take no negated operand);
+// padded rows get 0.
 // Each row is read with 16-byte loads by D/8 lanes, so one warp covers 256/D rows.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dO,
-                                                            const float* __restrict__ lse, float* lse2,
-                                                            float* dd, long long BHq, int N) {
+                                                            const float* __restrict__ lse, float* nlse2,
+                                                            float* ndd, long long BHq, int N) {
   constexpr int LPR = D / 8;             // lanes per row
   constexpr int RPW = 32 / LPR;          // rows per warp pass
   const int npad = (N + 127) / 128 * 128;
@@ -102,8 +104,8 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (part == 0 && r < rows) {
-      dd[r] = acc;
-      lse2[r] = l2;
+      ndd[r] = -acc;
+      nlse2[r] = -l2;
     }
   }
 }
@@ -112,8 +114,8 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  const float* lse2;
-  const float* dd;
+  const float* nlse2;   // -LSE * log2(e) per row (padded to whole tiles)
+  const float* ndd;     // -D per row
   int B, Hq, Hkv, N, G;
   int nt;           // number of 128-row tiles along N
   int npair;        // (nt + 1) / 2: key-tile pairs per KV head (causal dK/dV units)
@@ -125,27 +127,30 @@ struct BwdParams {
   float scale;
 };
 
-// Exps of one 16-column slice of a score tile held by this thread: p = 2^(s c - l).
-// Masked columns (only on band-edge / ragged tiles) get s = -inf first; c > 0 (the
-// host floors it at 1e-30), so p = 0 (or 2^-126.5 on the FMA-pipe path); the exp
-// loop itself has no branch.
-__device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const float (&lv)[16], float c, bool masked,
-                                          int col0, int lo, int hi, float* pf) {
+// Exps of one 16-column slice of a score tile held by this thread, two columns per
+// packed f32x2 instruction: p = 2^(s c + nl) with nl = -lse2 (the column's or the
+// row's).  Masked columns (only on band-edge / ragged tiles) get s = -inf first; c > 0
+// (the host floors it at 1e-30), so p = 0 (or 2^-126.5 on the FMA-pipe path); the exp
+// loop itself has no branch.  pf2[k] holds columns 2k and 2k+1.
+__device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const uint64_t (&nl)[8], uint64_t c2, bool masked,
+                                          int col0, int lo, int hi, uint64_t* pf2) {
   if (masked) {
 #pragma unroll
     for (int k = 0; k < 16; ++k)
       if (col0 + k < lo || col0 + k > hi) sr[k] = 0xff800000u;
   }
 #pragma unroll
-  for (int k = 0; k < 16; k += 2) {
-    const float x0 = fmaf(__uint_as_float(sr[k]), c, -lv[k]);
-    const float x1 = fmaf(__uint_as_float(sr[k + 1]), c, -lv[k + 1]);
-    if ((k & 6) == 6) {
-      exp2_fma_pair(x0, x1, pf[k], pf[k + 1]);   // one pair in four on the FMA pipe
+  for (int k = 0; k < 8; ++k) {
+    const uint64_t x = ffma2(f2pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nl[k]);
+    float x0, x1, y0, y1;
+    f2unpack(x, x0, x1);
+    if ((k & 3) == 3) {
+      exp2_fma_pair(x0, x1, y0, y1);   // one pair in four on the FMA pipe
     } else {
-      pf[k] = ex2_approx(x0);
-      pf[k + 1] = ex2_approx(x1);
+      y0 = ex2_approx(x0);
+      y1 = ex2_approx(x1);
     }
+    pf2[k] = f2pack(y0, y1);
   }
 }
 
@@ -168,7 +173,7 @@ struct KvCfg {
   static constexpr int kOffK = 0, kOffV = kTile;
   static constexpr int kOffQ = 2 * kTile;                // 2 stages
   static constexpr int kOffDO = 4 * kTile;               // 2 stages
-  static constexpr int kOffVec = 6 * kTile;              // per stage: lse2[128], dd[128]
+  static constexpr int kOffVec = 6 * kTile;              // per stage: -lse2[128], -D[128]
   static constexpr int kOffBar = kOffVec + 2048;
   static constexpr int kLayout = kOffBar + 256;
   static constexpr int kSmem = kLayout + 1024;
@@ -243,7 +248,7 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
   uint8_t* sV = smem + C::kOffV;
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sDO = smem + C::kOffDO;
-  float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);   // [stage][lse2 128 | dd 128]
+  float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);   // [stage][-lse2 128 | -D 128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -311,8 +316,8 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
             size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + i * 128;
             in_range(i, p.nt);
             if (!in_range(bhq, static_cast<long long>(p.B) * p.Hq)) vrow = 0;   // keep the bulk copy inside
-            bulk_load(sVec + st * 256, p.lse2 + vrow, 512, &sh.qdo_full[st]);
-            bulk_load(sVec + st * 256 + 128, p.dd + vrow, 512, &sh.qdo_full[st]);
+            bulk_load(sVec + st * 256, p.nlse2 + vrow, 512, &sh.qdo_full[st]);
+            bulk_load(sVec + st * 256 + 128, p.ndd + vrow, 512, &sh.qdo_full[st]);
             nq = gs + 1;
           }
         }
@@ -435,7 +440,7 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
     const int hb = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const float c = p.c;
+    const uint64_t c2 = f2pack(p.c, p.c);
     int gs = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
@@ -451,8 +456,8 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
         const int i = kv_q_tile(i0, i1, up, s);
         for (int h = 0; h < p.G && ok; ++h, ++gs) {
           const int st = gs & 1;
-          const float* sLse = sVec + st * 256 + CW * hb;
-          const float* sDd = sLse + 128;
+          const float* sNlse = sVec + st * 256 + CW * hb;
+          const float* sNdd = sNlse + 128;
           // visible query columns (relative to this warpgroup's CW) for this key row:
           // queries key - wr .. key + wl
           const int qbase = i * 128 + CW * hb;
@@ -463,24 +468,25 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
           if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full, gs & 1));
           if (!ok) break;
           tc_fence_after();
-          // ---- phase A: P^T = exp2(S^T c - lse2); bf16 into TMEM, fp32 kept for phase B
-          float pf[CW];
+          // ---- phase A: P^T = exp2(S^T c - lse2); bf16 into TMEM, fp32 pairs kept for phase B
+          uint64_t pf2[CW / 2];
 #pragma unroll
           for (int q16 = 0; q16 < CW / 16; ++q16) {
             uint32_t sr[16];
             tmem_ld16(lane_base + C::kS + CW * hb + q16 * 16, sr);
-            float lv[16];
+            uint64_t nl[8];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const float4 a = reinterpret_cast<const float4*>(sLse + q16 * 16)[k];
-              lv[4 * k] = a.x; lv[4 * k + 1] = a.y; lv[4 * k + 2] = a.z; lv[4 * k + 3] = a.w;
+              const ulonglong2 a = reinterpret_cast<const ulonglong2*>(sNlse + q16 * 16)[k];
+              nl[2 * k] = a.x;
+              nl[2 * k + 1] = a.y;
             }
             tmem_wait_ld();
             reg_fence(sr);
-            bwd_exp16(sr, lv, c, masked, q16 * 16, lo, hi, pf + q16 * 16);
+            bwd_exp16(sr, nl, c2, masked, q16 * 16, lo, hi, pf2 + q16 * 8);
             uint32_t pk[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k], pf[q16 * 16 + 2 * k + 1]);
+            for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2_2(pf2[q16 * 8 + k]);
             tmem_st8(lane_base + C::kS + CW * hb + q16 * 8, pk);
           }
           tmem_wait_st();
@@ -495,19 +501,20 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
           for (int q16 = 0; q16 < CW / 16; ++q16) {
             uint32_t dr[16];
             tmem_ld16(lane_base + C::kDP + CW * hb + q16 * 16, dr);
-            float dv[16];
+            uint64_t nd[8];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const float4 b = reinterpret_cast<const float4*>(sDd + q16 * 16)[k];
-              dv[4 * k] = b.x; dv[4 * k + 1] = b.y; dv[4 * k + 2] = b.z; dv[4 * k + 3] = b.w;
+              const ulonglong2 b = reinterpret_cast<const ulonglong2*>(sNdd + q16 * 16)[k];
+              nd[2 * k] = b.x;
+              nd[2 * k + 1] = b.y;
             }
             tmem_wait_ld();
             reg_fence(dr);
             uint32_t dk[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              dk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k] * (__uint_as_float(dr[2 * k]) - dv[2 * k]),
-                                  pf[q16 * 16 + 2 * k + 1] * (__uint_as_float(dr[2 * k + 1]) - dv[2 * k + 1]));
+              dk[k] = pack_bf16x2_2(fmul2(pf2[q16 * 8 + k],
+                                          fadd2(f2pack(__uint_as_float(dr[2 * k]), __uint_as_float(dr[2 * k + 1])), nd[k])));
             tmem_st8(lane_base + C::kDP + CW * hb + q16 * 8, dk);
           }
           tmem_wait_st();
@@ -838,7 +845,7 @@ __global__ void __launch_bounds__(QCfg<D>::kThreads, 1)
     const int hb = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const float c = p.c;
+    const uint64_t c2 = f2pack(p.c, p.c);
     int gj = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.total_items && ok; t += gridDim.x)
@@ -850,10 +857,11 @@ __global__ void __launch_bounds__(QCfg<D>::kThreads, 1)
       const int qrow = i * 128 + r;
       size_t vrow = static_cast<size_t>(bhq) * (p.nt * 128) + qrow;
       if (!in_range(static_cast<long long>(vrow), static_cast<long long>(p.B) * p.Hq * p.nt * 128)) vrow = 0;
-      const float l2 = p.lse2[vrow], drow = p.dd[vrow];
-      float lv[16];
+      const float nl2 = p.nlse2[vrow], nd = p.ndd[vrow];
+      uint64_t nl[8];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) lv[k] = l2;
+      for (int k = 0; k < 8; ++k) nl[k] = f2pack(nl2, nl2);
+      const uint64_t nd2 = f2pack(nd, nd);
       for (int u = 0; u < n_kv && ok; ++u) {
         const int g = gj + u, sb = g & 1;
         const uint32_t sbase = lane_base + (sb ? C::kS1 : C::kS0) + CW * hb;
@@ -867,14 +875,14 @@ __global__ void __launch_bounds__(QCfg<D>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         // phase A: P = exp2(S c - lse2) for this warpgroup's CW keys
-        float pf[CW];
+        uint64_t pf2[CW / 2];
 #pragma unroll
         for (int q16 = 0; q16 < CW / 16; ++q16) {
           uint32_t sr[16];
           tmem_ld16(sbase + q16 * 16, sr);
           tmem_wait_ld();
           reg_fence(sr);
-          bwd_exp16(sr, lv, c, masked, q16 * 16, lo, hi, pf + q16 * 16);
+          bwd_exp16(sr, nl, c2, masked, q16 * 16, lo, hi, pf2 + q16 * 8);
         }
         // phase B: dS = P (dP - D) -> bf16 over the S buffer
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.dp_full, g & 1));
@@ -889,8 +897,8 @@ __global__ void __launch_bounds__(QCfg<D>::kThreads, 1)
           uint32_t dk[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            dk[k] = pack_bf16x2(pf[q16 * 16 + 2 * k] * (__uint_as_float(dr[2 * k]) - drow),
-                                pf[q16 * 16 + 2 * k + 1] * (__uint_as_float(dr[2 * k + 1]) - drow));
+            dk[k] = pack_bf16x2_2(fmul2(pf2[q16 * 8 + k],
+                                        fadd2(f2pack(__uint_as_float(dr[2 * k]), __uint_as_float(dr[2 * k + 1])), nd2)));
           tmem_st8(sbase + q16 * 8, dk);
         }
         tc_fence_before();

@@ -446,6 +446,11 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 
 // exp2 of a pair on the FMA pipe, to take load off the MUFU pipe (16 ex2 per SM
 // per clock).  Range reduction x = n + f with n = round(x), |f| <= 1/2, via the
@@ -484,6 +489,13 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two packed fp32 to one bf16x2 word (round to nearest even), first value in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2_2(uint64_t v) {
+  float lo, hi;
+  f2unpack(v, lo, hi);
+  return pack_bf16x2(lo, hi);
 }
 
 }  // namespace attn
