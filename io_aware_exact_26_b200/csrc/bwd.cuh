@@ -131,7 +131,10 @@ struct BwdParams {
 // packed f32x2 instruction: p = 2^(s c + nl) with nl = -lse2 (the column's or the
 // row's).  Masked columns (only on band-edge / ragged tiles) get s = -inf first; c > 0
 // (the host floors it at 1e-30), so p = 0 (or 2^-126.5 on the FMA-pipe path); the exp
-// loop itself has no branch.  pf2[k] holds columns 2k and 2k+1.
+// loop itself has no branch.  pf2[k] holds columns 2k and 2k+1.  One pair in four
+// goes to the FMA pipe, one in two at d = 64 (measured: +2-3% there, no change at
+// d = 128 for none, one or two in four).
+template <int D>
 __device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const uint64_t (&nl)[8], uint64_t c2, bool masked,
                                           int col0, int lo, int hi, uint64_t* pf2) {
   if (masked) {
@@ -144,8 +147,8 @@ __device__ __forceinline__ void bwd_exp16(uint32_t (&sr)[16], const uint64_t (&n
     const uint64_t x = ffma2(f2pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nl[k]);
     float x0, x1, y0, y1;
     f2unpack(x, x0, x1);
-    if ((k & 3) == 3) {
-      exp2_fma_pair(x0, x1, y0, y1);   // one pair in four on the FMA pipe
+    if (D == 64 ? (k & 1) == 1 : (k & 3) == 3) {
+      exp2_fma_pair(x0, x1, y0, y1);
     } else {
       y0 = ex2_approx(x0);
       y1 = ex2_approx(x1);
@@ -483,7 +486,7 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
             }
             tmem_wait_ld();
             reg_fence(sr);
-            bwd_exp16(sr, nl, c2, masked, q16 * 16, lo, hi, pf2 + q16 * 8);
+            bwd_exp16<D>(sr, nl, c2, masked, q16 * 16, lo, hi, pf2 + q16 * 8);
             uint32_t pk[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2_2(pf2[q16 * 8 + k]);
@@ -882,7 +885,7 @@ __global__ void __launch_bounds__(QCfg<D>::kThreads, 1)
           tmem_ld16(sbase + q16 * 16, sr);
           tmem_wait_ld();
           reg_fence(sr);
-          bwd_exp16(sr, nl, c2, masked, q16 * 16, lo, hi, pf2 + q16 * 8);
+          bwd_exp16<D>(sr, nl, c2, masked, q16 * 16, lo, hi, pf2 + q16 * 8);
         }
         // phase B: dS = P (dP - D) -> bf16 over the S buffer
         ok = __all_sync(0xffffffffu, mbar_wait(&sh.dp_full, g & 1));
