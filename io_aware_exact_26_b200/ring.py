@@ -19,12 +19,20 @@ and earlier shards are seen in full.
 B200 notes.  Remote K/V always land in a local buffer first (point-to-point sends
 of the communication backend, NCCL over NVLink on GPUs), so no kernel reads another
 GPU's memory; the transfer of the next shard overlaps the compute of the current
-one.  Every rank takes the same W - 1 exchange steps in the same order, skipped
-compute included.  Only the forward is provided.
+one.  Every rank takes the same exchange steps in the same order, skipped compute
+included.
 
-The partial and merge steps are parameters: on GPUs they are ``attn_fwd`` and
-``attn_merge`` of the CUDA library (the defaults); tests pass other functions to
-check the ring logic on CPU ranks.
+Backward (recompute, as on one GPU): the shards travel the same ring, each with
+fp32 accumulators for its dK and dV.  At step s rank r computes the gradient
+contributions of its query shard against the shard it holds -- with the global LSE
+and O of its rows from the forward, the probabilities and D = rowsum(dO * O) are
+those of the whole sequence -- adds dQ to its own accumulator and dK, dV to the
+travelling ones, and passes them on.  After the last step one more hop brings every
+shard's accumulators back to their owner.
+
+The partial and merge steps are parameters: on GPUs they are ``attn_fwd``,
+``attn_merge`` and ``attn_bwd`` of the CUDA library (the defaults); tests pass other
+functions to check the ring logic on CPU ranks.
 """
 from __future__ import annotations
 
@@ -99,3 +107,56 @@ def ring_attention_fwd(q, k, v, *, causal: bool, group=None, scale=None, partial
         if step + 1 < world:
             cur, nxt = nxt, cur
     return o_acc, lse_acc
+
+
+def _cuda_partial_bwd(q, k, v, o, lse, do, causal, scale):
+    from . import binding
+    return binding.attn_bwd(q, k, v, o, lse, do, scale=scale, causal=causal)
+
+
+def ring_attention_bwd(q, k, v, o, lse, do, *, causal: bool, group=None, scale=None, partial=None,
+                       acc_dtype=torch.float32):
+    """Gradients of this rank's shards, for attention over the whole ring's sequence.
+
+    q, o, do: [B, Hq, n, d]; k, v: [B, Hkv, n, d] -- this rank's shard; lse: [B, Hq, n]
+    (natural log), o and lse being this rank's rows of the forward over the whole
+    sequence (``ring_attention_fwd``; o in the dtype ``partial`` takes).
+    Returns (dq, dk, dv) for this rank's shards in ``acc_dtype``.
+    ``partial(q, k, v, o, lse, do, causal, scale) -> (dq, dk, dv)`` gives one shard
+    pair's contribution; it defaults to the CUDA library's ``attn_bwd``.
+    """
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    partial = partial or _cuda_partial_bwd
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    dq = torch.zeros(q.shape, dtype=acc_dtype, device=q.device)
+    cur = torch.stack((k, v)).contiguous()                          # the shard held at this step
+    nxt = torch.empty_like(cur)
+    acc = torch.zeros((2,) + tuple(k.shape), dtype=acc_dtype, device=q.device)   # its dK, dV so far
+    acc_in = torch.empty_like(acc)
+    nxt_rank = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
+    prv_rank = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
+    for step, src, kind in ring_schedule(rank, world, causal):
+        reqs = []
+        if step + 1 < world:                        # the next shard is in flight during the compute
+            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur, nxt_rank, group),
+                                           dist.P2POp(dist.irecv, nxt, prv_rank, group)])
+        if kind != SKIP:
+            dq_p, dk_p, dv_p = partial(q, cur[0], cur[1], o, lse, do, kind == CAUSAL, scale)
+            dq += dq_p.to(acc_dtype)
+            acc[0] += dk_p.to(acc_dtype)
+            acc[1] += dv_p.to(acc_dtype)
+        # this shard's accumulators move on with it (the last hop brings them home)
+        if world > 1:
+            reqs += dist.batch_isend_irecv([dist.P2POp(dist.isend, acc, nxt_rank, group),
+                                            dist.P2POp(dist.irecv, acc_in, prv_rank, group)])
+        for r in reqs:
+            r.wait()
+        if world > 1:
+            acc, acc_in = acc_in, acc
+        if step + 1 < world:
+            cur, nxt = nxt, cur
+    return dq, acc[0], acc[1]

@@ -82,3 +82,62 @@ def test_ring_equals_attention_over_the_whole_sequence(tmp_path, world, causal):
                                    rtol=1e-12, atol=1e-13)
         np.testing.assert_allclose(np.load(tmp_path / f"lse{r}.npy"), lse_ref[:, :, r * n:(r + 1) * n],
                                    rtol=1e-12, atol=1e-13)
+
+
+def _partial_bwd(q, k, v, o, lse, do, causal, scale):
+    """One shard pair's gradient contribution in fp64, with the rows' global O and LSE:
+    P = exp(scale q k^T - lse), D = rowsum(dO * O), dS = P (dO v^T - D)."""
+    G = q.shape[1] // k.shape[1]
+    kk, vv = k.repeat_interleave(G, dim=1), v.repeat_interleave(G, dim=1)
+    s = scale * q @ kk.transpose(-1, -2)
+    if causal:
+        n = q.shape[2]
+        s = s.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+    p = torch.exp(s - lse[..., None])
+    ds = p * (do @ vv.transpose(-1, -2) - (do * o).sum(-1, keepdim=True))
+    dq = scale * ds @ kk
+    B, Hkv, n, d = k.shape
+    dk = (scale * ds.transpose(-1, -2) @ q).reshape(B, Hkv, G, n, d).sum(2)
+    dv = (p.transpose(-1, -2) @ do).reshape(B, Hkv, G, n, d).sum(2)
+    return dq, dk, dv
+
+
+def _rank_bwd(rank, world, port, causal, shape, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, Hq, Hkv, N, d = shape
+        g = torch.Generator().manual_seed(4321)            # the same full problem on every rank
+        q, k, v = (torch.randn(B, h, N, d, generator=g, dtype=torch.float64) for h in (Hq, Hkv, Hkv))
+        do = torch.randn(B, Hq, N, d, generator=g, dtype=torch.float64)
+        n = N // world
+        sl = slice(rank * n, (rank + 1) * n)
+        shard = lambda t: t[:, :, sl].contiguous()
+        o, lse = ring.ring_attention_fwd(shard(q), shard(k), shard(v), causal=causal, scale=0.4,
+                                         partial=_partial, merge=_merge, acc_dtype=torch.float64)
+        dq, dk, dv = ring.ring_attention_bwd(shard(q), shard(k), shard(v), o, lse, shard(do), causal=causal,
+                                             scale=0.4, partial=_partial_bwd, acc_dtype=torch.float64)
+        for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+            np.save(os.path.join(out_dir, f"{name}{rank}.npy"), t.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_backward_equals_gradients_over_the_whole_sequence(tmp_path, world, causal):
+    """Every rank's dQ and the dK, dV its shards collect on their way round the ring
+    equal the oracle's gradients over the whole sequence (GQA, group of 2)."""
+    shape = (2, 4, 2, 8 * world, 5)
+    mp.start_processes(_rank_bwd, args=(world, _free_port(), causal, shape, str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    B, Hq, Hkv, N, d = shape
+    g = torch.Generator().manual_seed(4321)
+    q, k, v = (torch.randn(B, h, N, d, generator=g, dtype=torch.float64).numpy() for h in (Hq, Hkv, Hkv))
+    do = torch.randn(B, Hq, N, d, generator=g, dtype=torch.float64).numpy()
+    grads = dict(zip(("dq", "dk", "dv"), ref.ref_bwd(q, k, v, do, 0.4, causal)))
+    n = N // world
+    for r in range(world):
+        for name, full in grads.items():
+            np.testing.assert_allclose(np.load(tmp_path / f"{name}{r}.npy"), full[:, :, r * n:(r + 1) * n],
+                                       rtol=1e-10, atol=1e-11, err_msg=f"{name} rank {r}")
