@@ -22,6 +22,13 @@ GPU's memory; the transfer of the next shard overlaps the compute of the current
 one.  Every rank takes the same exchange steps in the same order, skipped compute
 included.
 
+Layouts.  ``contiguous``: rank r holds chunk r of W equal chunks, as above; under
+causal masking rank r then does r + 1 of the W shard pairs' work.  ``zigzag``: the
+sequence is cut into 2W chunks and rank r holds chunks r and 2W - 1 - r (in that
+order, as one local tensor); every rank then does the same causal work, 2W - 1 full
+chunk pairs and 2 diagonal ones.  Chunk pairs are computed one by one: full where
+the key chunk precedes the query chunk, causal on the diagonal, skipped after it.
+
 Backward (recompute, as on one GPU): the shards travel the same ring, each with
 fp32 accumulators for its dK and dV.  At step s rank r computes the gradient
 contributions of its query shard against the shard it holds -- with the global LSE
@@ -39,11 +46,12 @@ from __future__ import annotations
 import torch
 
 FULL, CAUSAL, SKIP = "full", "causal", "skip"
+LAYOUTS = ("contiguous", "zigzag")
 
 
 def ring_schedule(rank: int, world: int, causal: bool):
-    """[(step, source rank, kind)] for one rank: the shard it holds at each step and
-    what it computes against it."""
+    """[(step, source rank, kind)] for one rank under the contiguous layout: the shard
+    it holds at each step and what it computes against it."""
     out = []
     for s in range(world):
         src = (rank - s) % world
@@ -59,6 +67,44 @@ def ring_schedule(rank: int, world: int, causal: bool):
     return out
 
 
+def shard_chunks(rank: int, world: int, layout: str = "contiguous"):
+    """Global chunk indices held by ``rank``, in local order (chunks of N / W positions
+    for ``contiguous``, of N / (2W) for ``zigzag``)."""
+    if layout == "contiguous":
+        return [rank]
+    if layout == "zigzag":
+        return [rank, 2 * world - 1 - rank]
+    raise ValueError(f"layout must be one of {LAYOUTS}")
+
+
+def chunk_kind(a: int, b: int, causal: bool):
+    """What query chunk a computes against key chunk b."""
+    if not causal or b < a:
+        return FULL
+    return CAUSAL if a == b else SKIP
+
+
+def shard_sequence(x, rank: int, world: int, layout: str = "contiguous", dim: int = 2):
+    """This rank's local tensor of a full-sequence tensor ``x`` (sequence along ``dim``)."""
+    chunks = shard_chunks(rank, world, layout)
+    nchunks = world * len(chunks)
+    c = x.shape[dim] // nchunks
+    if c * nchunks != x.shape[dim]:
+        raise ValueError(f"sequence length {x.shape[dim]} is not a multiple of {nchunks} chunks")
+    return torch.cat([x.narrow(dim, a * c, c) for a in chunks], dim=dim).contiguous()
+
+
+def _chunked(x, m):
+    """[B, H, m*c, d] -> [m, B, H, c, d] (each chunk contiguous)."""
+    B, H, n, d = x.shape
+    return x.reshape(B, H, m, n // m, d).permute(2, 0, 1, 3, 4).contiguous()
+
+
+def _unchunked(x):
+    """[m, B, H, c, ...] -> [B, H, m*c, ...]."""
+    return torch.cat(list(x.unbind(0)), dim=2)
+
+
 def _cuda_partial(q, k, v, causal, scale):
     from . import binding
     return binding.attn_fwd(q, k, v, scale=scale, causal=causal)
@@ -69,13 +115,21 @@ def _cuda_merge(o_acc, lse_acc, o_part, lse_part):
     binding.attn_merge(o_acc, lse_acc, o_part, lse_part)
 
 
+def _ring_peers(group, rank, world):
+    import torch.distributed as dist
+    if group is None:
+        return (rank + 1) % world, (rank - 1) % world
+    return dist.get_global_rank(group, (rank + 1) % world), dist.get_global_rank(group, (rank - 1) % world)
+
+
 def ring_attention_fwd(q, k, v, *, causal: bool, group=None, scale=None, partial=None, merge=None,
-                       acc_dtype=torch.float32):
+                       acc_dtype=torch.float32, layout: str = "contiguous"):
     """Attention of this rank's query shard against the whole sequence.
 
-    q: [B, Hq, n, d]; k, v: [B, Hkv, n, d] -- this rank's shard (all ranks the same n).
+    q: [B, Hq, n, d]; k, v: [B, Hkv, n, d] -- this rank's shard (all ranks the same n;
+    under ``zigzag`` the rank's two chunks, in order, see ``shard_sequence``).
     Returns (o, lse): o [B, Hq, n, d] and lse [B, Hq, n] (natural log) in ``acc_dtype``
-    (fp32 by default: merged in fp32, cast as needed).
+    (fp32 by default: merged in fp32, cast as needed), rows in the shard's order.
     ``partial(q, k, v, causal, scale) -> (o, lse)`` and ``merge(o_acc, lse_acc, o_part,
     lse_part)`` (in place) default to the CUDA library.
     """
@@ -87,26 +141,32 @@ def ring_attention_fwd(q, k, v, *, causal: bool, group=None, scale=None, partial
     merge = merge or _cuda_merge
     if scale is None:
         scale = q.shape[-1] ** -0.5
+    mine = shard_chunks(rank, world, layout)
+    m = len(mine)
     B, Hq, n, d = q.shape
-    o_acc = torch.zeros((B, Hq, n, d), dtype=acc_dtype, device=q.device)
-    lse_acc = torch.full((B, Hq, n), float("-inf"), dtype=acc_dtype, device=q.device)
-    cur = torch.stack((k, v)).contiguous()          # [2, B, Hkv, n, d]: one message per step
+    qc = _chunked(q, m)                                       # [m, B, Hq, c, d]
+    o_acc = torch.zeros((m, B, Hq, n // m, d), dtype=acc_dtype, device=q.device)
+    lse_acc = torch.full((m, B, Hq, n // m), float("-inf"), dtype=acc_dtype, device=q.device)
+    cur = torch.stack((_chunked(k, m), _chunked(v, m))).contiguous()   # [2, m, B, Hkv, c, d]: one message
     nxt = torch.empty_like(cur)
-    nxt_rank = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
-    prv_rank = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
-    for step, src, kind in ring_schedule(rank, world, causal):
+    nxt_rank, prv_rank = _ring_peers(group, rank, world)
+    for step in range(world):
+        src = (rank - step) % world
         reqs = []
         if step + 1 < world:                        # post the exchange for the next step first
             ops = [dist.P2POp(dist.isend, cur, nxt_rank, group), dist.P2POp(dist.irecv, nxt, prv_rank, group)]
             reqs = dist.batch_isend_irecv(ops)
-        if kind != SKIP:
-            o_p, lse_p = partial(q, cur[0], cur[1], kind == CAUSAL, scale)
-            merge(o_acc, lse_acc, o_p, lse_p)
+        for i, a in enumerate(mine):
+            for j, b in enumerate(shard_chunks(src, world, layout)):
+                kind = chunk_kind(a, b, causal)
+                if kind != SKIP:
+                    o_p, lse_p = partial(qc[i], cur[0, j], cur[1, j], kind == CAUSAL, scale)
+                    merge(o_acc[i], lse_acc[i], o_p, lse_p)
         for r in reqs:
             r.wait()
         if step + 1 < world:
             cur, nxt = nxt, cur
-    return o_acc, lse_acc
+    return _unchunked(o_acc), _unchunked(lse_acc[..., None])[..., 0]
 
 
 def _cuda_partial_bwd(q, k, v, o, lse, do, causal, scale):
@@ -115,14 +175,14 @@ def _cuda_partial_bwd(q, k, v, o, lse, do, causal, scale):
 
 
 def ring_attention_bwd(q, k, v, o, lse, do, *, causal: bool, group=None, scale=None, partial=None,
-                       acc_dtype=torch.float32):
+                       acc_dtype=torch.float32, layout: str = "contiguous"):
     """Gradients of this rank's shards, for attention over the whole ring's sequence.
 
     q, o, do: [B, Hq, n, d]; k, v: [B, Hkv, n, d] -- this rank's shard; lse: [B, Hq, n]
     (natural log), o and lse being this rank's rows of the forward over the whole
-    sequence (``ring_attention_fwd``; o in the dtype ``partial`` takes).
-    Returns (dq, dk, dv) for this rank's shards in ``acc_dtype``.
-    ``partial(q, k, v, o, lse, do, causal, scale) -> (dq, dk, dv)`` gives one shard
+    sequence (``ring_attention_fwd`` with the same layout; o in the dtype ``partial``
+    takes).  Returns (dq, dk, dv) for this rank's shards in ``acc_dtype``.
+    ``partial(q, k, v, o, lse, do, causal, scale) -> (dq, dk, dv)`` gives one chunk
     pair's contribution; it defaults to the CUDA library's ``attn_bwd``.
     """
     import torch.distributed as dist
@@ -132,23 +192,32 @@ def ring_attention_bwd(q, k, v, o, lse, do, *, causal: bool, group=None, scale=N
     partial = partial or _cuda_partial_bwd
     if scale is None:
         scale = q.shape[-1] ** -0.5
-    dq = torch.zeros(q.shape, dtype=acc_dtype, device=q.device)
-    cur = torch.stack((k, v)).contiguous()                          # the shard held at this step
+    mine = shard_chunks(rank, world, layout)
+    m = len(mine)
+    qc, oc, doc = _chunked(q, m), _chunked(o, m), _chunked(do, m)
+    lsec = _chunked(lse[..., None], m)[..., 0]
+    dq = torch.zeros(qc.shape, dtype=acc_dtype, device=q.device)
+    cur = torch.stack((_chunked(k, m), _chunked(v, m))).contiguous()   # the shard held at this step
     nxt = torch.empty_like(cur)
-    acc = torch.zeros((2,) + tuple(k.shape), dtype=acc_dtype, device=q.device)   # its dK, dV so far
+    acc = torch.zeros(cur.shape, dtype=acc_dtype, device=q.device)      # its dK, dV so far
     acc_in = torch.empty_like(acc)
-    nxt_rank = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
-    prv_rank = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
-    for step, src, kind in ring_schedule(rank, world, causal):
+    nxt_rank, prv_rank = _ring_peers(group, rank, world)
+    for step in range(world):
+        src = (rank - step) % world
         reqs = []
         if step + 1 < world:                        # the next shard is in flight during the compute
             reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur, nxt_rank, group),
                                            dist.P2POp(dist.irecv, nxt, prv_rank, group)])
-        if kind != SKIP:
-            dq_p, dk_p, dv_p = partial(q, cur[0], cur[1], o, lse, do, kind == CAUSAL, scale)
-            dq += dq_p.to(acc_dtype)
-            acc[0] += dk_p.to(acc_dtype)
-            acc[1] += dv_p.to(acc_dtype)
+        for i, a in enumerate(mine):
+            for j, b in enumerate(shard_chunks(src, world, layout)):
+                kind = chunk_kind(a, b, causal)
+                if kind == SKIP:
+                    continue
+                dq_p, dk_p, dv_p = partial(qc[i], cur[0, j], cur[1, j], oc[i], lsec[i], doc[i], kind == CAUSAL,
+                                           scale)
+                dq[i] += dq_p.to(acc_dtype)
+                acc[0, j] += dk_p.to(acc_dtype)
+                acc[1, j] += dv_p.to(acc_dtype)
         # this shard's accumulators move on with it (the last hop brings them home)
         if world > 1:
             reqs += dist.batch_isend_irecv([dist.P2POp(dist.isend, acc, nxt_rank, group),
@@ -159,4 +228,4 @@ def ring_attention_bwd(q, k, v, o, lse, do, *, causal: bool, group=None, scale=N
             acc, acc_in = acc_in, acc
         if step + 1 < world:
             cur, nxt = nxt, cur
-    return dq, acc[0], acc[1]
+    return _unchunked(dq), _unchunked(acc[0]), _unchunked(acc[1])

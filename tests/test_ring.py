@@ -48,40 +48,54 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, causal, shape, out_dir):
+def _rank_main(rank, world, port, causal, shape, out_dir, layout="contiguous"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         B, Hq, Hkv, N, d = shape
         g = torch.Generator().manual_seed(1234)            # the same full problem on every rank
         q, k, v = (torch.randn(B, h, N, d, generator=g, dtype=torch.float64) for h in (Hq, Hkv, Hkv))
-        n = N // world
-        sl = slice(rank * n, (rank + 1) * n)
-        o, lse = ring.ring_attention_fwd(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
-                                         v[:, :, sl].contiguous(), causal=causal, scale=0.4,
-                                         partial=_partial, merge=_merge, acc_dtype=torch.float64)
+        shard = lambda t: ring.shard_sequence(t, rank, world, layout)
+        o, lse = ring.ring_attention_fwd(shard(q), shard(k), shard(v), causal=causal, scale=0.4,
+                                         partial=_partial, merge=_merge, acc_dtype=torch.float64, layout=layout)
         np.save(os.path.join(out_dir, f"o{rank}.npy"), o.numpy())
         np.save(os.path.join(out_dir, f"lse{rank}.npy"), lse.numpy())
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world,layout", [(2, "contiguous"), (3, "contiguous"), (2, "zigzag"), (3, "zigzag")])
 @pytest.mark.parametrize("causal", [False, True])
-def test_ring_equals_attention_over_the_whole_sequence(tmp_path, world, causal):
+def test_ring_equals_attention_over_the_whole_sequence(tmp_path, world, layout, causal):
     shape = (2, 4, 2, 12 * world, 5)
-    mp.start_processes(_rank_main, args=(world, _free_port(), causal, shape, str(tmp_path)), nprocs=world,
+    mp.start_processes(_rank_main, args=(world, _free_port(), causal, shape, str(tmp_path), layout), nprocs=world,
                        join=True, start_method="spawn")
     B, Hq, Hkv, N, d = shape
     g = torch.Generator().manual_seed(1234)
     q, k, v = (torch.randn(B, h, N, d, generator=g, dtype=torch.float64).numpy() for h in (Hq, Hkv, Hkv))
     o_ref, lse_ref = ref.ref_fwd(q, k, v, 0.4, causal)
-    n = N // world
     for r in range(world):
-        np.testing.assert_allclose(np.load(tmp_path / f"o{r}.npy"), o_ref[:, :, r * n:(r + 1) * n],
-                                   rtol=1e-12, atol=1e-13)
-        np.testing.assert_allclose(np.load(tmp_path / f"lse{r}.npy"), lse_ref[:, :, r * n:(r + 1) * n],
-                                   rtol=1e-12, atol=1e-13)
+        mine = lambda a, dim: ring.shard_sequence(torch.from_numpy(a), r, world, layout, dim).numpy()
+        np.testing.assert_allclose(np.load(tmp_path / f"o{r}.npy"), mine(o_ref, 2), rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(np.load(tmp_path / f"lse{r}.npy"), mine(lse_ref, 2), rtol=1e-12, atol=1e-13)
+
+
+def test_shards_partition_the_sequence_and_zigzag_balances_causal_work():
+    for world in (1, 2, 3, 4, 8):
+        for layout in ring.LAYOUTS:
+            held = sorted(a for r in range(world) for a in ring.shard_chunks(r, world, layout))
+            assert held == list(range(world * len(ring.shard_chunks(0, world, layout))))
+            x = torch.arange(2 * world * 3).reshape(1, 1, -1, 1)
+            got = torch.cat([ring.shard_sequence(x, r, world, layout) for r in range(world)], dim=2)
+            assert sorted(got.flatten().tolist()) == x.flatten().tolist()
+        # causal work per rank, counting a diagonal chunk pair as half a full one
+        work = lambda r, layout: sum(
+            {ring.FULL: 1.0, ring.CAUSAL: 0.5, ring.SKIP: 0.0}[ring.chunk_kind(a, b, True)]
+            for a in ring.shard_chunks(r, world, layout)
+            for s in range(world) for b in ring.shard_chunks(s, world, layout))
+        assert len({work(r, "zigzag") for r in range(world)}) == 1
+        if world > 1:
+            assert work(world - 1, "contiguous") > work(0, "contiguous")
 
 
 def _partial_bwd(q, k, v, o, lse, do, causal, scale):
@@ -102,7 +116,7 @@ def _partial_bwd(q, k, v, o, lse, do, causal, scale):
     return dq, dk, dv
 
 
-def _rank_bwd(rank, world, port, causal, shape, out_dir):
+def _rank_bwd(rank, world, port, causal, shape, out_dir, layout="contiguous"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -110,34 +124,34 @@ def _rank_bwd(rank, world, port, causal, shape, out_dir):
         g = torch.Generator().manual_seed(4321)            # the same full problem on every rank
         q, k, v = (torch.randn(B, h, N, d, generator=g, dtype=torch.float64) for h in (Hq, Hkv, Hkv))
         do = torch.randn(B, Hq, N, d, generator=g, dtype=torch.float64)
-        n = N // world
-        sl = slice(rank * n, (rank + 1) * n)
-        shard = lambda t: t[:, :, sl].contiguous()
+        shard = lambda t: ring.shard_sequence(t, rank, world, layout)
         o, lse = ring.ring_attention_fwd(shard(q), shard(k), shard(v), causal=causal, scale=0.4,
-                                         partial=_partial, merge=_merge, acc_dtype=torch.float64)
+                                         partial=_partial, merge=_merge, acc_dtype=torch.float64, layout=layout)
         dq, dk, dv = ring.ring_attention_bwd(shard(q), shard(k), shard(v), o, lse, shard(do), causal=causal,
-                                             scale=0.4, partial=_partial_bwd, acc_dtype=torch.float64)
+                                             scale=0.4, partial=_partial_bwd, acc_dtype=torch.float64,
+                                             layout=layout)
         for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
             np.save(os.path.join(out_dir, f"{name}{rank}.npy"), t.numpy())
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3, 4])
+@pytest.mark.parametrize("world,layout", [(2, "contiguous"), (3, "contiguous"), (4, "contiguous"),
+                                          (2, "zigzag"), (3, "zigzag")])
 @pytest.mark.parametrize("causal", [False, True])
-def test_ring_backward_equals_gradients_over_the_whole_sequence(tmp_path, world, causal):
+def test_ring_backward_equals_gradients_over_the_whole_sequence(tmp_path, world, layout, causal):
     """Every rank's dQ and the dK, dV its shards collect on their way round the ring
     equal the oracle's gradients over the whole sequence (GQA, group of 2)."""
     shape = (2, 4, 2, 8 * world, 5)
-    mp.start_processes(_rank_bwd, args=(world, _free_port(), causal, shape, str(tmp_path)), nprocs=world,
+    mp.start_processes(_rank_bwd, args=(world, _free_port(), causal, shape, str(tmp_path), layout), nprocs=world,
                        join=True, start_method="spawn")
     B, Hq, Hkv, N, d = shape
     g = torch.Generator().manual_seed(4321)
     q, k, v = (torch.randn(B, h, N, d, generator=g, dtype=torch.float64).numpy() for h in (Hq, Hkv, Hkv))
     do = torch.randn(B, Hq, N, d, generator=g, dtype=torch.float64).numpy()
     grads = dict(zip(("dq", "dk", "dv"), ref.ref_bwd(q, k, v, do, 0.4, causal)))
-    n = N // world
     for r in range(world):
         for name, full in grads.items():
-            np.testing.assert_allclose(np.load(tmp_path / f"{name}{r}.npy"), full[:, :, r * n:(r + 1) * n],
+            mine = ring.shard_sequence(torch.from_numpy(full), r, world, layout).numpy()
+            np.testing.assert_allclose(np.load(tmp_path / f"{name}{r}.npy"), mine,
                                        rtol=1e-10, atol=1e-11, err_msg=f"{name} rank {r}")

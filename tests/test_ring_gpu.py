@@ -71,42 +71,52 @@ def test_merge_into_an_empty_accumulator_copies_the_partial(attn):
     assert torch.allclose(lse_acc, lse_p, rtol=0, atol=1e-6)
 
 
-@pytest.mark.parametrize("world,causal,d", [(2, True, 128), (4, True, 128), (3, False, 64)])
-def test_ring_backward_decomposition_matches_oracle(attn, world, causal, d):
-    B, Hq, Hkv, n = 1, 4, 2, 320
-    N = n * world
+@pytest.mark.parametrize("world,causal,d,layout", [(2, True, 128, "contiguous"), (4, True, 128, "contiguous"),
+                                                   (3, False, 64, "contiguous"), (2, True, 128, "zigzag"),
+                                                   (3, True, 64, "zigzag")])
+def test_ring_backward_decomposition_matches_oracle(attn, world, causal, d, layout):
+    """Forward and backward over the ring, chunk pair by chunk pair as ``ring.py`` takes
+    them (both layouts), against the oracle over the whole sequence."""
+    B, Hq, Hkv, c = 1, 4, 2, 192                          # c: rows per chunk
+    m = len(ring.shard_chunks(0, world, layout))
+    N = c * m * world
     x = make_inputs(B, Hq, Hkv, N, d, seed=200 + world + d, with_grad=True)
     q, k, v, do = (x[t].cuda() for t in ("q", "k", "v", "do"))
-    sl = lambda t, s: t[:, :, s * n:(s + 1) * n].contiguous()
+    ch = lambda t, a: t[:, :, a * c:(a + 1) * c].contiguous()      # global chunk a
     dq_ref, dk_ref, dv_ref = ref.ref_bwd(*(to_f64(x[t]) for t in ("q", "k", "v", "do")), d ** -0.5, causal)
-    # the forward over the ring, rank by rank: each rank's rows of O (bf16) and LSE
-    o_rows, lse_rows = [], []
-    for r in range(world):
-        o_acc = torch.zeros((B, Hq, n, d), dtype=torch.float32, device="cuda")
-        lse_acc = torch.full((B, Hq, n), float("-inf"), dtype=torch.float32, device="cuda")
-        out = torch.empty((B, Hq, n, d), dtype=torch.bfloat16, device="cuda")
-        for step, src, kind in ring.ring_schedule(r, world, causal):
+    nchunks = m * world
+    # forward: every query chunk's O (bf16) and LSE, merged over the key chunks
+    o_ch, lse_ch = {}, {}
+    for a in range(nchunks):
+        o_acc = torch.zeros((B, Hq, c, d), dtype=torch.float32, device="cuda")
+        lse_acc = torch.full((B, Hq, c), float("-inf"), dtype=torch.float32, device="cuda")
+        out = torch.empty((B, Hq, c, d), dtype=torch.bfloat16, device="cuda")
+        for b in range(nchunks):
+            kind = ring.chunk_kind(a, b, causal)
             if kind != ring.SKIP:
-                o_p, lse_p = attn.attn_fwd(sl(q, r), sl(k, src), sl(v, src), causal=(kind == ring.CAUSAL))
+                o_p, lse_p = attn.attn_fwd(ch(q, a), ch(k, b), ch(v, b), causal=(kind == ring.CAUSAL))
                 attn.attn_merge(o_acc, lse_acc, o_p, lse_p, out)
-        o_rows.append(out)
-        lse_rows.append(lse_acc)
-    # the backward over the ring: dQ per rank, dK and dV per shard, fp32 sums
-    dq = [torch.zeros((B, Hq, n, d), device="cuda") for _ in range(world)]
-    dkv = [torch.zeros((2, B, Hkv, n, d), device="cuda") for _ in range(world)]
+        o_ch[a], lse_ch[a] = out, lse_acc
+    # backward in ring order: rank r's chunks against the shard held at each step
+    dq = {a: torch.zeros((B, Hq, c, d), device="cuda") for a in range(nchunks)}
+    dkv = {a: torch.zeros((2, B, Hkv, c, d), device="cuda") for a in range(nchunks)}
     for r in range(world):
-        for step, src, kind in ring.ring_schedule(r, world, causal):
-            if kind == ring.SKIP:
-                continue
-            g = attn.attn_bwd(sl(q, r), sl(k, src), sl(v, src), o_rows[r], lse_rows[r], sl(do, r),
-                              causal=(kind == ring.CAUSAL))
-            dq[r] += g[0].float()
-            dkv[src][0] += g[1].float()
-            dkv[src][1] += g[2].float()
+        for step in range(world):
+            src = (r - step) % world
+            for a in ring.shard_chunks(r, world, layout):
+                for b in ring.shard_chunks(src, world, layout):
+                    kind = ring.chunk_kind(a, b, causal)
+                    if kind == ring.SKIP:
+                        continue
+                    g = attn.attn_bwd(ch(q, a), ch(k, b), ch(v, b), o_ch[a], lse_ch[a], ch(do, a),
+                                      causal=(kind == ring.CAUSAL))
+                    dq[a] += g[0].float()
+                    dkv[b][0] += g[1].float()
+                    dkv[b][1] += g[2].float()
     torch.cuda.synchronize()
     assert attn.attn_get_device_status() == 0
-    for r in range(world):
-        rows = slice(r * n, (r + 1) * n)
-        check_grad(f64(dq[r]), dq_ref[:, :, rows], f"ring bwd W={world} rank {r} dQ")
-        check_grad(f64(dkv[r][0]), dk_ref[:, :, rows], f"ring bwd W={world} shard {r} dK")
-        check_grad(f64(dkv[r][1]), dv_ref[:, :, rows], f"ring bwd W={world} shard {r} dV")
+    for a in range(nchunks):
+        rows = slice(a * c, (a + 1) * c)
+        check_grad(f64(dq[a]), dq_ref[:, :, rows], f"ring bwd {layout} W={world} chunk {a} dQ")
+        check_grad(f64(dkv[a][0]), dk_ref[:, :, rows], f"ring bwd {layout} W={world} chunk {a} dK")
+        check_grad(f64(dkv[a][1]), dv_ref[:, :, rows], f"ring bwd {layout} W={world} chunk {a} dV")
