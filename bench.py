@@ -453,7 +453,8 @@ def run_fp8(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    for name in ("causal_b8_h16_n4096_d128", "long_causal_b1_h32_n32768_d128", "gqa_causal_b4_hq32_hkv8_n8192_d128"):
+    for name in ("causal_b8_h16_n4096_d128", "long_causal_b1_h32_n32768_d128", "gqa_causal_b4_hq32_hkv8_n8192_d128",
+                 "gpt2_medium_b64_h16_n1024_d64"):
         w = WORKLOADS[name]
         x8 = make_fp8_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, qk_std=w.qk_std, device=dev)
         x16 = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, qk_std=w.qk_std, vo_std=w.vo_std,

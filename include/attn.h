@@ -80,7 +80,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  * sums and the LSE use the unrounded P, as in attn_fwd.  O is bf16, lse fp32
  * (page "attention 的显存线性化" §五 names FP8 support for the later versions; the
  * pages give no recipe, so the per-tensor descales are this library's reading).
- * d must be 128 (ATTN_ERR_UNSUPPORTED otherwise); descales finite and > 0. */
+ * d is 64 or 128 (a 64-byte e4m3 row is zero-padded to the 128-byte swizzle row on
+ * chip; ATTN_ERR_UNSUPPORTED otherwise); descales finite and > 0. */
 int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                  int B, int Hq, int Hkv, int N, int d, float scale,
                  float q_descale, float k_descale, float v_descale, int causal, void* stream);

@@ -151,7 +151,7 @@ def attn_fwd(q, k, v, o=None, lse=None, *, scale=None, causal=False, stream=None
 def attn_fwd_fp8(q, k, v, o=None, lse=None, *, q_descale, k_descale, v_descale, scale=None, causal=False,
                  stream=None):
     """Forward with e4m3 Q, K, V (torch.float8_e4m3fn) and per-tensor descales; returns
-    (o bf16, lse fp32).  The attended values are q * q_descale etc.; d must be 128."""
+    (o bf16, lse fp32).  The attended values are q * q_descale etc.; d is 64 or 128."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n, torch.float8_e4m3fn)
     B, Hq, N, d = q.shape

@@ -418,7 +418,6 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
                  int d, float scale, float q_descale, float k_descale, float v_descale, int causal, void* stream) {
   int st = check_common(B, Hq, Hkv, N, d, scale, causal);
   if (st != ATTN_OK) return st;
-  if (d != 128) return ATTN_ERR_UNSUPPORTED;
   for (float x : {q_descale, k_descale, v_descale})
     if (!std::isfinite(x) || !(x > 0.f)) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale * q_descale * k_descale)) return ATTN_ERR_INVALID_ARG;
@@ -427,6 +426,9 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
     return ATTN_ERR_ALIGNMENT;
   DeviceInfo* di = nullptr;
   if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (d == 64)
+    return launch_fwd_pp<64, true>(q, k, v, o, lse, B, Hq, Hkv, N, scale, band_of_causal(N, causal),
+                                   static_cast<cudaStream_t>(stream), *di, q_descale * k_descale, v_descale);
   return launch_fwd_pp<128, true>(q, k, v, o, lse, B, Hq, Hkv, N, scale, band_of_causal(N, causal),
                                   static_cast<cudaStream_t>(stream), *di, q_descale * k_descale, v_descale);
 }

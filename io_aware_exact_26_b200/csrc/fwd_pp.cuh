@@ -40,27 +40,31 @@ namespace attn {
 
 // F8 = false: bf16 Q, K, V and P (kind::f16).  F8 = true: e4m3 Q, K, V and P
 // (kind::f8f6f4), each tile row of d bytes, with per-tensor descales folded into
-// the exponent scale (Q, K) and the output (V).
+// the exponent scale (Q, K) and the output (V).  An e4m3 row of d = 64 is 64 bytes:
+// its tiles are padded to the 128-byte swizzle row (DT = 128 columns), the TMA
+// filling columns 64-127 with zeros, so S = Q K^T is unchanged, O's padding columns
+// stay 0 and only the first d columns are written out.
 template <int D, bool F8 = false>
 struct PpCfg {
   static constexpr int ES = F8 ? 1 : 2;                 // bytes per element
-  static constexpr int kTile = 128 * D * ES;
+  static constexpr int DT = (F8 && D * ES < 128) ? 128 / ES : D;   // tile columns (padded)
+  static constexpr int kTile = 128 * DT * ES;
   static constexpr int kBox = 128 * 128;                // one TMA box: 128 rows x 128 bytes
-  static constexpr int NB = D * ES / 128;               // boxes per tile
-  static constexpr int KS = D * ES / 32;                // S = Q K^T: 32-byte K steps
+  static constexpr int NB = DT * ES / 128;              // boxes per tile
+  static constexpr int KS = DT * ES / 32;               // S = Q K^T: 32-byte K steps
   static constexpr int PVK = F8 ? 32 : 16;              // keys per P V instruction
   static_assert(NB >= 1, "a tile row must fill one 128-byte swizzle row");
   static constexpr int KST = 2;
   static constexpr int VST = 2;
   static constexpr int kThreads = 576;
   // Of every 8 score pairs, how many are exponentiated on the FMA pipe instead of
-  // MUFU (16 ex2 per SM per clock).  At d = 64 a tile's two products take 768
-  // tensor-core cycles against 1024 MUFU cycles for its exponentials, so MUFU alone
-  // bounds the step and moving 2 pairs in 8 to the FMA pipe measured +8% to +21%
-  // (N = 1024 to 4096); at d = 128 the two are even and the share measured no gain.
-  static constexpr int kFmaPairs = (D == 64 && !F8) ? 2 : 0;
+  // MUFU (16 ex2 per SM per clock).  At d = 64 a tile's two products take 512
+  // tensor-core cycles (bf16; fewer with e4m3) against 1024 MUFU cycles for its
+  // exponentials, and moving 2 pairs in 8 to the FMA pipe measured +8% to +21%
+  // (N = 1024 to 4096); at d = 128 the share measured no gain.
+  static constexpr int kFmaPairs = D == 64 ? 2 : 0;
   static constexpr int kTmemCols = 512;
-  static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
+  static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + DT;
   // Q buffers per team: two at d = 64, so the next unit's Q loads while the current
   // unit still reads its own (short units, e.g. N = 1024, would wait for it); one
   // at d = 128, where shared memory has no room and units are longer.
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(576, 1)
     // (the P it overwrites); meanwhile the tensor cores run the other team's work.
     const bool leader = elect_one();
     constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
-    constexpr uint32_t idO = F8 ? idesc_e4m3_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
+    constexpr uint32_t idO = F8 ? idesc_e4m3_f32(128, C::DT, false, true) : idesc_bf16_f32(128, D, false, true);
     constexpr uint32_t hi = sdesc_hi_sw128(1024);
     const uint32_t q_lo0 = sdesc_lo(smem_u32(sQ), 16);
     const uint32_t k_lo0 = sdesc_lo(smem_u32(sK), 16);
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(576, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const uint32_t s_base = lane_base + (x ? C::kS1 : C::kS0) + grp * 64;
-    constexpr int OH = D / 2;
+    constexpr int OH = C::DT / 2;                               // O columns per group (padded)
     const uint32_t o_base = lane_base + (x ? C::kO1 : C::kO0) + grp * OH;
     const float c = p.c;
     const uint64_t c2 = f2pack(c, c);
@@ -558,6 +562,7 @@ __global__ void __launch_bounds__(576, 1)
       const float inv_l = p.oscale / l;      // oscale: V's descale (1 for bf16)
       const bool live = qrow < p.N && in_range(bh, static_cast<long long>(p.B) * p.Hq);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D + grp * OH;
+      const bool cols = grp * OH < D;       // padded tiles: the second group's columns are padding
       // all of this group's O columns in one round of TMEM loads (no softmax registers are
       // live here), then convert and store
       uint32_t o[OH / 16][16];
@@ -571,7 +576,7 @@ __global__ void __launch_bounds__(576, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           pk[k] = pack_bf16x2(__uint_as_float(o[q4][2 * k]) * inv_l, __uint_as_float(o[q4][2 * k + 1]) * inv_l);
-        if (live) {
+        if (live && cols) {
           uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 16);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);

@@ -169,7 +169,7 @@ def test_merge_validates_before_any_launch(L):
 def test_fp8_forward_validates_before_any_launch(L):
     def f8(q=FAKE, d=128, dq=0.01, dk=0.01, dv=0.01, scale=0.088, N=256):
         return L.attn_fwd_fp8(q, FAKE, FAKE, FAKE, FAKE, 1, 2, 1, N, d, scale, dq, dk, dv, 1, None)
-    assert f8(d=64) == -2                 # e4m3 tiles need 128-byte rows
+    assert f8(d=32) == -2                 # head dims 64 and 128 only
     assert f8(dq=0.0) == -1
     assert f8(dk=-1.0) == -1
     assert f8(dv=float("inf")) == -1

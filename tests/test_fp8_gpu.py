@@ -52,20 +52,24 @@ def fp8_bound(qf, kf, vf, scale, causal, o_ref):
 
 
 CASES = [
-    # B, Hq, Hkv, N, causal
-    (1, 2, 2, 256, False),
-    (1, 4, 2, 1000, True),
-    (2, 2, 2, 1024, False),
-    (1, 2, 1, 130, True),
-    (1, 1, 1, 17, False),
-    (1, 8, 2, 512, True),
+    # B, Hq, Hkv, N, causal, d
+    (1, 2, 2, 256, False, 128),
+    (1, 4, 2, 1000, True, 128),
+    (2, 2, 2, 1024, False, 128),
+    (1, 2, 1, 130, True, 128),
+    (1, 1, 1, 17, False, 128),
+    (1, 8, 2, 512, True, 128),
+    # d = 64: 64-byte e4m3 rows, zero-padded to the 128-byte swizzle row on chip
+    (1, 2, 2, 256, False, 64),
+    (1, 4, 2, 1000, True, 64),
+    (2, 2, 1, 1024, False, 64),
+    (1, 1, 1, 17, True, 64),
 ]
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,N,causal", CASES)
-def test_fp8_forward_matches_oracle_within_e4m3_rounding_of_p(attn, B, Hq, Hkv, N, causal):
-    d = 128
-    x = make_fp8_inputs(B, Hq, Hkv, N, d, seed=N + Hq + causal)
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,d", CASES)
+def test_fp8_forward_matches_oracle_within_e4m3_rounding_of_p(attn, B, Hq, Hkv, N, causal, d):
+    x = make_fp8_inputs(B, Hq, Hkv, N, d, seed=N + Hq + causal + d)
     ds = {n: x[n + "_descale"] for n in ("q", "k", "v")}
     o, lse = attn.attn_fwd_fp8(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), q_descale=ds["q"], k_descale=ds["k"],
                                v_descale=ds["v"], causal=causal)
@@ -73,7 +77,7 @@ def test_fp8_forward_matches_oracle_within_e4m3_rounding_of_p(attn, B, Hq, Hkv, 
     assert attn.attn_get_device_status() == 0
     q8, k8, v8 = (x[n].view(torch.uint8).numpy() for n in ("q", "k", "v"))
     o_ref, lse_ref = ref.ref_fwd_fp8(q8, k8, v8, ds["q"], ds["k"], ds["v"], d ** -0.5, causal)
-    tag = f"fp8 B{B} Hq{Hq} Hkv{Hkv} N{N} {'causal' if causal else 'full'}"
+    tag = f"fp8 B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} {'causal' if causal else 'full'}"
     check_lse(f64(lse), lse_ref, f"{tag} LSE")
     qf, kf, vf = (ref.decode_e4m3(a) * ds[n] for a, n in ((q8, "q"), (k8, "k"), (v8, "v")))
     bound = fp8_bound(qf, kf, vf, d ** -0.5, causal, o_ref)
@@ -85,6 +89,7 @@ def test_fp8_forward_matches_oracle_within_e4m3_rounding_of_p(attn, B, Hq, Hkv, 
 
 
 def test_fp8_forward_is_deterministic_and_rejects_other_head_sizes(attn):
+    """Two calls give the same bits at d = 128 and d = 64; d = 32 is refused."""
     x = make_fp8_inputs(1, 2, 2, 300, 128, seed=1)
     args = dict(q_descale=x["q_descale"], k_descale=x["k_descale"], v_descale=x["v_descale"], causal=True)
     q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
@@ -92,8 +97,14 @@ def test_fp8_forward_is_deterministic_and_rejects_other_head_sizes(attn):
     o2, l2 = attn.attn_fwd_fp8(q, k, v, **args)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
-    y = make_fp8_inputs(1, 1, 1, 128, 64, seed=2)
+    y = make_fp8_inputs(1, 2, 1, 300, 64, seed=2)
+    q6, k6, v6 = (y[n].cuda() for n in ("q", "k", "v"))
+    o3, l3 = attn.attn_fwd_fp8(q6, k6, v6, q_descale=1.0, k_descale=1.0, v_descale=1.0, causal=True)
+    o4, l4 = attn.attn_fwd_fp8(q6, k6, v6, q_descale=1.0, k_descale=1.0, v_descale=1.0, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o3, o4) and torch.equal(l3, l4)
+    z = make_fp8_inputs(1, 1, 1, 128, 32, seed=2)
     with pytest.raises(attn.AttnError):
-        attn.attn_fwd_fp8(y["q"].cuda(), y["k"].cuda(), y["v"].cuda(), q_descale=1.0, k_descale=1.0, v_descale=1.0)
+        attn.attn_fwd_fp8(z["q"].cuda(), z["k"].cuda(), z["v"].cuda(), q_descale=1.0, k_descale=1.0, v_descale=1.0)
     with pytest.raises(attn.AttnError):
         attn.attn_fwd_fp8(q, k, v, q_descale=0.0, k_descale=1.0, v_descale=1.0)
