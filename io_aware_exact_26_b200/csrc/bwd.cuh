@@ -9,7 +9,7 @@
 //   dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Kernels
-//   bwd_prep : one row per D/8 lanes: D_i and LSE in log2 units.
+//   bwd_prep : one row per D/8 lanes: D_i and LSE in log2 units, both stored negated.
 //   bwd_kv   : persistent; one work item = (b, kv-head, 128-key tile j).  K_j, V_j
 //              stay in shared memory while the item walks its G q-heads and the
 //              query tiles that see tile j; dK_j and dV_j accumulate in TMEM and are

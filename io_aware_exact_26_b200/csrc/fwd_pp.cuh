@@ -18,13 +18,14 @@
 // other team's S or PV, and the two teams' MUFU phases alternate.
 //   warps 0-7, 8-15  softmax teams; inside a team, group k = (warp % 8) / 4 owns
 //                    keys [64k, 64k+64) of each S tile and O columns
-//                    [k*D/2, (k+1)*D/2); thread = query row = TMEM lane.
+//                    [k*DT/2, (k+1)*DT/2); thread = query row = TMEM lane.
 //   warp 16          TMA producer: Q_A, Q_B (one buffer per team at d = 128, two
 //                    at d = 64), K and V rings (2 stages each), loaded as K(0) V(0)
 //                    K(1) V(1) ..., the order in which the MMA warp releases them
 //   warp 17          MMA issuer
 // TMEM: S_A at 0, S_B at 128 (P written over S as bf16: keys 0-63 in columns
-// 0-31, keys 64-127 in 64-95), O_A at 256, O_B at 256 + D.
+// 0-31, keys 64-127 in 64-95), O_A at 256, O_B at 256 + DT (DT = d, or 128 for
+// zero-padded e4m3 tiles at d = 64).
 // Per team the loop is S(j) -> softmax(j) -> PV(j) -> S(j+1), one S buffer per
 // tile with P written over it.  S(j+1) is issued right behind PV(j): MMAs issued
 // by one thread are performed in issue order, so PV(j) has read P(j) before
