@@ -677,6 +677,9 @@ def main():
     # training or serving loop would; the serial figure (copy in, compute, copy out, one step at a
     # time) is reported beside it.
     host = {n: x[n].cpu().pin_memory() for n in x}
+    # SHA-256 of each input's bytes as generated (this rank's replica), so a run's inputs can
+    # be checked against another run's
+    digests = {n: hashlib.sha256(host[n].view(torch.uint8).numpy()).hexdigest() for n in sorted(host)}
 
     def make_outs():
         out = {"o": torch.empty_like(q), "lse": torch.empty_like(lse)}
@@ -778,7 +781,9 @@ def main():
             "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "strong" if args.shard else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_dict(WORKLOADS[args.workload], world, shard=args.shard),
+            "config": dict(config_dict(WORKLOADS[args.workload], world, shard=args.shard),
+                           inputs={"generator": f"torch.Generator on {dev}, seed {rank_seed(w, rank)} (rank {rank})",
+                                   "sha256": digests}),
             "fwd": {"ms": round(fwd_avg, 4), "tflops": round(f_fwd / (fwd_avg * 1e-3) / 1e12, 1),
                     "frac_of_peak": round(f_fwd / (fwd_avg * 1e-3) / 1e12 / peak, 4)},
             "roofline": roofline,

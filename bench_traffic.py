@@ -48,6 +48,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+from attn_inputs import sweep_workloads  # noqa: E402
+
+# The benchmark workloads and the sequence-length sweep's points (B*N = 16384, Hq*d = 2048)
+ALL_WORKLOADS = {**bench.WORKLOADS, **{w.name: w for w in sweep_workloads()}}
 
 DRAM_METRICS = "dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum"
 # pipe utilisation read in the same one-kernel capture
@@ -154,7 +158,7 @@ def git_revision() -> str:
 
 def write_launches(workload: str, csv_text: str, profiles_dir: str, revision: str | None = None) -> str:
     agg = parse_launches(csv_text)
-    w = bench.WORKLOADS[workload]
+    w = ALL_WORKLOADS[workload]
     passes = "one attn_fwd and one attn_bwd (prep + dK/dV + dQ kernels)" if "bwd" in w.passes else "one attn_fwd"
     note = (f"Kernel sources: git revision {revision or git_revision()} (source fingerprints: forward "
             f"{bench.kernel_source_hash('fwd')}, backward {bench.kernel_source_hash('bwd')}). The bench step is "
@@ -198,7 +202,7 @@ def dram_entry(workload: str, div: int, csv_texts, revision: str | None = None, 
 
 def dram_table(workload: str, entry) -> str:
     from io_aware_exact_26_b200 import accounting as acc
-    w = bench.WORKLOADS[workload]
+    w = ALL_WORKLOADS[workload]
     alg = {"fwd": acc.min_bytes_fwd(w.B, w.Hq, w.Hkv, w.N, w.d), "bwd": acc.min_bytes_bwd(w.B, w.Hq, w.Hkv, w.N, w.d)}
     rw = reduced(w, entry["div"])
     out = [f"# DRAM traffic: {workload}", "",
@@ -253,12 +257,56 @@ def write_dram(workload: str, div: int, csv_texts, profiles_dir: str, revision: 
     return entry
 
 
+def write_sweep_dram(d: int, causal: bool, csv_dir: str, profiles_dir: str, revision: str | None = None):
+    """DRAM bytes of every sweep point at head size ``d`` (causal or not) from per-kernel
+    captures named ``dram_<workload>_<kernel>.csv`` in ``csv_dir`` (each point captured
+    whole, div 1).  The sweep holds B*N fixed, so the algorithmic bytes are the same at
+    every N: traffic that grew with N (re-reads, spilled score tiles) would show as a
+    rising ratio.  Writes profiles/dram_sweep_<causal|full>_d<d>.md; returns the rows."""
+    from io_aware_exact_26_b200 import accounting as acc
+    rows = []
+    for w in sweep_workloads():
+        if w.d != d or w.causal != causal:
+            continue
+        texts = []
+        for k in ("fwd_pp", "bwd_prep", "bwd_kv", "bwd_q"):
+            with open(os.path.join(csv_dir, f"dram_{w.name}_{k}.csv")) as f:
+                texts.append(f.read())
+        e = dram_entry(w.name, 1, texts, revision)
+        alg = {"fwd": acc.min_bytes_fwd(w.B, w.Hq, w.Hkv, w.N, w.d), "bwd": acc.min_bytes_bwd(w.B, w.Hq, w.Hkv, w.N, w.d)}
+        rows.append({"workload": w.name, "N": w.N, "B": w.B, "H": w.Hq,
+                     "fwd": e["fwd"]["bytes_per_launch"], "bwd": e["bwd"]["bytes_per_launch"],
+                     "alg_fwd": alg["fwd"], "alg_bwd": alg["bwd"], "revision": e["revision"]})
+    kind = "causal" if causal else "full"
+    name = f"dram_sweep_{kind}_d{d}"
+    w0 = rows[0]["workload"]
+    out = [f"# DRAM traffic over the sequence-length sweep: {kind}, d = {d}", "",
+           f"Each point of `bench.py --sweep` (B·N = 16384 tokens, Hq·d = 2048) captured whole, one launch per "
+           f"kernel, kernel sources of revision {rows[0]['revision']}. With B·N fixed the algorithmic bytes are the "
+           "same at every N (N = 32768 holds 32768 tokens, as B cannot go below 1), so the ratios to the "
+           "algorithmic bytes should stay flat: traffic that grew like N² would double from one row to the "
+           "next.", "", "Command per point and kernel (here the first point, dK/dV kernel):", "",
+           "```", dram_command(w0, 1, "bwd_kv").replace("dram_bwd_kv.csv", f"dram_{w0}_bwd_kv.csv"), "```", "",
+           "| N | B×H | fwd DRAM MB | fwd ÷ algorithmic | bwd DRAM MB | bwd ÷ algorithmic | bwd ÷ previous row |",
+           "|---|---|---|---|---|---|---|"]
+    prev = None
+    for r in rows:
+        step = "-" if prev is None else f"{r['bwd'] / prev:.2f}"
+        out.append(f"| {r['N']} | {r['B']}×{r['H']} | {r['fwd'] / 1e6:.1f} | {r['fwd'] / r['alg_fwd']:.2f} | "
+                   f"{r['bwd'] / 1e6:.1f} | {r['bwd'] / r['alg_bwd']:.2f} | {step} |")
+        prev = r["bwd"]
+    os.makedirs(profiles_dir, exist_ok=True)
+    with open(os.path.join(profiles_dir, name + ".md"), "w") as f:
+        f.write("\n".join(out) + "\n")
+    return rows
+
+
 def run_case(workload: str, div: int, reps: int):
     """The kernels of one bench step on the reduced case, ``reps`` times (for ncu -k/-s/-c)."""
     import torch
     import io_aware_exact_26_b200 as attn
     from attn_inputs import make_inputs
-    w = reduced(bench.WORKLOADS[workload], div)
+    w = reduced(ALL_WORKLOADS[workload], div)
     dev = torch.device("cuda", 0)
     x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, qk_std=w.qk_std, vo_std=w.vo_std,
                     boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=True)
@@ -278,19 +326,25 @@ def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     sub = ap.add_subparsers(dest="cmd", required=True)
     a = sub.add_parser("launches", help="launch table from a time-only ncu launch list")
-    a.add_argument("--workload", required=True, choices=sorted(bench.WORKLOADS))
+    a.add_argument("--workload", required=True, choices=sorted(ALL_WORKLOADS))
     a.add_argument("--revision", default=None)
     a.add_argument("--profiles", default=os.path.join(ROOT, "profiles"))
     a.add_argument("csv")
     b = sub.add_parser("dram", help="DRAM bytes per full-size launch from per-kernel captures")
-    b.add_argument("--workload", required=True, choices=sorted(bench.WORKLOADS))
+    b.add_argument("--workload", required=True, choices=sorted(ALL_WORKLOADS))
     b.add_argument("--div", type=int, required=True)
     b.add_argument("--revision", default=None)
     b.add_argument("--csrc", default=None, help="kernel sources of the captured revision (default: this tree)")
     b.add_argument("--profiles", default=os.path.join(ROOT, "profiles"))
     b.add_argument("csv", nargs="+")
+    e = sub.add_parser("sweep-dram", help="DRAM bytes over the sequence-length sweep from per-kernel captures")
+    e.add_argument("--d", type=int, required=True, choices=[64, 128])
+    e.add_argument("--causal", action="store_true")
+    e.add_argument("--revision", default=None)
+    e.add_argument("--profiles", default=os.path.join(ROOT, "profiles"))
+    e.add_argument("csv_dir")
     c = sub.add_parser("run", help="run one reduced case of the workload (the program ncu captures)")
-    c.add_argument("--workload", required=True, choices=sorted(bench.WORKLOADS))
+    c.add_argument("--workload", required=True, choices=sorted(ALL_WORKLOADS))
     c.add_argument("--div", type=int, default=1)
     c.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
@@ -304,6 +358,8 @@ def main():
                 texts.append(f.read())
         print(json.dumps({args.workload: write_dram(args.workload, args.div, texts, args.profiles, args.revision,
                                                     args.csrc)}))
+    elif args.cmd == "sweep-dram":
+        print(json.dumps(write_sweep_dram(args.d, args.causal, args.csv_dir, args.profiles, args.revision)))
     else:
         run_case(args.workload, args.div, args.reps)
 

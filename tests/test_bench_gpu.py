@@ -39,6 +39,8 @@ def test_bench_line_keeps_its_contract():
         assert key in d, key
     assert d["steps"] == steps and d["warmup"] == warmup and d["n_gpus"] == 1
     assert d["config"]["workload"] == WORKLOAD and d["higher_is_better"] is True
+    sha = d["config"]["inputs"]["sha256"]
+    assert set(sha) == {"q", "k", "v", "do"} and all(len(h) == 64 for h in sha.values())
     f, fb = bench.step_flops(bench.WORKLOADS[WORKLOAD])
     # value is the step's FLOPs over the timed step time
     assert abs(d["value"] - (f + fb) / (d["ms_per_step"] * 1e-3) / 1e12) <= 0.01 * d["value"] + 1e-3

@@ -127,3 +127,21 @@ def test_source_fingerprint_ignores_comments_and_layout_but_not_code():
     assert bench.code_text(src) == bench.code_text(same)
     assert bench.code_text(src) != bench.code_text(other)
     assert "scale" not in bench.code_text(src) and "twice" not in bench.code_text(src)
+
+
+def test_sweep_dram_summarises_every_point_of_one_head_size(tmp_path):
+    """Per-kernel captures of every causal d = 128 sweep point become one table, with the
+    ratio to the algorithmic bytes (the same at every N but the last) and row to row."""
+    from attn_inputs import sweep_workloads
+    pts = [w for w in sweep_workloads() if w.d == 128 and w.causal]
+    for i, w in enumerate(pts):
+        for k, name in (("fwd_pp", "attn::attn_fwd_pp_kernel<128>(x)"), ("bwd_prep", "attn::attn_bwd_prep_kernel<128>(x)"),
+                        ("bwd_kv", "attn::attn_bwd_kv_kernel<128>(x)"), ("bwd_q", "attn::attn_bwd_q_kernel<128>(x)")):
+            mb = str(100 + i)                                     # traffic that grows a little with N
+            text = "\n".join([HDR] + launch(0, name, "1,000", mb, "Mbyte", "10", "Mbyte"))
+            (tmp_path / f"dram_{w.name}_{k}.csv").write_text(text)
+    rows = bench_traffic.write_sweep_dram(128, True, str(tmp_path), str(tmp_path), revision="abc1234")
+    assert [r["N"] for r in rows] == [w.N for w in pts]
+    assert rows[0]["fwd"] == 110e6 and rows[0]["bwd"] == 3 * 110e6
+    md = (tmp_path / "dram_sweep_causal_d128.md").read_text()
+    assert "abc1234" in md and md.count("\n| ") == len(pts) + 1    # header + one row per point
