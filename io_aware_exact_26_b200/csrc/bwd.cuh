@@ -170,8 +170,13 @@ struct KvCfg {
   // TMEM columns: S^T (lane = key, column = query), P^T as bf16 over it (warpgroup g
   // packs its kCols queries into the first kCols / 2 of the columns it read, so it
   // overwrites only columns it has read); dP^T with dS^T as bf16 over it (same
-  // placement); dV and dK accumulators (D columns each).
-  static constexpr int kS = 0, kDP = 128, kDV = 256, kDK = 256 + D;
+  // placement); dV and dK accumulators (D columns each).  At d = 64 the accumulators
+  // leave 128 columns free for a second S^T buffer (step g uses buffer g % 2), so S^T of
+  // the next step is computed while the exponentials of this one run; at d = 128 there
+  // is one buffer and S^T(g+1) follows dV(g), which reads P^T(g) from it.
+  static constexpr int SB = (D == 64) ? 2 : 1;           // S^T buffers
+  static constexpr int kS = 0, kDP = 128, kDV = 256, kDK = 256 + D, kS1 = 256 + 2 * D;
+  static_assert(SB == 1 || kS1 + 128 <= 512, "second S^T buffer must fit in TMEM");
   static constexpr int kTmemCols = 512;
   static constexpr int kOffK = 0, kOffV = kTile;
   static constexpr int kOffQ = 2 * kTile;                // 2 stages
@@ -186,7 +191,7 @@ struct KvCfg {
 struct KvShared {
   uint64_t kv_full, kv_empty;
   uint64_t qdo_full[2], qdo_empty[2];
-  uint64_t s_full, dp_full;     // S^T / dP^T of the step in TMEM
+  uint64_t s_full[2], dp_full;  // S^T of the step (in buffer step % SB) / dP^T in TMEM
   uint64_t p_ready, ds_ready;   // P^T / dS^T (bf16) written back by both dS warpgroups
   uint64_t k_done;              // dK MMA of the step complete (the item's last one ends it)
   uint64_t acc_free;            // dV / dK of the previous item read out
@@ -261,7 +266,8 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
       mbar_init(&sh.qdo_full[i], 1);
       mbar_init(&sh.qdo_empty[i], 1);
     }
-    mbar_init(&sh.s_full, 1);
+    mbar_init(&sh.s_full[0], 1);
+    mbar_init(&sh.s_full[1], 1);
     mbar_init(&sh.dp_full, 1);
     mbar_init(&sh.p_ready, C::kDsWarps);
     mbar_init(&sh.ds_ready, C::kDsWarps);
@@ -332,10 +338,11 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
     }
   } else if (warp == C::kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    // Order per step g:  dV(g) S^T(g+1) dK(g) dP^T(g+1).  The exps of step g+1
-    // (phase A) run under dK(g) and dP^T(g+1); dS of step g (phase B) under dV(g)
-    // and S^T(g+1).  The whole warp follows the schedule (descriptor arithmetic
-    // stays warp-uniform); one lane, elected once, issues every MMA and commit.
+    // Order per step g:  dV(g) S^T(g+1) dK(g) dP^T(g+1) with one S^T buffer (d = 128),
+    // S^T(g+1) dV(g) dK(g) dP^T(g+1) with two (d = 64).  The exps of step g+1 (phase A)
+    // run under dK(g) and dP^T(g+1); dS of step g (phase B) under dV(g) and S^T(g+1).
+    // The whole warp follows the schedule (descriptor arithmetic stays warp-uniform);
+    // one lane, elected once, issues every MMA and commit.
     const bool leader = elect_one();
     constexpr uint32_t idST = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
     constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);      // dV, dK
@@ -348,10 +355,10 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
     };
     int gs = 0, it = 0;
     bool ok = true;
-    auto issue_st = [&](int g) -> bool {   // S^T(g) = K Q(g)^T
-      const int st = g & 1;
+    auto issue_st = [&](int g) -> bool {   // S^T(g) = K Q(g)^T into buffer g % SB
+      const int st = g & 1, sb = g % C::SB;
       if (!wait(&sh.qdo_full[st], (g >> 1) & 1)) return false;
-      // S^T(g) overwrites P^T(g-1): issued behind dV(g-1) by this thread, which the
+      // S^T(g) overwrites P^T(g - SB): issued behind dV(g - SB) by this thread, which the
       // tensor cores perform first (MMAs of one thread run in issue order).
       tc_fence_after();
       if (leader) {
@@ -359,9 +366,9 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = ((k >> 2) * C::kBox + (k & 3) * 32) >> 4;
-          umma_ss_lo(tmem + C::kS, k_lo + off, q_lo + off, hi, idST, k > 0);
+          umma_ss_lo(tmem + (sb ? C::kS1 : C::kS), k_lo + off, q_lo + off, hi, idST, k > 0);
         }
-        umma_commit(&sh.s_full);
+        umma_commit(&sh.s_full[sb]);
       }
       __syncwarp();
       return true;
@@ -395,6 +402,9 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
       ok = issue_st(gs) && issue_dp(gs);
       for (int u = 0; u < n_steps && ok; ++u, ++gs) {
         const int st = gs & 1;
+        // Two S^T buffers: S^T(g+1) goes first, into the buffer dV(g-1) has finished
+        // with, and runs under the exponentials of step g.
+        if (C::SB == 2 && u + 1 < n_steps && !issue_st(gs + 1)) { ok = false; break; }
         // dV += P^T dO  (A = P^T in TMEM, K = queries; B = dO MN-major)
         ok = wait(&sh.p_ready, gs & 1);
         if (ok && u == 0 && it >= 1) ok = wait(&sh.acc_free, (it - 1) & 1);
@@ -402,13 +412,14 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
         tc_fence_after();
         if (leader) {
           const uint32_t do_mn = do_mn0 + st * (C::kTile >> 4);
+          const uint32_t pcol = (gs % C::SB) ? C::kS1 : C::kS;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_ts_lo(tmem + C::kDV, tmem + C::kS + packed_col(k, C::kCols), do_mn + ((k * 2048) >> 4), hi,
+            umma_ts_lo(tmem + C::kDV, tmem + pcol + packed_col(k, C::kCols), do_mn + ((k * 2048) >> 4), hi,
                        idKV, !(u == 0 && k == 0));
         }
         __syncwarp();
-        if (u + 1 < n_steps && !issue_st(gs + 1)) { ok = false; break; }
+        if (C::SB == 1 && u + 1 < n_steps && !issue_st(gs + 1)) { ok = false; break; }
         // dK += dS^T Q  (A = dS^T in TMEM; B = Q MN-major)
         ok = wait(&sh.ds_ready, gs & 1);
         if (!ok) break;
@@ -468,15 +479,16 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
           const int lo = key - p.wr - qbase;
           const bool masked = !__all_sync(0xffffffffu, lo <= 0 && hi >= CW - 1);
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.qdo_full[st], (gs >> 1) & 1));
-          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full, gs & 1));
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[gs % C::SB], (gs / C::SB) & 1));
           if (!ok) break;
           tc_fence_after();
           // ---- phase A: P^T = exp2(S^T c - lse2); bf16 into TMEM, fp32 pairs kept for phase B
+          const uint32_t sbuf = (gs % C::SB) ? C::kS1 : C::kS;
           uint64_t pf2[CW / 2];
 #pragma unroll
           for (int q16 = 0; q16 < CW / 16; ++q16) {
             uint32_t sr[16];
-            tmem_ld16(lane_base + C::kS + CW * hb + q16 * 16, sr);
+            tmem_ld16(lane_base + sbuf + CW * hb + q16 * 16, sr);
             uint64_t nl[8];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -490,7 +502,7 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
             uint32_t pk[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2_2(pf2[q16 * 8 + k]);
-            tmem_st8(lane_base + C::kS + CW * hb + q16 * 8, pk);
+            tmem_st8(lane_base + sbuf + CW * hb + q16 * 8, pk);
           }
           tmem_wait_st();
           tc_fence_before();
