@@ -200,7 +200,7 @@ def online_fwd_head(qh, kh, vh, scale, causal, bounds, window=None):
             s = np.where(visible(rows, kh.shape[0], causal, window)[:, a:b], s, -np.inf)
         m_new = np.maximum(m, s.max(axis=1))
         live = np.isfinite(m_new)   # rows that have seen at least one unmasked key
-        alpha = np.where(live, np.exp(np.where(live, m - m_new, 0.0)), 1.0)
+        alpha = np.where(live, np.exp(np.where(live, m, 0.0) - np.where(live, m_new, 0.0)), 1.0)
         pt = np.where(live[:, None], np.exp(s - np.where(live, m_new, 0.0)[:, None]), 0.0)
         l = alpha * l + pt.sum(axis=1)
         acc = alpha[:, None] * acc + pt @ vh[a:b]
