@@ -546,9 +546,15 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
       tc_fence_after();
       constexpr int kHalf = C::kGroups / 2;
       const bool is_dv = hb < kHalf;
-      const bool live = key < p.N && in_range(bhkv, static_cast<long long>(p.B) * p.Hkv);
+      const bool head_live = in_range(bhkv, static_cast<long long>(p.B) * p.Hkv);
       const float mul = is_dv ? 1.f : p.scale;
-      __nv_bfloat16* dst = (is_dv ? p.dv : p.dk) + (static_cast<size_t>(bhkv) * p.N + key) * D;
+      // d = 128: rows of 256 bytes, stored whole after a 4-lane chunk exchange (lane 4g + i
+      // writes 16 bytes of keys row0 + t, t = 0..3), so each store instruction covers 64
+      // contiguous bytes of 8 keys instead of 16 bytes of 32 (measured: +5-10% backward at
+      // N = 1024-4096, +0.7% at N = 32768).  d = 64: each thread stores its own row (the
+      // exchange measured slower there).
+      const int row0 = j * 128 + (warp & 3) * 32 + (lane & ~3);
+      __nv_bfloat16* dst = (is_dv ? p.dv : p.dk) + static_cast<size_t>(bhkv) * p.N * D + (lane & 3) * 8;
       const uint32_t col = is_dv ? C::kDV : C::kDK;
 #pragma unroll 1
       for (int q4 = hb % kHalf; q4 < D / 32; q4 += kHalf) {
@@ -556,10 +562,26 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
         tmem_ld32(lane_base + col + q4 * 32, x);
         tmem_wait_ld();
         reg_fence(x);
-        if (live) {
+        if constexpr (D == 128) {
+          uint32_t ch[4][4];
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            reinterpret_cast<uint4*>(dst + q4 * 32)[k] = make_uint4(
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              ch[k][e] = pack_bf16x2(__uint_as_float(x[8 * k + 2 * e]) * mul, __uint_as_float(x[8 * k + 2 * e + 1]) * mul);
+          transpose_row_chunks<4>(ch, lane);
+          if (head_live) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              if (row0 + t < p.N)
+                *reinterpret_cast<uint4*>(dst + static_cast<size_t>(row0 + t) * D + q4 * 32) =
+                    make_uint4(ch[t][0], ch[t][1], ch[t][2], ch[t][3]);
+          }
+        } else if (head_live && key < p.N) {
+          uint4* own = reinterpret_cast<uint4*>((is_dv ? p.dv : p.dk) + (static_cast<size_t>(bhkv) * p.N + key) * D + q4 * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            own[k] = make_uint4(
                 pack_bf16x2(__uint_as_float(x[8 * k]) * mul, __uint_as_float(x[8 * k + 1]) * mul),
                 pack_bf16x2(__uint_as_float(x[8 * k + 2]) * mul, __uint_as_float(x[8 * k + 3]) * mul),
                 pack_bf16x2(__uint_as_float(x[8 * k + 4]) * mul, __uint_as_float(x[8 * k + 5]) * mul),
@@ -930,18 +952,37 @@ __global__ void __launch_bounds__(QCfg<D>::kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sh.q_done[glast & 1], (glast >> 1) & 1));
       if (!ok) break;
       tc_fence_after();
-      const bool live = qrow < p.N && in_range(bhq, static_cast<long long>(p.B) * p.Hq);
-      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bhq) * p.N + qrow) * D;
+      const bool head_live = in_range(bhq, static_cast<long long>(p.B) * p.Hq);
+      // rows stored as for dK and dV (exchanged among 4 lanes at d = 128)
+      const int row0 = i * 128 + (warp & 3) * 32 + (lane & ~3);
+      __nv_bfloat16* dst = p.dq + static_cast<size_t>(bhq) * p.N * D + (lane & 3) * 8;
 #pragma unroll 1
       for (int q4 = hb; q4 < D / 32; q4 += C::kGroups) {
         uint32_t x[32];
         tmem_ld32(lane_base + C::kDQ + q4 * 32, x);
         tmem_wait_ld();
         reg_fence(x);
-        if (live) {
+        if constexpr (D == 128) {
+          uint32_t ch[4][4];
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            reinterpret_cast<uint4*>(dst + q4 * 32)[k] = make_uint4(
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              ch[k][e] = pack_bf16x2(__uint_as_float(x[8 * k + 2 * e]) * p.scale,
+                                     __uint_as_float(x[8 * k + 2 * e + 1]) * p.scale);
+          transpose_row_chunks<4>(ch, lane);
+          if (head_live) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              if (row0 + t < p.N)
+                *reinterpret_cast<uint4*>(dst + static_cast<size_t>(row0 + t) * D + q4 * 32) =
+                    make_uint4(ch[t][0], ch[t][1], ch[t][2], ch[t][3]);
+          }
+        } else if (head_live && qrow < p.N) {
+          uint4* own = reinterpret_cast<uint4*>(p.dq + (static_cast<size_t>(bhq) * p.N + qrow) * D + q4 * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            own[k] = make_uint4(
                 pack_bf16x2(__uint_as_float(x[8 * k]) * p.scale, __uint_as_float(x[8 * k + 1]) * p.scale),
                 pack_bf16x2(__uint_as_float(x[8 * k + 2]) * p.scale, __uint_as_float(x[8 * k + 3]) * p.scale),
                 pack_bf16x2(__uint_as_float(x[8 * k + 4]) * p.scale, __uint_as_float(x[8 * k + 5]) * p.scale),

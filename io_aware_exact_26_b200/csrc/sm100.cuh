@@ -498,4 +498,32 @@ __device__ __forceinline__ uint32_t pack_bf16x2_2(uint64_t v) {
   return pack_bf16x2(lo, hi);
 }
 
+// Row-per-lane tiles to row-contiguous stores.  A thread that owns one row of a
+// tile holds NC 16-byte chunks of it; a warp storing chunk k of its 32 rows per
+// instruction touches 32 separate lines.  This exchanges chunks inside each group
+// of NC lanes (an NC x NC transpose in log2(NC) butterfly steps of shuffles), so
+// that afterwards lane NC*g + i holds chunk i of the group's rows NC*g + t in c[t]:
+// storing c[t] from every lane writes 32 / NC whole row segments of NC * 16 bytes.
+template <int NC>
+__device__ __forceinline__ void transpose_row_chunks(uint32_t (&c)[NC][4], int lane) {
+  static_assert(NC == 2 || NC == 4 || NC == 8, "NC must be 2, 4 or 8");
+#pragma unroll
+  for (int m = NC / 2; m >= 1; m >>= 1) {
+    const bool up = (lane & m) != 0;
+#pragma unroll
+    for (int lo = 0; lo < NC; ++lo) {
+      if (lo & m) continue;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        // the lower lane of a pair sends its upper chunk and takes the partner's lower one
+        const uint32_t r = __shfl_xor_sync(0xffffffffu, up ? c[lo][w] : c[lo | m][w], m);
+        if (up)
+          c[lo][w] = r;
+        else
+          c[lo | m][w] = r;
+      }
+    }
+  }
+}
+
 }  // namespace attn
