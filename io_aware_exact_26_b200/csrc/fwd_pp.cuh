@@ -66,8 +66,9 @@ struct PpCfg {
   // MUFU (16 ex2 per SM per clock).  At d = 64 a tile's two products take 512
   // tensor-core cycles (bf16; fewer with e4m3) against 1024 MUFU cycles for its
   // exponentials, and moving 2 pairs in 8 to the FMA pipe measured +8% to +21%
-  // (N = 1024 to 4096); at d = 128 the share measured no gain.
-  static constexpr int kFmaPairs = D == 64 ? 2 : 0;
+  // (N = 1024 to 4096).  At d = 128, once PV is issued in halves and the exponent
+  // pass is on the critical path, 1 pair in 8 measured +1.0% to +1.7% (2 or 3: less).
+  static constexpr int kFmaPairs = D == 64 ? 2 : 1;
   static constexpr int kTmemCols = 512;
   static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + DT;
   // Q buffers per team: two at d = 64, so the next unit's Q loads while the current
