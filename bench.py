@@ -542,6 +542,122 @@ def run_window(args):
         torch.cuda.empty_cache()
 
 
+# Peer copy bandwidth per direction per GPU measured on this machine's NVLink 5 (the
+# ring's exchange is one such copy per step and direction).
+PEER_COPY_GBS = 770.0
+RING_WORLDS = (2, 4, 8)
+
+
+def ring_step_bytes(w: Workload, world: int, layout: str):
+    """Bytes one rank sends per ring step: the K/V shard it holds (bf16), and in the
+    backward also that shard's fp32 dK/dV accumulators, which travel with it."""
+    from io_aware_exact_26_b200 import ring
+    m = len(ring.shard_chunks(0, world, layout))
+    rows = w.N // world                                   # rows per shard (m chunks of N / (m W))
+    kv = 2 * w.B * w.Hkv * rows * w.d * 2
+    return {"fwd": kv, "bwd": kv + 2 * w.B * w.Hkv * rows * w.d * 4, "chunks_per_shard": m}
+
+
+def run_ring(args):
+    """Sequence parallelism (ring of W ranks), its compute measured on one GPU: the W
+    ranks' chunk-pair partials, merges and accumulations (``ring.rank_chunk_pairs``, the
+    order ring_attention_fwd / _bwd take them) run one rank after another, each timed
+    with CUDA events; no exchange runs.  The link time is modelled from the bytes a rank
+    sends per step at the measured peer copy bandwidth.  One JSON line per W."""
+    import torch
+    import io_aware_exact_26_b200 as attn
+    from io_aware_exact_26_b200 import ring
+
+    w = WORKLOADS[args.workload]
+    peaks, peaks_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    x = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=w.seed, qk_std=w.qk_std, vo_std=w.vo_std,
+                    boost_frac=w.boost_frac, boost=w.boost, device=dev, with_grad=True)
+    o, lse = attn.attn_fwd(x["q"], x["k"], x["v"], causal=w.causal)   # the rows' global O and LSE
+    f_fwd, f_bwd = step_flops(w)
+    layout = "zigzag" if w.causal else "contiguous"
+    for world in RING_WORLDS:
+        m = len(ring.shard_chunks(0, world, layout))
+        nch = m * world
+        if w.N % (nch * 128):
+            continue
+        c = w.N // nch
+        ch = lambda t, a: t[:, :, a * c:(a + 1) * c].contiguous()
+        qc, kc, vc, doc = ([ch(x[t], a) for a in range(nch)] for t in ("q", "k", "v", "do"))
+        oc = [ch(o, a) for a in range(nch)]
+        lsec = [lse[:, :, a * c:(a + 1) * c].contiguous() for a in range(nch)]
+        shp, kshp = (w.B, w.Hq, c, w.d), (w.B, w.Hkv, c, w.d)
+        o_p = torch.empty(shp, dtype=torch.bfloat16, device=dev)
+        lse_p = torch.empty(shp[:3], dtype=torch.float32, device=dev)
+        o_acc = [torch.empty(shp, dtype=torch.float32, device=dev) for _ in range(m)]
+        lse_acc = [torch.empty(shp[:3], dtype=torch.float32, device=dev) for _ in range(m)]
+        out = [torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(m)]
+        dq_p, dk_p, dv_p = (torch.empty(s_, dtype=torch.bfloat16, device=dev) for s_ in (shp, kshp, kshp))
+        dq_acc = [torch.zeros(shp, dtype=torch.float32, device=dev) for _ in range(m)]
+        dkv_acc = [[torch.zeros(kshp, dtype=torch.float32, device=dev) for _ in range(2)] for _ in range(m)]
+        ws = torch.empty(attn.attn_bwd_workspace_size(w.B, w.Hq, w.Hkv, c, w.d, True), dtype=torch.uint8,
+                         device=dev)
+
+        def fwd_rank(pairs):
+            for _, i, a, j, b, kind in pairs:
+                attn.attn_fwd(qc[a], kc[b], vc[b], o_p, lse_p, causal=(kind == ring.CAUSAL), scale=w.scale)
+                attn.attn_merge(o_acc[i], lse_acc[i], o_p, lse_p, out[i])
+
+        def bwd_rank(pairs):
+            for _, i, a, j, b, kind in pairs:
+                attn.attn_bwd(qc[a], kc[b], vc[b], oc[a], lsec[a], doc[a], dq_p, dk_p, dv_p, scale=w.scale,
+                              causal=(kind == ring.CAUSAL), workspace=ws)
+                attn.attn_accumulate(dq_acc[i], dq_p)
+                attn.attn_accumulate(dkv_acc[j][0], dk_p)
+                attn.attn_accumulate(dkv_acc[j][1], dv_p)
+
+        sampler = ClockSampler(0)
+        sampler.start()
+        ms = {"fwd": [], "bwd": []}
+        for r in range(world):
+            pairs = ring.rank_chunk_pairs(r, world, w.causal, layout)
+            for kind, fn in (("fwd", fwd_rank), ("bwd", bwd_rank)):
+                times = []
+                for rep in range(args.warmup + args.sweep_reps):
+                    for t_ in lse_acc:
+                        t_.fill_(float("-inf"))                 # empty accumulators, before the timed region
+                    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a_.record(stream)
+                    fn(pairs)
+                    b_.record(stream)
+                    if rep >= args.warmup:
+                        times.append((a_, b_))
+                torch.cuda.synchronize()
+                ms[kind].append(statistics.median(a_.elapsed_time(b_) for a_, b_ in times))
+        clocks = sampler.stop()
+        if attn.attn_get_device_status() != 0:
+            raise SystemExit(f"device-side error in the ring run at W={world}")
+        sb = ring_step_bytes(w, world, layout)
+        line = {"ring": w.name, "ranks": world, "layout": layout, "chunk_rows": c, "reps": args.sweep_reps,
+                "warmup": args.warmup, "emulated": "the ranks' compute runs one rank after another on one GPU; "
+                "no exchange runs; the link time is modelled at the measured peer copy bandwidth",
+                "peer_copy_gbs": PEER_COPY_GBS, "peak": peak, "peak_source": f"{peaks_kind} bf16 dense (burst)"}
+        for kind, fl in (("fwd", f_fwd), ("bwd", f_bwd)):
+            worst = max(ms[kind])
+            link_ms = sb[kind] / (PEER_COPY_GBS * 1e9) * 1e3
+            step_ms = worst / world                               # compute per ring step (mean over steps)
+            modelled = max(worst, world * link_ms)
+            line[kind] = {"ms_per_rank": [round(v, 4) for v in ms[kind]], "ms_max_rank": round(worst, 4),
+                          "compute_tflops": round(fl / (worst * 1e-3) / 1e12, 1),
+                          "compute_tflops_per_gpu": round(fl / (worst * 1e-3) / 1e12 / world, 1),
+                          "frac_of_peak_per_gpu": round(fl / (worst * 1e-3) / 1e12 / world / peak, 4),
+                          "bytes_sent_per_step": sb[kind], "link_ms_per_step": round(link_ms, 4),
+                          "compute_ms_per_step": round(step_ms, 4),
+                          "modelled_tflops": round(fl / (modelled * 1e-3) / 1e12, 1)}
+        line["clocks"] = clocks
+        print(json.dumps(line), flush=True)
+        del qc, kc, vc, doc, oc, lsec, o_acc, lse_acc, out, dq_acc, dkv_acc, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -559,6 +675,8 @@ def main():
     ap.add_argument("--decode", action="store_true", help="time split-KV decoding, one line per decode workload")
     ap.add_argument("--fp8", action="store_true", help="time the fp8 forward next to the bf16 forward")
     ap.add_argument("--window", action="store_true", help="time local (sliding-window) attention, fwd and bwd")
+    ap.add_argument("--ring", action="store_true",
+                    help="sequence parallelism: each rank's compute of a W-rank ring, emulated on one GPU")
     ap.add_argument("--shard", action="store_true",
                     help="N > 1: split one job's (b, kv-head) units across the ranks (strong scaling) "
                          "instead of running N replicas")
@@ -576,6 +694,9 @@ def main():
         return
     if args.window:
         run_window(args)
+        return
+    if args.ring:
+        run_ring(args)
         return
 
     rank = int(os.environ.get("RANK", "0"))

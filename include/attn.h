@@ -169,6 +169,18 @@ int attn_decode_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal
 int attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                long long rows, int d, void* out, void* stream);
 
+/* Accumulation of a gradient contribution in fp32, for gradients summed over key or
+ * query blocks -- e.g. the backward over a ring of GPUs, where each step's attn_bwd
+ * returns one block pair's dQ, dK, dV (no counterpart on the pages; the plain sum of
+ * the per-block gradients that the recompute backward of page "attention 的显存线性化"
+ * §五 implies when the keys are split into blocks):
+ *   acc[i] += part[i] for 0 <= i < n.
+ *   acc : fp32 [n], updated in place;  part : bf16 [n].
+ * n is a multiple of 8 (>= 8); both pointers 16-byte aligned.  One kernel on `stream`.
+ * The sum is taken in fp32 in the order of the calls, so a fixed call order gives a
+ * bitwise reproducible result. */
+int attn_accumulate(float* acc, const void* part, long long n, void* stream);
+
 /* Backward without a caller-provided workspace (no counterpart on the pages; an
  * interface convenience).  Same arguments, layouts and results as attn_bwd, minus
  * `workspace`/`workspace_bytes`: the scratch lives in a fixed 64 MiB device array

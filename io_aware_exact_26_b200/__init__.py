@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     attn_decode_splits,
     attn_decode_workspace_size,
     attn_merge,
+    attn_accumulate,
     NOALLOC_SCRATCH_BYTES,
     attn_bwd_workspace_size,
     attn_fwd,

@@ -84,6 +84,8 @@ def load(path):
     L.attn_fwd_fp8.restype = i
     L.attn_merge.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, i, vp, vp]
     L.attn_merge.restype = i
+    L.attn_accumulate.argtypes = [vp, vp, ctypes.c_longlong, vp]
+    L.attn_accumulate.restype = i
     L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     L.attn_bwd_noalloc.restype = i
     L.attn_get_device_status.argtypes = [vp]
@@ -265,6 +267,19 @@ def attn_merge(o_acc, lse_acc, o_part, lse_part, out=None, *, stream=None):
     if st != ATTN_OK:
         raise AttnError(st, "attn_merge")
     return o_acc, lse_acc
+
+
+def attn_accumulate(acc, part, *, stream=None):
+    """acc += part in fp32, in place (acc fp32, part bf16, the same number of elements, a
+    multiple of 8); returns acc."""
+    _check(acc, "acc", torch.float32)
+    _check(part, "part")
+    if part.numel() != acc.numel():
+        raise ValueError("attn_accumulate: the accumulator and the part differ in size")
+    st = lib().attn_accumulate(_ptr(acc), _ptr(part), acc.numel(), _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_accumulate")
+    return acc
 
 
 def attn_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal=False) -> int:

@@ -554,6 +554,20 @@ int attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* ls
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
+int attn_accumulate(float* acc, const void* part, long long n, void* stream) {
+  if (!acc || !part || n < 8 || n % 8 != 0 || n >= (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(acc) || !aligned16(part)) return ATTN_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != 0) return ATTN_ERR_UNSUPPORTED;
+  const long long n8 = n / 8;
+  long long blocks = (n8 + 255) / 256;
+  const long long cap = static_cast<long long>(di->sms) * 8;
+  if (blocks > cap) blocks = cap;
+  attn::attn_accumulate_kernel<<<static_cast<int>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      acc, static_cast<const __nv_bfloat16*>(part), n8);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
                      float scale, int causal, void* stream) {

@@ -568,4 +568,28 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(float* __restrict__ o_a
   }
 }
 
+// acc[i] += part[i] for i < n (fp32 accumulator, bf16 part), 8 elements per thread and
+// iteration: one 16-byte load of the part, two of the accumulator.  n is a multiple of 8
+// and both pointers are 16-byte aligned (checked on the host).
+__global__ void __launch_bounds__(256) attn_accumulate_kernel(float* __restrict__ acc,
+                                                              const __nv_bfloat16* __restrict__ part, long long n8) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const uint4 pv = reinterpret_cast<const uint4*>(part)[i];
+    float4* a = reinterpret_cast<float4*>(acc) + 2 * i;
+    float4 lo = a[0], hi = a[1];
+    const uint32_t w[4] = {pv.x, pv.y, pv.z, pv.w};
+    float f[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __uint_as_float(w[k] << 16);             // bf16 -> fp32: the high half of the word
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+    lo.x += f[0]; lo.y += f[1]; lo.z += f[2]; lo.w += f[3];
+    hi.x += f[4]; hi.y += f[5]; hi.z += f[6]; hi.w += f[7];
+    a[0] = lo;
+    a[1] = hi;
+  }
+}
+
 }  // namespace attn

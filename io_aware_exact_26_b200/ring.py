@@ -84,6 +84,23 @@ def chunk_kind(a: int, b: int, causal: bool):
     return CAUSAL if a == b else SKIP
 
 
+def rank_chunk_pairs(rank: int, world: int, causal: bool, layout: str = "contiguous"):
+    """[(step, i, a, j, b, kind)]: at ring step ``step`` this rank's local chunk i (global
+    chunk a) against local chunk j (global chunk b) of the shard it then holds, skipped
+    pairs left out -- the pairs ``ring_attention_fwd`` and ``ring_attention_bwd`` compute,
+    in their order."""
+    out = []
+    mine = shard_chunks(rank, world, layout)
+    for step in range(world):
+        src = (rank - step) % world
+        for i, a in enumerate(mine):
+            for j, b in enumerate(shard_chunks(src, world, layout)):
+                kind = chunk_kind(a, b, causal)
+                if kind != SKIP:
+                    out.append((step, i, a, j, b, kind))
+    return out
+
+
 def shard_sequence(x, rank: int, world: int, layout: str = "contiguous", dim: int = 2):
     """This rank's local tensor of a full-sequence tensor ``x`` (sequence along ``dim``)."""
     chunks = shard_chunks(rank, world, layout)
@@ -150,18 +167,15 @@ def ring_attention_fwd(q, k, v, *, causal: bool, group=None, scale=None, partial
     cur = torch.stack((_chunked(k, m), _chunked(v, m))).contiguous()   # [2, m, B, Hkv, c, d]: one message
     nxt = torch.empty_like(cur)
     nxt_rank, prv_rank = _ring_peers(group, rank, world)
+    pairs = rank_chunk_pairs(rank, world, causal, layout)
     for step in range(world):
-        src = (rank - step) % world
         reqs = []
         if step + 1 < world:                        # post the exchange for the next step first
             ops = [dist.P2POp(dist.isend, cur, nxt_rank, group), dist.P2POp(dist.irecv, nxt, prv_rank, group)]
             reqs = dist.batch_isend_irecv(ops)
-        for i, a in enumerate(mine):
-            for j, b in enumerate(shard_chunks(src, world, layout)):
-                kind = chunk_kind(a, b, causal)
-                if kind != SKIP:
-                    o_p, lse_p = partial(qc[i], cur[0, j], cur[1, j], kind == CAUSAL, scale)
-                    merge(o_acc[i], lse_acc[i], o_p, lse_p)
+        for _, i, _, j, _, kind in (pr for pr in pairs if pr[0] == step):
+            o_p, lse_p = partial(qc[i], cur[0, j], cur[1, j], kind == CAUSAL, scale)
+            merge(o_acc[i], lse_acc[i], o_p, lse_p)
         for r in reqs:
             r.wait()
         if step + 1 < world:
@@ -174,8 +188,13 @@ def _cuda_partial_bwd(q, k, v, o, lse, do, causal, scale):
     return binding.attn_bwd(q, k, v, o, lse, do, scale=scale, causal=causal)
 
 
+def _cuda_accumulate(acc, part):
+    from . import binding
+    binding.attn_accumulate(acc, part)
+
+
 def ring_attention_bwd(q, k, v, o, lse, do, *, causal: bool, group=None, scale=None, partial=None,
-                       acc_dtype=torch.float32, layout: str = "contiguous"):
+                       accumulate=None, acc_dtype=torch.float32, layout: str = "contiguous"):
     """Gradients of this rank's shards, for attention over the whole ring's sequence.
 
     q, o, do: [B, Hq, n, d]; k, v: [B, Hkv, n, d] -- this rank's shard; lse: [B, Hq, n]
@@ -183,13 +202,16 @@ def ring_attention_bwd(q, k, v, o, lse, do, *, causal: bool, group=None, scale=N
     sequence (``ring_attention_fwd`` with the same layout; o in the dtype ``partial``
     takes).  Returns (dq, dk, dv) for this rank's shards in ``acc_dtype``.
     ``partial(q, k, v, o, lse, do, causal, scale) -> (dq, dk, dv)`` gives one chunk
-    pair's contribution; it defaults to the CUDA library's ``attn_bwd``.
+    pair's contribution and ``accumulate(acc, part)`` adds one into an accumulator in
+    place; they default to the CUDA library's ``attn_bwd`` and ``attn_accumulate``
+    (fp32 accumulators, ``acc_dtype`` torch.float32).
     """
     import torch.distributed as dist
 
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     partial = partial or _cuda_partial_bwd
+    accumulate = accumulate or _cuda_accumulate
     if scale is None:
         scale = q.shape[-1] ** -0.5
     mine = shard_chunks(rank, world, layout)
@@ -202,22 +224,17 @@ def ring_attention_bwd(q, k, v, o, lse, do, *, causal: bool, group=None, scale=N
     acc = torch.zeros(cur.shape, dtype=acc_dtype, device=q.device)      # its dK, dV so far
     acc_in = torch.empty_like(acc)
     nxt_rank, prv_rank = _ring_peers(group, rank, world)
+    pairs = rank_chunk_pairs(rank, world, causal, layout)
     for step in range(world):
-        src = (rank - step) % world
         reqs = []
         if step + 1 < world:                        # the next shard is in flight during the compute
             reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur, nxt_rank, group),
                                            dist.P2POp(dist.irecv, nxt, prv_rank, group)])
-        for i, a in enumerate(mine):
-            for j, b in enumerate(shard_chunks(src, world, layout)):
-                kind = chunk_kind(a, b, causal)
-                if kind == SKIP:
-                    continue
-                dq_p, dk_p, dv_p = partial(qc[i], cur[0, j], cur[1, j], oc[i], lsec[i], doc[i], kind == CAUSAL,
-                                           scale)
-                dq[i] += dq_p.to(acc_dtype)
-                acc[0, j] += dk_p.to(acc_dtype)
-                acc[1, j] += dv_p.to(acc_dtype)
+        for _, i, _, j, _, kind in (pr for pr in pairs if pr[0] == step):
+            dq_p, dk_p, dv_p = partial(qc[i], cur[0, j], cur[1, j], oc[i], lsec[i], doc[i], kind == CAUSAL, scale)
+            accumulate(dq[i], dq_p)
+            accumulate(acc[0, j], dk_p)
+            accumulate(acc[1, j], dv_p)
         # this shard's accumulators move on with it (the last hop brings them home)
         if world > 1:
             reqs += dist.batch_isend_irecv([dist.P2POp(dist.isend, acc, nxt_rank, group),

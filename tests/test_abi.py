@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
         ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_get_device_status",
          "attn_status_string", "attn_selftest_timeout", "attn_fwd_window", "attn_bwd_window", "attn_decode",
          "attn_decode_workspace_size", "attn_decode_splits", "attn_merge", "attn_fwd_fp8", "attn_checks_enabled",
-         "attn_selftest_bounds", "attn_selftest_sched"])
+         "attn_selftest_bounds", "attn_selftest_sched", "attn_accumulate"])
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -164,6 +164,16 @@ def test_merge_validates_before_any_launch(L):
     assert L.attn_merge(ctypes.c_void_p(0), FAKE, FAKE, FAKE, 10, 128, None, None) == -1
     assert L.attn_merge(FAKE, FAKE, ODD, FAKE, 10, 128, None, None) == -3
     assert L.attn_merge(FAKE, FAKE, FAKE, FAKE, 10, 128, ODD, None) == -3
+
+
+def test_accumulate_validates_before_any_launch(L):
+    L.attn_accumulate.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p]
+    assert L.attn_accumulate(ctypes.c_void_p(0), FAKE, 64, None) == -1      # null accumulator
+    assert L.attn_accumulate(FAKE, ctypes.c_void_p(0), 64, None) == -1      # null part
+    assert L.attn_accumulate(FAKE, FAKE, 0, None) == -1                     # empty
+    assert L.attn_accumulate(FAKE, FAKE, 100, None) == -1                   # not a multiple of 8
+    assert L.attn_accumulate(ODD, FAKE, 64, None) == -3
+    assert L.attn_accumulate(FAKE, ODD, 64, None) == -3
 
 
 def test_fp8_forward_validates_before_any_launch(L):

@@ -116,6 +116,10 @@ def _partial_bwd(q, k, v, o, lse, do, causal, scale):
     return dq, dk, dv
 
 
+def _accumulate(acc, part):
+    acc += part.to(acc.dtype)
+
+
 def _rank_bwd(rank, world, port, causal, shape, out_dir, layout="contiguous"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -128,8 +132,8 @@ def _rank_bwd(rank, world, port, causal, shape, out_dir, layout="contiguous"):
         o, lse = ring.ring_attention_fwd(shard(q), shard(k), shard(v), causal=causal, scale=0.4,
                                          partial=_partial, merge=_merge, acc_dtype=torch.float64, layout=layout)
         dq, dk, dv = ring.ring_attention_bwd(shard(q), shard(k), shard(v), o, lse, shard(do), causal=causal,
-                                             scale=0.4, partial=_partial_bwd, acc_dtype=torch.float64,
-                                             layout=layout)
+                                             scale=0.4, partial=_partial_bwd, accumulate=_accumulate,
+                                             acc_dtype=torch.float64, layout=layout)
         for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
             np.save(os.path.join(out_dir, f"{name}{rank}.npy"), t.numpy())
     finally:
@@ -155,3 +159,30 @@ def test_ring_backward_equals_gradients_over_the_whole_sequence(tmp_path, world,
             mine = ring.shard_sequence(torch.from_numpy(full), r, world, layout).numpy()
             np.testing.assert_allclose(np.load(tmp_path / f"{name}{r}.npy"), mine,
                                        rtol=1e-10, atol=1e-11, err_msg=f"{name} rank {r}")
+
+
+@pytest.mark.parametrize("world,causal,layout", [(2, True, "zigzag"), (4, True, "zigzag"), (8, True, "zigzag"),
+                                                 (3, True, "contiguous"), (4, False, "contiguous")])
+def test_rank_chunk_pairs_cover_every_visible_pair_once(world, causal, layout):
+    """Over all ranks the ring computes every (query chunk, key chunk) pair the mask leaves
+    visible exactly once, each at the step its key chunk is held, with the right kind."""
+    nch = world * len(ring.shard_chunks(0, world, layout))
+    seen = []
+    for r in range(world):
+        for step, i, a, j, b, kind in ring.rank_chunk_pairs(r, world, causal, layout):
+            assert ring.shard_chunks(r, world, layout)[i] == a
+            assert ring.shard_chunks((r - step) % world, world, layout)[j] == b
+            assert kind == (ring.CAUSAL if causal and a == b else ring.FULL)
+            seen.append((a, b))
+    want = [(a, b) for a in range(nch) for b in range(nch) if not causal or b <= a]
+    assert sorted(seen) == sorted(want)
+
+
+def test_ring_step_bytes_of_the_long_causal_workload():
+    import bench
+    w = bench.WORKLOADS["long_causal_b1_h32_n32768_d128"]
+    sb = bench.ring_step_bytes(w, 4, "zigzag")
+    rows = 32768 // 4
+    assert sb["chunks_per_shard"] == 2
+    assert sb["fwd"] == 2 * 32 * rows * 128 * 2                 # K and V of the shard, bf16
+    assert sb["bwd"] == sb["fwd"] + 2 * 32 * rows * 128 * 4     # plus its fp32 dK, dV accumulators

@@ -8,7 +8,7 @@ attn_merge, exactly as ``ring_attention_fwd`` does between its exchanges.  The
 merged result of every rank must match the fp64 oracle over the whole sequence.
 The backward is emulated the same way: every rank's query shard runs attn_bwd against
 each K/V shard in ring order with its rows' global O and LSE, its dQ and the shards'
-dK, dV summed in fp32 as ``ring_attention_bwd`` does, and all must match the oracle's
+dK, dV summed in fp32 by attn_accumulate as ``ring_attention_bwd`` does, and all must match the oracle's
 gradients over the whole sequence.  The exchange itself is tested on CPU ranks
 (tests/test_ring.py).
 """
@@ -55,6 +55,22 @@ def test_ring_decomposition_matches_oracle(attn, world, causal, d):
         check_o(f64(out), o_ref[:, :, r * n:(r + 1) * n], f"ring W={world} rank {r} O")
         check_lse(f64(lse_acc), lse_ref[:, :, r * n:(r + 1) * n], f"ring W={world} rank {r} LSE")
         assert np.abs(f64(o_acc) - o_ref[:, :, r * n:(r + 1) * n]).max() < 1e-2
+
+
+@pytest.mark.parametrize("n", [8, 1000, 131072 + 24])
+def test_accumulate_adds_bf16_into_fp32_exactly(attn, n):
+    """acc += part: bf16 to fp32 is exact, so the kernel's sum equals torch's fp32 add
+    bit for bit, and a run of calls equals the same run of torch adds."""
+    g = torch.Generator().manual_seed(n)
+    acc = torch.randn(n, generator=g).cuda()
+    parts = [torch.randn(n, generator=g).mul(10 ** k).to(torch.bfloat16).cuda() for k in range(-2, 3)]
+    want = acc.clone()
+    for part in parts:
+        attn.attn_accumulate(acc, part)
+        want += part.float()
+    torch.cuda.synchronize()
+    assert attn.attn_get_device_status() == 0
+    assert torch.equal(acc, want)
 
 
 def test_merge_into_an_empty_accumulator_copies_the_partial(attn):
@@ -110,9 +126,9 @@ def test_ring_backward_decomposition_matches_oracle(attn, world, causal, d, layo
                         continue
                     g = attn.attn_bwd(ch(q, a), ch(k, b), ch(v, b), o_ch[a], lse_ch[a], ch(do, a),
                                       causal=(kind == ring.CAUSAL))
-                    dq[a] += g[0].float()
-                    dkv[b][0] += g[1].float()
-                    dkv[b][1] += g[2].float()
+                    attn.attn_accumulate(dq[a], g[0])
+                    attn.attn_accumulate(dkv[b][0], g[1])
+                    attn.attn_accumulate(dkv[b][1], g[2])
     torch.cuda.synchronize()
     assert attn.attn_get_device_status() == 0
     for a in range(nchunks):
