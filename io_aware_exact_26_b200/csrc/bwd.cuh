@@ -192,7 +192,15 @@ struct KvShared {
   uint64_t kv_full, kv_empty;
   uint64_t qdo_full[2], qdo_empty[2];
   uint64_t s_full[2], dp_full;  // S^T of the step (in buffer step % SB) / dP^T in TMEM
-  uint64_t p_ready, ds_ready;   // P^T / dS^T (bf16) written back by both dS warpgroups
+  // P^T (bf16) written back by both dS warpgroups, one barrier per S^T buffer (step g
+  // uses p_ready[g % SB]).  With two buffers S^T(g+1) is ready before dV(g) is issued,
+  // so a fast warp can finish the exponentials of step g+1 before a slow one has
+  // arrived for step g; on a single barrier that early arrival would complete step g's
+  // phase with one of its warps' P^T columns still unwritten.  Per buffer, a warp's
+  // next arrival on the same barrier is two steps later, after S^T(g+2), which is
+  // issued behind dV(g).
+  uint64_t p_ready[2];
+  uint64_t ds_ready;            // dS^T (bf16) written back by both dS warpgroups
   uint64_t p_half;              // one S^T buffer: the first half of each warpgroup's P^T written
   uint64_t k_done;              // dK MMA of the step complete (the item's last one ends it)
   uint64_t acc_free;            // dV / dK of the previous item read out
@@ -270,7 +278,8 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
     mbar_init(&sh.s_full[0], 1);
     mbar_init(&sh.s_full[1], 1);
     mbar_init(&sh.dp_full, 1);
-    mbar_init(&sh.p_ready, C::kDsWarps);
+    mbar_init(&sh.p_ready[0], C::kDsWarps);
+    mbar_init(&sh.p_ready[1], C::kDsWarps);
     mbar_init(&sh.p_half, C::kDsWarps);
     mbar_init(&sh.ds_ready, C::kDsWarps);
     mbar_init(&sh.k_done, 1);
@@ -419,7 +428,7 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
           if (!ok) break;
 #pragma unroll 1
           for (int half = 0; half < 2 && ok; ++half) {
-            if (half == 1) ok = wait(&sh.p_ready, gs & 1);
+            if (half == 1) ok = wait(&sh.p_ready[gs % C::SB], (gs / C::SB) & 1);
             if (!ok) break;
             tc_fence_after();
             if (leader) {
@@ -435,7 +444,7 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
           }
           if (!ok) break;
         } else {
-          ok = wait(&sh.p_ready, gs & 1);
+          ok = wait(&sh.p_ready[gs % C::SB], (gs / C::SB) & 1);
           if (ok && u == 0 && it >= 1) ok = wait(&sh.acc_free, (it - 1) & 1);
           if (!ok) break;
           tc_fence_after();
@@ -544,7 +553,7 @@ __global__ void __launch_bounds__(KvCfg<D>::kThreads, 1)
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.p_ready);
+          if (lane == 0) mbar_arrive(&sh.p_ready[gs % C::SB]);
           // ---- phase B: dS^T = P^T (dP^T - D); bf16 into TMEM over dP^T
           ok = __all_sync(0xffffffffu, mbar_wait(&sh.dp_full, gs & 1));
           if (!ok) break;

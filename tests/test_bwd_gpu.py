@@ -64,6 +64,26 @@ def test_bwd_is_bitwise_deterministic(attn):
             assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("B,H,N,d,causal", [(4, 32, 4096, 64, True), (2, 8, 2048, 64, False),
+                                             (2, 8, 1000, 64, True), (1, 16, 4096, 128, True)])
+def test_bwd_is_bitwise_deterministic_across_memory_states(attn, B, H, N, d, causal):
+    """The same backward, repeated with fresh outputs and workspace after other device
+    memory was overwritten with noise, gives the same bits every time."""
+    x = make_inputs(B, H, H, N, d, seed=11)
+    ins, g1, scale = run_fwd_bwd(attn, x, d, causal)
+    q, k, v, do, o, lse = ins
+    for rep in range(3):
+        noise = torch.randn(64 << 20, device="cuda")           # 256 MB of other data in the allocator's pool
+        del noise
+        ws = torch.empty(attn.attn_bwd_workspace_size(B, H, H, N, d, causal), dtype=torch.uint8, device="cuda")
+        ws.random_()
+        g2 = attn.attn_bwd(q, k, v, o, lse, do, scale=scale, causal=causal, workspace=ws)
+        torch.cuda.synchronize()
+        assert attn.attn_get_device_status() == 0
+        for a, b, name in zip(g1, g2, ("dQ", "dK", "dV")):
+            assert torch.equal(a, b), (rep, name, (a.float() - b.float()).abs().max().item())
+
+
 def test_bwd_null_workspace_through_c_abi(attn):
     """workspace = NULL: the library allocates on the stream; same bits as a caller workspace."""
     import ctypes
