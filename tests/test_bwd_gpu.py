@@ -64,20 +64,32 @@ def test_bwd_is_bitwise_deterministic(attn):
             assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("B,H,N,d,causal", [(4, 32, 4096, 64, True), (2, 8, 2048, 64, False),
-                                             (2, 8, 1000, 64, True), (1, 16, 4096, 128, True)])
-def test_bwd_is_bitwise_deterministic_across_memory_states(attn, B, H, N, d, causal):
+@pytest.mark.parametrize("B,H,N,d,causal,window", [(4, 32, 4096, 64, True, None), (2, 8, 2048, 64, False, None),
+                                                    (2, 8, 1000, 64, True, None), (1, 16, 4096, 128, True, None),
+                                                    (1, 16, 8192, 64, False, (256, 256))])
+def test_bwd_is_bitwise_deterministic_across_memory_states(attn, B, H, N, d, causal, window):
     """The same backward, repeated with fresh outputs and workspace after other device
-    memory was overwritten with noise, gives the same bits every time."""
+    memory was overwritten with noise, gives the same bits every time (masked tiles make
+    the warps' times differ, which is where barrier races would show)."""
     x = make_inputs(B, H, H, N, d, seed=11)
-    ins, g1, scale = run_fwd_bwd(attn, x, d, causal)
-    q, k, v, do, o, lse = ins
+    if window is None:
+        ins, g1, scale = run_fwd_bwd(attn, x, d, causal)
+        q, k, v, do, o, lse = ins
+    else:
+        q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+        scale = d ** -0.5
+        o, lse = attn.attn_fwd_window(q, k, v, window=window)
+        g1 = attn.attn_bwd_window(q, k, v, o, lse, do, window=window)
     for rep in range(3):
         noise = torch.randn(64 << 20, device="cuda")           # 256 MB of other data in the allocator's pool
         del noise
-        ws = torch.empty(attn.attn_bwd_workspace_size(B, H, H, N, d, causal), dtype=torch.uint8, device="cuda")
+        ws = torch.empty(attn.attn_bwd_workspace_size(B, H, H, N, d, bool(causal)), dtype=torch.uint8,
+                         device="cuda")
         ws.random_()
-        g2 = attn.attn_bwd(q, k, v, o, lse, do, scale=scale, causal=causal, workspace=ws)
+        if window is None:
+            g2 = attn.attn_bwd(q, k, v, o, lse, do, scale=scale, causal=causal, workspace=ws)
+        else:
+            g2 = attn.attn_bwd_window(q, k, v, o, lse, do, window=window, workspace=ws)
         torch.cuda.synchronize()
         assert attn.attn_get_device_status() == 0
         for a, b, name in zip(g1, g2, ("dQ", "dK", "dV")):
