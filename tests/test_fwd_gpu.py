@@ -75,3 +75,22 @@ def test_fwd_is_deterministic(attn):
     o2, l2 = attn.attn_fwd(q, k, v, causal=True)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", [(4, 32, 32, 4096, 64, True), (4, 32, 8, 4096, 64, True),
+                                                 (2, 16, 16, 4096, 128, True), (2, 8, 8, 1000, 128, False)])
+def test_fwd_is_bitwise_deterministic_across_memory_states(attn, B, Hq, Hkv, N, d, causal):
+    """The forward repeated with fresh outputs after other device memory was overwritten
+    with noise gives the same bits every time.  The two softmax teams and the split PV
+    issue meet on barriers that the warps arrive on without waiting; masked diagonal
+    tiles make the warps' times differ, which is where a race between steps would show."""
+    x = make_inputs(B, Hq, Hkv, N, d, seed=13, with_grad=False)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o1, l1 = attn.attn_fwd(q, k, v, causal=causal)
+    for rep in range(3):
+        noise = torch.randn(64 << 20, device="cuda")           # 256 MB of other data in the allocator's pool
+        del noise
+        o2, l2 = attn.attn_fwd(q, k, v, causal=causal)
+        torch.cuda.synchronize()
+        assert attn.attn_get_device_status() == 0
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), rep
