@@ -542,8 +542,8 @@ def run_window(args):
         torch.cuda.empty_cache()
 
 
-# Peer copy bandwidth per direction per GPU measured on this machine's NVLink 5 (the
-# ring's exchange is one such copy per step and direction).
+# Peer-to-peer copy bandwidth per direction per GPU, measured between B200s over
+# NVLink 5 and NVSwitch (the ring's exchange is one such copy per step and direction).
 PEER_COPY_GBS = 770.0
 RING_WORLDS = (2, 4, 8)
 
