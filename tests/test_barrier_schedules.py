@@ -1,0 +1,169 @@
+"""The dK/dV kernel's barrier schedule, checked on a model under random interleavings.
+
+The kernel's warps meet on mbarriers: the MMA warp's commits complete a phase when the
+tensor cores finish, and the dS warps arrive on ``p_ready`` / ``ds_ready`` without
+waiting on them.  A wait asks for the phase of one parity, so it can only tell the
+current phase from the one before.  The model below replays the schedule of
+``attn_bwd_kv_kernel`` (csrc/bwd.cuh) step by step -- which MMA is issued after which
+wait, which buffer each product reads and writes, which barrier each warp arrives on --
+and explores random interleavings of the MMA warp, the tensor pipe (in-order completion)
+and the dS warps, checking that every product reads what the schedule says it reads
+(S^T(g), P^T(g) of every warp, dS^T(g)) and that no schedule deadlocks.
+
+Two S^T buffers with one shared ``p_ready`` barrier is the schedule that let dV(g)
+read a slow warp's P^T columns before it wrote them: the model finds that interleaving.
+The schedules the kernel uses (one buffer with the split dV issue at d = 128; two
+buffers with one ``p_ready`` per buffer at d = 64) pass.
+"""
+import random
+
+import pytest
+
+
+class Barrier:
+    """An mbarrier: ``count`` arrivals complete a phase; a parity wait passes once the
+    phase of that parity is the last completed one."""
+
+    def __init__(self, count):
+        self.count, self.pending, self.completed = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        if self.pending == 0:
+            self.completed += 1
+            self.pending = self.count
+
+    def passed(self, parity):
+        return (self.completed & 1) != parity
+
+
+class Violation(Exception):
+    pass
+
+
+def run(steps, warps, two_buffers, p_ready_per_buffer, split_dv, seed, s_early=None):
+    """One random interleaving.  ``s_early``: issue S^T(g+1) before dV(g) (the default
+    with two buffers) rather than behind it."""
+    s_early = two_buffers if s_early is None else s_early
+    rnd = random.Random(seed)
+    nb = 2 if two_buffers else 1
+    bars = {"s_full": [Barrier(1) for _ in range(nb)], "dp_full": Barrier(1), "ds_ready": Barrier(warps),
+            "p_ready": [Barrier(warps) for _ in range(2 if p_ready_per_buffer else 1)], "p_half": Barrier(warps)}
+    sbuf = [[None] * warps for _ in range(nb)]     # per buffer, per warp's columns: ("S"|"P", step)
+    dpbuf = [None] * warps                          # per warp's columns: ("dP"|"dS", step)
+    pipe = []                                       # issued products, performed in order
+
+    def p_bar(g):
+        return bars["p_ready"][g % nb if p_ready_per_buffer else 0]
+
+    def p_par(g):
+        return (g // nb if p_ready_per_buffer else g) & 1
+
+    def perform(op):
+        kind, g = op[0], op[1]
+        if kind == "S":
+            for w in range(warps):
+                sbuf[g % nb][w] = ("S", g)
+            bars["s_full"][g % nb].arrive()
+        elif kind == "dP":
+            for w in range(warps):
+                dpbuf[w] = ("dP", g)
+            bars["dp_full"].arrive()
+        elif kind == "dV":                          # reads the half (or all) of P^T(g) it was issued for
+            for w in range(warps):
+                if sbuf[g % nb][w] != ("P", g):
+                    raise Violation(f"dV({g}) read warp {w}'s columns holding {sbuf[g % nb][w]}")
+        elif kind == "dK":
+            for w in range(warps):
+                if dpbuf[w] != ("dS", g):
+                    raise Violation(f"dK({g}) read warp {w}'s columns holding {dpbuf[w]}")
+
+    def mma():                                      # the MMA warp's program
+        yield ("issue", ("S", 0))
+        yield ("issue", ("dP", 0))
+        for g in range(steps):
+            if s_early and g + 1 < steps:
+                yield ("issue", ("S", g + 1))
+            if split_dv:
+                yield ("wait", bars["p_half"], g & 1)
+                yield ("issue", ("dVhalf", g))
+            yield ("wait", p_bar(g), p_par(g))
+            yield ("issue", ("dV", g))
+            if not s_early and g + 1 < steps:
+                yield ("issue", ("S", g + 1))
+            yield ("wait", bars["ds_ready"], g & 1)
+            yield ("issue", ("dK", g))
+            if g + 1 < steps:
+                yield ("issue", ("dP", g + 1))
+
+    def ds_warp(w):                                 # one dS warp's program
+        for g in range(steps):
+            yield ("wait", bars["s_full"][g % nb], (g // nb) & 1)
+            yield ("check", lambda g=g: sbuf[g % nb][w] == ("S", g), f"warp {w} phase A({g}) read S^T")
+            yield ("do", lambda g=g: sbuf[g % nb].__setitem__(w, ("P", g)))
+            if split_dv:
+                yield ("arrive", bars["p_half"])
+            yield ("arrive", p_bar(g))
+            yield ("wait", bars["dp_full"], g & 1)
+            yield ("check", lambda g=g: dpbuf[w] == ("dP", g), f"warp {w} phase B({g}) read dP^T")
+            yield ("do", lambda g=g: dpbuf.__setitem__(w, ("dS", g)))
+            yield ("arrive", bars["ds_ready"])
+
+    agents = {"mma": mma(), **{f"w{w}": ds_warp(w) for w in range(warps)}}
+    nxt = {name: next(gen) for name, gen in agents.items()}
+    while nxt or pipe:
+        ready = [n for n, op in nxt.items() if op[0] != "wait" or op[1].passed(op[2])]
+        choices = ready + (["pipe"] if pipe else [])
+        if not choices:
+            raise Violation("deadlock")
+        who = rnd.choice(choices)
+        if who == "pipe":
+            op = pipe.pop(0)
+            if op[0] != "dVhalf":                   # the first half reads what p_half guarantees
+                perform(op)
+            continue
+        op = nxt[who]
+        if op[0] == "issue":
+            pipe.append(op[1])
+        elif op[0] == "arrive":
+            op[1].arrive()
+        elif op[0] == "check" and not op[1]():
+            raise Violation(op[2])
+        elif op[0] == "do":
+            op[1]()
+        try:
+            nxt[who] = next(agents[who])
+        except StopIteration:
+            del nxt[who]
+
+
+def explore(seeds=400, **kw):
+    for seed in range(seeds):
+        try:
+            run(seed=seed, **kw)
+        except Violation as e:
+            return str(e)
+    return None
+
+
+def test_two_buffers_with_one_shared_p_ready_lets_dv_read_unwritten_columns():
+    found = explore(steps=6, warps=4, two_buffers=True, p_ready_per_buffer=False, split_dv=False)
+    assert found is not None and found.startswith("dV(")
+
+
+def test_one_buffer_with_s_issued_before_dv_overwrites_p():
+    """The model also catches the ordering mistake the in-order issue rule prevents."""
+    found = explore(steps=4, warps=2, two_buffers=False, p_ready_per_buffer=True, split_dv=False, s_early=True)
+    assert found is not None
+
+
+@pytest.mark.parametrize("steps", [1, 2, 7])
+def test_two_buffers_with_a_p_ready_per_buffer_is_safe(steps):
+    """The d = 64 schedule of the kernel."""
+    assert explore(steps=steps, warps=4, two_buffers=True, p_ready_per_buffer=True, split_dv=False) is None
+
+
+@pytest.mark.parametrize("steps", [1, 2, 7])
+def test_one_buffer_with_the_split_dv_issue_is_safe(steps):
+    """The d = 128 schedule of the kernel (p_ready per buffer, one buffer: one barrier)."""
+    assert explore(steps=steps, warps=4, two_buffers=False, p_ready_per_buffer=True, split_dv=True) is None
