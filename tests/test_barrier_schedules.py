@@ -1,4 +1,5 @@
-"""The dK/dV kernel's barrier schedule, checked on a model under random interleavings.
+"""The barrier schedules of the dK/dV kernel and the forward, checked on a model under
+random interleavings.
 
 The kernel's warps meet on mbarriers: the MMA warp's commits complete a phase when the
 tensor cores finish, and the dS warps arrive on ``p_ready`` / ``ds_ready`` without
@@ -13,7 +14,8 @@ and the dS warps, checking that every product reads what the schedule says it re
 Two S^T buffers with one shared ``p_ready`` barrier is the schedule that let dV(g)
 read a slow warp's P^T columns before it wrote them: the model finds that interleaving.
 The schedules the kernel uses (one buffer with the split dV issue at d = 128; two
-buffers with one ``p_ready`` per buffer at d = 64) pass.
+buffers with one ``p_ready`` per buffer at d = 64) pass, and so does the forward's
+(two teams on one MMA warp, PV in two halves, S(j+1) behind PV(j)).
 """
 import random
 
@@ -167,3 +169,104 @@ def test_two_buffers_with_a_p_ready_per_buffer_is_safe(steps):
 def test_one_buffer_with_the_split_dv_issue_is_safe(steps):
     """The d = 128 schedule of the kernel (p_ready per buffer, one buffer: one barrier)."""
     assert explore(steps=steps, warps=4, two_buffers=False, p_ready_per_buffer=True, split_dv=True) is None
+
+
+def run_forward(steps, warps, split_pv, seed, s_before_pv=False):
+    """One random interleaving of the forward's schedule (fwd_pp.cuh): two teams, each
+    with its S/P buffer in TMEM, served by one MMA warp in the order PV_A(j), S_A(j+1),
+    PV_B(j), S_B(j+1); a team's warps post partial maxima (arrive and wait on xbar, one
+    barrier per step parity), write P in two halves (p_half after the first) and arrive
+    on p_ready.  ``s_before_pv`` issues S_X(j+1) ahead of PV_X(j) (a mistake)."""
+    rnd = random.Random(seed)
+    teams = (0, 1)
+    bars = {x: {"s_full": Barrier(1), "p_half": Barrier(warps), "p_ready": Barrier(warps),
+                "xbar": [Barrier(warps), Barrier(warps)]} for x in teams}
+    buf = {x: [[None, None] for _ in range(warps)] for x in teams}   # [warp][half] of P, or S
+    pipe = []
+
+    def perform(op):
+        kind, x, j, half = op
+        if kind == "S":
+            for w in range(warps):
+                buf[x][w] = [("S", j), ("S", j)]
+            bars[x]["s_full"].arrive()
+        else:                                        # PV half reads P(j) of every warp
+            for w in range(warps):
+                for h in ((half,) if half is not None else (0, 1)):
+                    if buf[x][w][h] != ("P", j):
+                        raise Violation(f"PV_{x}({j}) half {h} read warp {w}'s {buf[x][w][h]}")
+
+    def mma():
+        for x in teams:
+            yield ("issue", ("S", x, 0, None))
+        for j in range(steps):
+            for x in teams:
+                if s_before_pv and j + 1 < steps:
+                    yield ("issue", ("S", x, j + 1, None))
+                if split_pv:
+                    yield ("wait", bars[x]["p_half"], j & 1)
+                    yield ("issue", ("PV", x, j, 0))
+                    yield ("wait", bars[x]["p_ready"], j & 1)
+                    yield ("issue", ("PV", x, j, 1))
+                else:
+                    yield ("wait", bars[x]["p_ready"], j & 1)
+                    yield ("issue", ("PV", x, j, None))
+                if not s_before_pv and j + 1 < steps:
+                    yield ("issue", ("S", x, j + 1, None))
+
+    def warp(x, w):
+        for j in range(steps):
+            yield ("wait", bars[x]["s_full"], j & 1)
+            yield ("check", lambda j=j: buf[x][w] == [("S", j), ("S", j)], f"team {x} warp {w} read S({j})")
+            xb = bars[x]["xbar"][j & 1]
+            yield ("arrive", xb)
+            yield ("wait", xb, (j >> 1) & 1)
+            for h in (0, 1):
+                yield ("do", lambda h=h, j=j: buf[x][w].__setitem__(h, ("P", j)))
+                if h == 0 and split_pv:
+                    yield ("arrive", bars[x]["p_half"])
+            yield ("arrive", bars[x]["p_ready"])
+
+    agents = {"mma": mma(), **{f"t{x}w{w}": warp(x, w) for x in teams for w in range(warps)}}
+    nxt = {name: next(gen) for name, gen in agents.items()}
+    while nxt or pipe:
+        ready = [n for n, op in nxt.items() if op[0] != "wait" or op[1].passed(op[2])]
+        choices = ready + (["pipe"] if pipe else [])
+        if not choices:
+            raise Violation("deadlock")
+        who = rnd.choice(choices)
+        if who == "pipe":
+            perform(pipe.pop(0))
+            continue
+        op = nxt[who]
+        if op[0] == "issue":
+            pipe.append(op[1])
+        elif op[0] == "arrive":
+            op[1].arrive()
+        elif op[0] == "check" and not op[1]():
+            raise Violation(op[2])
+        elif op[0] == "do":
+            op[1]()
+        try:
+            nxt[who] = next(agents[who])
+        except StopIteration:
+            del nxt[who]
+
+
+def explore_forward(seeds=300, **kw):
+    for seed in range(seeds):
+        try:
+            run_forward(seed=seed, **kw)
+        except Violation as e:
+            return str(e)
+    return None
+
+
+@pytest.mark.parametrize("split_pv", [False, True])
+def test_forward_schedule_is_safe(split_pv):
+    """The forward's schedule, with PV issued whole or in the two halves the kernel uses."""
+    assert explore_forward(steps=5, warps=4, split_pv=split_pv) is None
+
+
+def test_forward_with_s_ahead_of_pv_overwrites_p():
+    assert explore_forward(steps=4, warps=2, split_pv=True, s_before_pv=True) is not None
