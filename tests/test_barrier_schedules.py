@@ -270,3 +270,119 @@ def test_forward_schedule_is_safe(split_pv):
 
 def test_forward_with_s_ahead_of_pv_overwrites_p():
     assert explore_forward(steps=4, warps=2, split_pv=True, s_before_pv=True) is not None
+
+
+def run_dq(steps, warps, seed, dp_early=False, dp_free_wait=True):
+    """One random interleaving of the dQ kernel's schedule: S(j+1) into the other of two
+    buffers before dQ(j); the dS warps read S(j) (phase A), then dP(j), arrive on
+    dp_free, write dS(j) over S(j) and arrive on ds_ready; dQ(j) reads dS(j); dP(j+1)
+    waits for dp_free(j).  ``dp_early`` issues dP(j+1) ahead of the wait for ds_ready(j)
+    (a variant that was measured); ``dp_free_wait`` False drops the dp_free wait."""
+    rnd = random.Random(seed)
+    bars = {"s_full": [Barrier(1), Barrier(1)], "dp_full": Barrier(1), "dp_free": Barrier(warps),
+            "ds_ready": Barrier(warps)}
+    sbuf = [[None] * warps for _ in range(2)]
+    dpbuf = [None] * warps
+    pipe = []
+
+    def perform(op):
+        kind, j = op
+        if kind == "S":
+            for w in range(warps):
+                sbuf[j % 2][w] = ("S", j)
+            bars["s_full"][j % 2].arrive()
+        elif kind == "dP":
+            for w in range(warps):
+                dpbuf[w] = ("dP", j)
+            bars["dp_full"].arrive()
+        else:
+            for w in range(warps):
+                if sbuf[j % 2][w] != ("dS", j):
+                    raise Violation(f"dQ({j}) read warp {w}'s {sbuf[j % 2][w]}")
+
+    def mma():
+        yield ("issue", ("S", 0))
+        yield ("issue", ("dP", 0))
+        def dp_next(j):
+            if dp_free_wait:
+                yield ("wait", bars["dp_free"], j & 1)
+            yield ("issue", ("dP", j + 1))
+
+        for j in range(steps):
+            if j + 1 < steps:
+                yield ("issue", ("S", j + 1))
+            if dp_early and j + 1 < steps:
+                yield from dp_next(j)
+            yield ("wait", bars["ds_ready"], j & 1)
+            yield ("issue", ("dQ", j))
+            if not dp_early and j + 1 < steps:
+                yield from dp_next(j)
+
+    def warp(w):
+        for j in range(steps):
+            yield ("wait", bars["s_full"][j % 2], (j >> 1) & 1)
+            yield ("check", lambda j=j: sbuf[j % 2][w] == ("S", j), f"warp {w} read S({j})")
+            yield ("wait", bars["dp_full"], j & 1)
+            yield ("check", lambda j=j: dpbuf[w] == ("dP", j), f"warp {w} read dP({j})")
+            yield ("arrive", bars["dp_free"])
+            yield ("do", lambda j=j: sbuf[j % 2].__setitem__(w, ("dS", j)))
+            yield ("arrive", bars["ds_ready"])
+
+    agents = {"mma": mma(), **{f"w{w}": warp(w) for w in range(warps)}}
+    nxt = {name: next(gen) for name, gen in agents.items()}
+    while nxt or pipe:
+        ready = [n for n, op in nxt.items() if op[0] != "wait" or op[1].passed(op[2])]
+        choices = ready + (["pipe"] if pipe else [])
+        if not choices:
+            raise Violation("deadlock")
+        who = rnd.choice(choices)
+        if who == "pipe":
+            perform(pipe.pop(0))
+            continue
+        op = nxt[who]
+        if op[0] == "issue":
+            pipe.append(op[1])
+        elif op[0] == "arrive":
+            op[1].arrive()
+        elif op[0] == "check" and not op[1]():
+            raise Violation(op[2])
+        elif op[0] == "do":
+            op[1]()
+        try:
+            nxt[who] = next(agents[who])
+        except StopIteration:
+            del nxt[who]
+
+
+def first_dq_violation(**kw):
+    for seed in range(300):
+        try:
+            run_dq(seed=seed, **kw)
+        except Violation as e:
+            return str(e)
+    return None
+
+
+def test_dq_schedule_is_safe():
+    """The kernel's order: dP(j+1) behind dQ(j), which waited for every warp's dS(j)."""
+    assert first_dq_violation(steps=6, warps=4) is None
+
+
+def test_dq_with_dp_ahead_of_dq_lets_ds_ready_complete_early():
+    """dP(j+1) ahead of dQ(j) (a measured variant, not kept) lets a fast warp reach
+    step j+1's dS and arrive on ds_ready before a slow warp's step-j arrival, even with
+    the dp_free wait: the same run-ahead as the old d = 64 dK/dV schedule.  Depending on
+    the interleaving dQ(j) reads unwritten dS, or the MMA warp's parity wait sees the
+    barrier two phases on and waits for good."""
+    outcomes = set()
+    for seed in range(300):
+        try:
+            run_dq(steps=4, warps=4, seed=seed, dp_early=True)
+            outcomes.add("ok")
+        except Violation as e:
+            outcomes.add("deadlock" if str(e) == "deadlock" else str(e).split("(")[0])
+    assert "dQ" in outcomes                     # a read of unwritten dS is reachable
+
+
+def test_dq_with_dp_ahead_and_no_dp_free_wait_overwrites_dp():
+    assert first_dq_violation(steps=4, warps=2, dp_early=True, dp_free_wait=False) is not None
